@@ -1,0 +1,225 @@
+"""ctypes front end of the fp64 C oracle (``kvring_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the benchmark's
+CPU-baseline leg use it; the product never does.  It imports nothing from the product
+package; inputs arrive as numpy arrays from the seeded generators.
+
+The arithmetic lives in the C file; this module only owns the host arrays of an oracle
+ring and marshals pointers.  See the C file's header for the definitions it follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kvring_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+
+# gcc flags: no contraction into FMA, no fast-math, so every binary64 op is IEEE.
+GCC_FLAGS = ["-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
+             "-std=c11", "-Wall", "-Wno-unknown-pragmas"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/liboracle.so`` (skipped when up to date)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    subprocess.check_call(["gcc", *GCC_FLAGS, "-o", tmp, _SRC, "-lm"])
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        L = _lib
+        P = ctypes.c_void_p
+        L.orc_e4m3_decode.restype = ctypes.c_double
+        L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_encode.restype = ctypes.c_uint8
+        L.orc_e4m3_encode.argtypes = [ctypes.c_float]
+        L.orc_bf16_round.restype = ctypes.c_float
+        L.orc_bf16_round.argtypes = [ctypes.c_float]
+        L.orc_rope_cs.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_double, P, P]
+        L.orc_rope_apply.argtypes = [P, ctypes.c_int, P, P, P]
+        L.orc_rope_apply_f64.argtypes = [P, ctypes.c_int, ctypes.c_int64, ctypes.c_double, P]
+        L.orc_quant_row.argtypes = [P, ctypes.c_int, P, P]
+        L.orc_slot_of_age.restype = ctypes.c_int64
+        L.orc_slot_of_age.argtypes = [P, ctypes.c_int64]
+        L.orc_ring_commit.argtypes = [P]
+        L.orc_ring_write.argtypes = [P, P, P, ctypes.c_int, ctypes.c_int]
+        L.orc_ring_delta_rotate.argtypes = [P, ctypes.c_int64]
+        L.orc_chunk_attention.argtypes = [
+            P, P, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_float, ctypes.c_int, P,
+            ctypes.c_int, P, P]
+        L.orc_e4m3_encode_n.argtypes = [P, ctypes.c_int64, P]
+        L.orc_e4m3_decode_n.argtypes = [P, ctypes.c_int64, P]
+        L.orc_bf16_round_n.argtypes = [P, ctypes.c_int64, P]
+        L.orc_quant_rows.argtypes = [P, ctypes.c_int64, ctypes.c_int, P, P]
+        L.orc_struct_size.restype = ctypes.c_int
+    return _lib
+
+
+def _p(a: np.ndarray) -> ctypes.c_void_p:
+    assert a.flags["C_CONTIGUOUS"]
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def _f32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+
+
+# ------------------------------------------------------------------ scalar/array helpers
+
+def e4m3_encode(v) -> np.ndarray:
+    v = _f32(v)
+    out = np.empty(v.shape, np.uint8)
+    lib().orc_e4m3_encode_n(_p(v), v.size, _p(out))
+    return out
+
+
+def e4m3_decode(c) -> np.ndarray:
+    c = np.ascontiguousarray(np.asarray(c, dtype=np.uint8))
+    out = np.empty(c.shape, np.float64)
+    lib().orc_e4m3_decode_n(_p(c), c.size, _p(out))
+    return out
+
+
+def bf16_round(v) -> np.ndarray:
+    v = _f32(v)
+    out = np.empty(v.shape, np.float32)
+    lib().orc_bf16_round_n(_p(v), v.size, _p(out))
+    return out
+
+
+def rope_cs(p: int, D: int, base: float = 10000.0):
+    c = np.empty(D // 2, np.float32)
+    s = np.empty(D // 2, np.float32)
+    lib().orc_rope_cs(int(p), D, float(base), _p(c), _p(s))
+    return c, s
+
+
+def rope_apply(x, p: int, base: float = 10000.0) -> np.ndarray:
+    """binary32 RoPE of one row at position p."""
+    x = _f32(x)
+    c, s = rope_cs(p, x.shape[-1], base)
+    y = np.empty_like(x)
+    lib().orc_rope_apply(_p(x), x.shape[-1], _p(c), _p(s), _p(y))
+    return y
+
+
+def rope_apply_f64(x, p: int, base: float = 10000.0) -> np.ndarray:
+    x = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    y = np.empty_like(x)
+    lib().orc_rope_apply_f64(_p(x), x.shape[-1], int(p), float(base), _p(y))
+    return y
+
+
+def quant_rows(y) -> tuple[np.ndarray, np.ndarray]:
+    """Per-row e4m3 quantisation of a [rows][D] binary32 array -> (codes, scales)."""
+    y = _f32(y)
+    rows, D = y.reshape(-1, y.shape[-1]).shape
+    codes = np.empty((rows, D), np.uint8)
+    scales = np.empty(rows, np.float32)
+    lib().orc_quant_rows(_p(y), rows, D, _p(codes), _p(scales))
+    return codes.reshape(y.shape), scales.reshape(y.shape[:-1])
+
+
+# ------------------------------------------------------------------ ring
+
+class _RingStruct(ctypes.Structure):
+    _fields_ = [("C", ctypes.c_int32), ("H", ctypes.c_int32), ("D", ctypes.c_int32),
+                ("_pad", ctypes.c_int32), ("base", ctypes.c_double),
+                ("write_slot", ctypes.c_int64), ("live", ctypes.c_int64),
+                ("pending", ctypes.c_int64), ("next_pos", ctypes.c_int64),
+                ("kc", ctypes.c_void_p), ("vc", ctypes.c_void_p), ("ks", ctypes.c_void_p),
+                ("vs", ctypes.c_void_p), ("slot_pos", ctypes.c_void_p)]
+
+
+class OracleRing:
+    """Host-side oracle ring: codes [H][C][D] u8, scales [H][C] f32, slot_pos [C] i32."""
+
+    def __init__(self, capacity: int, n_heads: int, head_dim: int, base: float = 10000.0,
+                 next_pos: int = 0):
+        assert head_dim % 2 == 0 and head_dim <= 512
+        self.C, self.H, self.D = capacity, n_heads, head_dim
+        self.kc = np.zeros((n_heads, capacity, head_dim), np.uint8)
+        self.vc = np.zeros((n_heads, capacity, head_dim), np.uint8)
+        self.ks = np.zeros((n_heads, capacity), np.float32)
+        self.vs = np.zeros((n_heads, capacity), np.float32)
+        self.slot_pos = np.zeros(capacity, np.int32)
+        self._s = _RingStruct(capacity, n_heads, head_dim, 0, float(base), 0, 0, 0,
+                              int(next_pos), self.kc.ctypes.data, self.vc.ctypes.data,
+                              self.ks.ctypes.data, self.vs.ctypes.data,
+                              self.slot_pos.ctypes.data)
+        assert lib().orc_struct_size() == ctypes.sizeof(_RingStruct)
+
+    # state integers
+    @property
+    def write_slot(self): return self._s.write_slot
+
+    @property
+    def live(self): return self._s.live
+
+    @property
+    def pending(self): return self._s.pending
+
+    @property
+    def next_pos(self): return self._s.next_pos
+
+    def state(self) -> tuple[int, int, int, int]:
+        return (self._s.write_slot, self._s.live, self._s.pending, self._s.next_pos)
+
+    def _ptr(self):
+        return ctypes.byref(self._s)
+
+    def slot_of_age(self, age: int) -> int:
+        return lib().orc_slot_of_age(self._ptr(), int(age))
+
+    def write(self, k, v, commit: bool = False) -> None:
+        k, v = _f32(k), _f32(v)
+        n = k.shape[0]
+        assert k.shape == (n, self.H, self.D) and v.shape == k.shape and 0 < n <= self.C
+        lib().orc_ring_write(self._ptr(), _p(k), _p(v), n, int(bool(commit)))
+
+    def commit(self) -> None:
+        lib().orc_ring_commit(self._ptr())
+
+    def delta_rotate(self, delta: int) -> None:
+        lib().orc_ring_delta_rotate(self._ptr(), int(delta))
+
+    def attention(self, q, q_pos0: int, n_current: int, mask=(1 << 30, 1 << 30, 1 << 30, 1 << 30),
+                  cache_bias: float = 0.0, softmax_scale: float | None = None, rows=None,
+                  mode_b: bool = False):
+        """Returns (out [rows][H][D] f64, lse [H][rows] f64).
+
+        mask = (q_first_len, q_block_len, k_first_len, k_block_len)."""
+        q = _f32(q)
+        n_q = q.shape[0]
+        assert q.shape == (n_q, self.H, self.D)
+        if softmax_scale is None:
+            softmax_scale = float(np.float32(1.0 / np.sqrt(self.D)))
+        if rows is None:
+            rows_arr, n_rows, rp = None, n_q, None
+        else:
+            rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+            assert rows_arr.min() >= 0 and rows_arr.max() < n_q
+            n_rows, rp = rows_arr.size, _p(rows_arr)
+        out = np.zeros((n_rows, self.H, self.D), np.float64)
+        lse = np.zeros((self.H, n_rows), np.float64)
+        qf, qb, kf, kb = (int(x) for x in mask)
+        lib().orc_chunk_attention(self._ptr(), _p(q), n_q, int(q_pos0), int(n_current), qf, qb,
+                                  kf, kb, float(cache_bias), float(softmax_scale),
+                                  int(bool(mode_b)), rp, n_rows, _p(out), _p(lse))
+        return out, lse
