@@ -175,8 +175,9 @@ class BruteRing:
             S = float(softmax_scale) * (Q.astype(np.float64) @ K[h].T) + bias[None, :]
             S = np.where(visible, S, -np.inf)
             m = S.max(axis=1, keepdims=True)
-            P = np.exp(S - m)
+            live = np.isfinite(m[:, 0])          # rows with at least one finite score
+            P = np.exp(S[live] - m[live])
             l = P.sum(axis=1, keepdims=True)
-            out[:, h] = (P @ V[h]) / l
-            lse[h] = (m + np.log(l))[:, 0]
+            out[live, h] = (P @ V[h]) / l
+            lse[h, live] = (m[live] + np.log(l))[:, 0]
         return out, lse

@@ -311,6 +311,7 @@ ORC_API void orc_chunk_attention(const orc_ring* r, const float* q, int n_q, int
         ++nvis;
         if (sv > m) m = sv;
       }
+      if (m == -INFINITY) nvis = 0;  /* every visible score is -inf: nothing attended */
       double* o = out + ((size_t)ri * H + h) * D;
       for (int d = 0; d < D; ++d) o[d] = 0.0;
       double l = 0.0;

@@ -298,3 +298,13 @@ def test_empty_ring_gives_zero_output_and_minus_inf_lse(orc):
     q = np.ones((3, 2, 32), np.float32)
     out, lse = o.attention(q, 0, 0)
     assert (out == 0).all() and np.isneginf(lse).all()
+
+
+def test_minus_inf_bias_without_current_keys_attends_nothing(orc):
+    o, q, _ = _ring_with_history(orc)
+    o.commit()
+    out, lse = o.attention(q, o.next_pos, 0, cache_bias=-np.inf)
+    assert (out == 0).all() and np.isneginf(lse).all()
+    b = brute.BruteRing(o.C, o.H, o.D)
+    bo, bl = b.attention(q, 0, 0, (1, 1, 1, 1), -np.inf, 0.125)
+    assert (bo == 0).all() and np.isneginf(bl).all()
