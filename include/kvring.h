@@ -1,0 +1,200 @@
+/*
+ * kvring.h -- C ABI of the ring KV-cache attention library (libkvring.so, sm_100a).
+ *
+ * One hot path of chunk-wise autoregressive video diffusion, on one GPU:
+ *   write side: a ring KV cache; RoPE and FP8 (e4m3, one fp32 scale per token and head)
+ *               are applied once, when a token is written; a delta rotation re-rotates
+ *               the cached keys when positions reset.
+ *   read side:  a chunk of new queries attends over the whole cache under a block-causal
+ *               mask, with an additive bias on history slots.
+ * Sources: "Runway Characters: Serving a 57B Video Diffusion Transformer for Real-Time
+ * Conversation" (abstract: ring cache, RoPE + FP8 once per write, delta rotation on
+ * position reset, 240 calls per chunk over a 5,788-slot cache with 757 new tokens);
+ * "KREA Real-Time 14B / video-conductor" (section "Plastic Windows": lowering the cache
+ * attention bias); "Why Live Video Generation Still Struggles With Timing" (bidirectional
+ * inside the current chunk, backward-only across chunks, sliding window of history);
+ * "Stream LTX" (section "Training": blocks and causal masks on every attention path).
+ *
+ * Conventions shared by every entry point
+ *  - Ownership: the caller allocates and owns every device buffer and the CUDA stream.
+ *    The library allocates no device memory, keeps no global state and never
+ *    synchronises the stream.  Kernels are enqueued on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream) and read/write only the buffers named in the call.
+ *  - Errors: every function returns KV_OK (0) or a negative KV_E* code.  Argument, shape,
+ *    state and range errors are detected on the host before anything is enqueued, and
+ *    leave the ring state unchanged.  A launch failure returns KV_ECUDA (the CUDA error
+ *    is also left for cudaGetLastError).  Faults during execution surface as CUDA errors
+ *    at the caller's next synchronisation.  Nothing aborts, throws or traps.
+ *  - Concurrency: one kv_ring_t per stream/session.  Calls on the same ring must be
+ *    ordered on one stream; the host-side state fields are updated when a call is
+ *    enqueued, not when it completes.
+ *
+ * Numerics (bit-exact contract for codes, scales and slot positions)
+ *  - RoPE: 1-D positions, interleaved pairs (x[2i], x[2i+1]); angle p * theta_i with
+ *    theta_i = base^(-2i/D) evaluated in binary64 as pow(base, -(2i)/D); the table holds
+ *    c = (float)cos(angle), s = (float)sin(angle).  Rotation, in binary32 with separate
+ *    round-to-nearest-even operations (no fused multiply-add, no flush to zero):
+ *        y0 = (x0*c) - (x1*s),   y1 = (x0*s) + (x1*c).
+ *  - Quantisation of a D-element row y: amax = max|y_i|; scale = amax/448,
+ *    inv = 448/amax (binary32 divisions); code_i = e4m3(y_i * inv), OCP e4m3fn,
+ *    round-to-nearest-even, saturating to +-448.  amax == 0, or 448/amax not finite:
+ *    scale 0, codes 0.  A row with a non-finite element: scale NaN (bits 0x7FC00000),
+ *    all codes 0x7F.
+ *  - Attention: q~ = bf16_rne(RoPE(q, q_pos0 + i)); k~ = e4m3(kc) * ks; v~ = e4m3(vc) * vs;
+ *    s_ij = softmax_scale * <q~_i, k~_j> + (slot j is history ? history_bias : 0);
+ *    masked pairs are excluded; out_i = sum_j softmax_j(s_i) v~_j; lse_i = log sum exp.
+ *    Accumulation is fp32 on tensor cores; accuracy vs an fp64 evaluation of the same
+ *    definition is a tolerance, not bit-exact.
+ */
+#ifndef KVRING_H
+#define KVRING_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KV_API __attribute__((visibility("default")))
+#else
+#define KV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ------------------------------------------------------------------ status codes */
+#define KV_OK 0
+#define KV_EINVAL (-1)        /* null pointer, bad shape, bad dtype, bad flag, misaligned */
+#define KV_ERANGE (-2)        /* a count or position outside what the ring/table holds */
+#define KV_EUNSUPPORTED (-3)  /* head_dim not 64/128, device is not sm_100, ... */
+#define KV_ECUDA (-4)         /* a CUDA runtime/driver call failed */
+#define KV_ESTATE (-5)        /* ring not initialised, or state fields inconsistent */
+
+/* ------------------------------------------------------------------ input dtypes */
+#define KV_DTYPE_BF16 1
+#define KV_DTYPE_FP32 2
+
+/* ------------------------------------------------------------------ flags */
+#define KV_COMMIT 1u          /* kv_ring_write: commit the chunk after writing it */
+
+/* Per-stream ring-head state.  Plain data: the caller fills the shape, the device
+ * pointers, the RoPE table fields and next_pos, then calls kv_ring_init.  Copying the
+ * struct together with the device buffers it points to is a complete snapshot.
+ *
+ * Device layouts (all row-major, caller-allocated, 16-byte aligned):
+ *   k_codes, v_codes  uint8  [n_heads][capacity][head_dim]   e4m3fn codes
+ *   k_scale, v_scale  float  [n_heads][capacity]             one scale per token, head
+ *   slot_pos          int32  [capacity]                      RoPE position of each slot
+ *   rope_table        float  [rope_pos_max-rope_pos_min+1][head_dim/2][2]  (cos, sin)
+ * Ring semantics ("Runway Characters", abstract: a ring cache; "Why Live Video
+ * Generation Still Struggles With Timing": a sliding window of recent history):
+ *   the pending chunk occupies slots [write_slot, write_slot+pending) mod capacity;
+ *   committed history occupies the `live` slots before write_slot (FIFO overwrite);
+ *   valid slots = min(live + pending, capacity), the newest ending at
+ *   write_slot + pending - 1 (mod capacity). */
+typedef struct kv_ring {
+  int32_t capacity;          /* C: number of slots, >= 1 */
+  int32_t n_heads;           /* H */
+  int32_t head_dim;          /* D: 64 or 128 */
+  int32_t initialized;       /* set by kv_ring_init; do not write */
+  int64_t write_slot;        /* physical slot of the first pending/next token, [0, C) */
+  int64_t live;              /* committed valid slots, [0, C] */
+  int64_t pending;           /* tokens written at write_slot but not committed */
+  int64_t next_pos;          /* RoPE position of the first pending/next token */
+  uint8_t* k_codes;
+  uint8_t* v_codes;
+  float* k_scale;
+  float* v_scale;
+  int32_t* slot_pos;
+  const float* rope_table;   /* device copy of kv_rope_table_build's output */
+  int64_t rope_pos_min;      /* first position held by rope_table */
+  int64_t rope_pos_max;      /* last position held by rope_table */
+  double rope_base;          /* base used to build the table (for the delta rotation) */
+  uint64_t opaque[48];       /* library-owned: encoded TMA descriptors of the caches */
+} kv_ring_t;
+
+/* Block-causal mask of the current chunk ("Stream LTX", section "Training": a block is
+ * the unit inside which attention is bidirectional; across blocks it only looks back;
+ * "Why Live Video Generation Still Struggles With Timing": bidirectional within the
+ * chunk, backward across chunks).  Block id of chunk token t:
+ *   t < first_len ? 0 : 1 + (t - first_len) / block_len     (queries: q_*, keys: k_*)
+ * A current-chunk key is visible iff its block id <= the query's.  History keys are
+ * always visible.  block_len = first_len = 1 gives token-causal masking; a length larger
+ * than the chunk gives one bidirectional block.  NULL means one block. */
+typedef struct kv_block_mask {
+  int32_t q_first_len, q_block_len, k_first_len, k_block_len; /* all >= 1 */
+} kv_block_mask_t;
+
+/* Additive logit on history slots ("KREA Real-Time 14B / video-conductor", section
+ * "Plastic Windows": lowering the cache attention bias opens a plastic window during
+ * prompt transitions; read here as a natural-log offset added after softmax_scale).
+ * NULL means 0.  -INFINITY removes history entirely. */
+typedef struct kv_cache_bias {
+  float history_bias;
+} kv_cache_bias_t;
+
+/* Fill host_out[(p - pos_min) * D + 2*i + {0,1}] = (cos, sin)(p * theta_i), rounded to
+ * binary32, for pos_min <= p <= pos_max and i < D/2, by the RoPE rule above.  Host only
+ * ("Runway Characters", abstract: RoPE applied once per write).  host_out holds
+ * (pos_max - pos_min + 1) * D floats.  Errors: KV_EINVAL (null, D not even, pos_max <
+ * pos_min, base <= 0). */
+KV_API int kv_rope_table_build(float* host_out, int64_t pos_min, int64_t pos_max, int head_dim,
+                        double base);
+
+/* Validate a filled kv_ring_t, check the current device is sm_100, encode the TMA
+ * descriptors of the caches into kv->opaque, and reset write_slot, live and pending to 0
+ * (next_pos is kept).  Must be called again after any device pointer changes.
+ * Errors: KV_EINVAL, KV_EUNSUPPORTED, KV_ECUDA. */
+KV_API int kv_ring_init(kv_ring_t* kv);
+
+/* Write n_tokens new tokens as the pending chunk ("Runway Characters", abstract: RoPE and
+ * FP8 quantisation applied once per write).  k, v: device [n_tokens][H][D] in in_dtype
+ * (KV_DTYPE_BF16 or KV_DTYPE_FP32), 16-byte aligned.  Token t goes to slot
+ * (write_slot + t) mod C at position next_pos + t: K is rotated then quantised, V is
+ * quantised; scales and slot_pos are written.  A previous pending chunk is replaced
+ * (denoising passes rewrite the same chunk); the rewrite must be at least as long as the
+ * pending chunk it replaces (else KV_ESTATE).  With KV_COMMIT the chunk is then
+ * committed as by kv_ring_commit.  Errors: KV_EINVAL, KV_ERANGE (n_tokens < 1 or > C,
+ * a position outside the table), KV_ESTATE, KV_ECUDA. */
+KV_API int kv_ring_write(kv_ring_t* kv, const void* k, const void* v, int in_dtype, int n_tokens,
+                  uint32_t flags, void* stream);
+
+/* Commit the pending chunk: write_slot += pending (mod C), live = min(C, live + pending),
+ * next_pos += pending, pending = 0.  Host only.  Errors: KV_EINVAL, KV_ESTATE. */
+KV_API int kv_ring_commit(kv_ring_t* kv);
+
+/* Position reset ("Runway Characters", abstract: a delta rotation when positions reset):
+ * every valid cached key row is dequantised (code * scale, binary32), rotated by the
+ * angles of `delta` (computed on the host by the RoPE rule with kv->rope_base) and
+ * requantised by the rule above; slot_pos of valid slots and next_pos shift by delta.
+ * V is untouched.  Errors: KV_EINVAL, KV_ERANGE (shifted positions leave int32),
+ * KV_ESTATE, KV_ECUDA. */
+KV_API int kv_ring_delta_rotate(kv_ring_t* kv, int64_t delta, void* stream);
+
+/* Chunk attention ("Runway Characters", abstract: each call reads the whole cache, only
+ * the newest tokens are new).  q: device bf16 [n_q][H][D]; query i is rotated at
+ * q_pos0 + i.  Keys are the valid slots; the newest n_current of them are the current
+ * chunk (masked by `mask`, no bias), the rest are history (bias added, always visible).
+ * out: device bf16 [n_q][H][D]; lse: device fp32 [H][n_q] natural-log sum of exp, or
+ * NULL.  A row with no visible key gets out = 0 and lse = -inf.  softmax_scale > 0.
+ * flags must be 0.  Errors: KV_EINVAL, KV_ERANGE (n_current > valid slots, a query
+ * position outside the table), KV_ESTATE, KV_ECUDA. */
+KV_API int chunk_attention(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
+                    int n_current, const kv_block_mask_t* mask, const kv_cache_bias_t* bias,
+                    float softmax_scale, void* out, float* lse, uint32_t flags, void* stream);
+
+/* Static description of a status code.  Never NULL. */
+KV_API const char* kv_status_string(int status);
+
+/* Number of device-side waits (on TMA or tensor-core completion) that gave up after
+ * about one second since the library was loaded on the current device.  A kernel whose
+ * wait gave up abandons its work, writes NaN to the rows it owned and exits; a non-zero
+ * count means those outputs are invalid.  Synchronous (reads a device word).  Errors:
+ * KV_EINVAL (null), KV_ECUDA. */
+KV_API int kv_wait_timeout_count(uint32_t* host_count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVRING_H */

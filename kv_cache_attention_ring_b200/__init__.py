@@ -1,0 +1,206 @@
+"""Ring KV-cache attention for chunk-wise video diffusion on B200 (sm_100a).
+
+Thin ctypes binding of ``libkvring.so`` (C ABI in ``include/kvring.h``).  The binding
+only marshals arguments: every step of the path runs in the library's CUDA kernels.
+PyTorch provides device memory and streams.  There is no fallback: if the library is
+missing or the device is not sm_100, calls raise.
+
+Entry points (same names as the C ABI): ``kv_rope_table_build``, ``KvRing`` (fills a
+``kv_ring_t`` and calls ``kv_ring_init``), ``kv_ring_write``, ``kv_ring_commit``,
+``kv_ring_delta_rotate``, ``chunk_attention``, ``kv_status_string``,
+``kv_wait_timeout_count``.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkvring.so")
+
+KV_OK, KV_EINVAL, KV_ERANGE, KV_EUNSUPPORTED, KV_ECUDA, KV_ESTATE = 0, -1, -2, -3, -4, -5
+KV_DTYPE_BF16, KV_DTYPE_FP32 = 1, 2
+KV_COMMIT = 1
+
+EXPORTS = ("kv_rope_table_build", "kv_ring_init", "kv_ring_write", "kv_ring_commit",
+           "kv_ring_delta_rotate", "chunk_attention", "kv_status_string",
+           "kv_wait_timeout_count")
+
+
+class KvError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {kv_status_string(status)} (status {status})")
+        self.status = status
+
+
+class kv_ring_t(ctypes.Structure):
+    _fields_ = [("capacity", ctypes.c_int32), ("n_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("initialized", ctypes.c_int32),
+                ("write_slot", ctypes.c_int64), ("live", ctypes.c_int64),
+                ("pending", ctypes.c_int64), ("next_pos", ctypes.c_int64),
+                ("k_codes", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
+                ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
+                ("slot_pos", ctypes.c_void_p), ("rope_table", ctypes.c_void_p),
+                ("rope_pos_min", ctypes.c_int64), ("rope_pos_max", ctypes.c_int64),
+                ("rope_base", ctypes.c_double), ("opaque", ctypes.c_uint64 * 48)]
+
+
+class kv_block_mask_t(ctypes.Structure):
+    _fields_ = [("q_first_len", ctypes.c_int32), ("q_block_len", ctypes.c_int32),
+                ("k_first_len", ctypes.c_int32), ("k_block_len", ctypes.c_int32)]
+
+
+class kv_cache_bias_t(ctypes.Structure):
+    _fields_ = [("history_bias", ctypes.c_float)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libkvring.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m kv_cache_attention_ring_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+        L.kv_rope_table_build.argtypes = [P, I64, I64, I, ctypes.c_double]
+        L.kv_ring_init.argtypes = [P]
+        L.kv_ring_write.argtypes = [P, P, P, I, I, ctypes.c_uint32, P]
+        L.kv_ring_commit.argtypes = [P]
+        L.kv_ring_delta_rotate.argtypes = [P, I64, P]
+        L.chunk_attention.argtypes = [P, P, I, I64, I, P, P, ctypes.c_float, P, P,
+                                      ctypes.c_uint32, P]
+        L.kv_status_string.argtypes = [I]
+        L.kv_status_string.restype = ctypes.c_char_p
+        L.kv_wait_timeout_count.argtypes = [P]
+        _lib = L
+    return _lib
+
+
+def kv_status_string(status: int) -> str:
+    return lib().kv_status_string(int(status)).decode()
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != KV_OK:
+        raise KvError(rc, what)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def kv_rope_table_build(pos_min: int, pos_max: int, head_dim: int,
+                        base: float = 10000.0) -> np.ndarray:
+    """Host RoPE table [(pos_max-pos_min+1)][head_dim/2][2] float32 (cos, sin)."""
+    out = np.empty((pos_max - pos_min + 1, head_dim // 2, 2), np.float32)
+    _check(lib().kv_rope_table_build(ctypes.c_void_p(out.ctypes.data), int(pos_min),
+                                     int(pos_max), int(head_dim), float(base)),
+           "kv_rope_table_build")
+    return out
+
+
+class KvRing:
+    """A ring with its caller-owned device buffers (torch tensors) and its kv_ring_t."""
+
+    def __init__(self, capacity: int, n_heads: int, head_dim: int, pos_min: int, pos_max: int,
+                 base: float = 10000.0, next_pos: int = 0, device=None, rope_table=None):
+        import torch
+        dev = torch.device("cuda") if device is None else torch.device(device)
+        C, H, D = int(capacity), int(n_heads), int(head_dim)
+        self.C, self.H, self.D = C, H, D
+        self.k_codes = torch.zeros((H, C, D), dtype=torch.uint8, device=dev)
+        self.v_codes = torch.zeros((H, C, D), dtype=torch.uint8, device=dev)
+        self.k_scale = torch.zeros((H, C), dtype=torch.float32, device=dev)
+        self.v_scale = torch.zeros((H, C), dtype=torch.float32, device=dev)
+        self.slot_pos = torch.zeros((C,), dtype=torch.int32, device=dev)
+        if rope_table is None:
+            rope_table = torch.from_numpy(kv_rope_table_build(pos_min, pos_max, D, base)).to(dev)
+        self.rope_table = rope_table
+        s = kv_ring_t()
+        s.capacity, s.n_heads, s.head_dim = C, H, D
+        s.next_pos = int(next_pos)
+        s.k_codes, s.v_codes = self.k_codes.data_ptr(), self.v_codes.data_ptr()
+        s.k_scale, s.v_scale = self.k_scale.data_ptr(), self.v_scale.data_ptr()
+        s.slot_pos = self.slot_pos.data_ptr()
+        s.rope_table = self.rope_table.data_ptr()
+        s.rope_pos_min, s.rope_pos_max, s.rope_base = int(pos_min), int(pos_max), float(base)
+        self.s = s
+        _check(lib().kv_ring_init(ctypes.byref(s)), "kv_ring_init")
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.s)
+
+    def state(self) -> tuple[int, int, int, int]:
+        return (self.s.write_slot, self.s.live, self.s.pending, self.s.next_pos)
+
+    @property
+    def next_pos(self) -> int:
+        return self.s.next_pos
+
+    @property
+    def n_valid(self) -> int:
+        return min(self.s.live + self.s.pending, self.C)
+
+
+def kv_ring_write(ring: KvRing, k, v, commit: bool = False, stream=None) -> None:
+    import torch
+    assert k.is_cuda and v.is_cuda and k.is_contiguous() and v.is_contiguous()
+    assert k.shape == v.shape and k.dim() == 3 and k.shape[1:] == (ring.H, ring.D)
+    dt = {torch.bfloat16: KV_DTYPE_BF16, torch.float32: KV_DTYPE_FP32}.get(k.dtype)
+    assert dt is not None and v.dtype == k.dtype
+    _check(lib().kv_ring_write(ring.ref, _ptr(k), _ptr(v), dt, int(k.shape[0]),
+                               KV_COMMIT if commit else 0, _stream(stream)), "kv_ring_write")
+
+
+def kv_ring_commit(ring: KvRing) -> None:
+    _check(lib().kv_ring_commit(ring.ref), "kv_ring_commit")
+
+
+def kv_ring_delta_rotate(ring: KvRing, delta: int, stream=None) -> None:
+    _check(lib().kv_ring_delta_rotate(ring.ref, int(delta), _stream(stream)),
+           "kv_ring_delta_rotate")
+
+
+def chunk_attention(ring: KvRing, q, q_pos0: int, n_current: int, mask=None,
+                    cache_bias: float = 0.0, softmax_scale: float | None = None, out=None,
+                    lse=None, want_lse: bool = True, stream=None):
+    """q: bf16 [n_q][H][D] on the GPU.  mask: (q_first, q_block, k_first, k_block) or None.
+    Returns (out bf16 [n_q][H][D], lse fp32 [H][n_q] or None)."""
+    import torch
+    assert q.is_cuda and q.dtype == torch.bfloat16 and q.is_contiguous()
+    n_q = int(q.shape[0])
+    assert q.shape == (n_q, ring.H, ring.D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((ring.H, n_q), dtype=torch.float32, device=q.device)
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(ring.D)
+    m = None if mask is None else kv_block_mask_t(*(int(x) for x in mask))
+    b = kv_cache_bias_t(float(cache_bias))
+    _check(lib().chunk_attention(ring.ref, _ptr(q), n_q, int(q_pos0), int(n_current),
+                                 None if m is None else ctypes.byref(m), ctypes.byref(b),
+                                 float(softmax_scale), _ptr(out),
+                                 None if lse is None else _ptr(lse), 0, _stream(stream)),
+           "chunk_attention")
+    return out, lse
+
+
+def kv_wait_timeout_count() -> int:
+    v = ctypes.c_uint32(0)
+    _check(lib().kv_wait_timeout_count(ctypes.byref(v)), "kv_wait_timeout_count")
+    return int(v.value)

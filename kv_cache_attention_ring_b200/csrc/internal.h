@@ -1,0 +1,60 @@
+// internal.h -- launch interfaces between the C ABI (kvring_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kvring {
+
+struct WriteArgs {
+  const void* k;            // [n][H][D] input dtype
+  const void* v;
+  uint8_t* kc;              // [H][C][D]
+  uint8_t* vc;
+  float* ks;                // [H][C]
+  float* vs;
+  int32_t* slot_pos;        // [C]
+  const float* rope_row0;   // table row of position `pos0`: [n][D/2][2] floats follow
+  int n, H, C;
+  int64_t w;                // first slot
+  int64_t pos0;             // position of token 0
+};
+
+struct RotateArgs {
+  uint8_t* kc;
+  float* ks;
+  int32_t* slot_pos;
+  int H, C;
+  int64_t first_slot;       // oldest valid slot
+  int64_t count;            // valid slots (contiguous mod C from first_slot)
+  int32_t delta;
+  float cs[128];            // (cos, sin) of delta * theta_i, i < D/2, interleaved
+};
+
+struct AttnArgs {
+  const uint16_t* q;        // bf16 [n_q][H][D]
+  uint16_t* out;            // bf16 [n_q][H][D]
+  float* lse;               // [H][n_q] or null
+  const float* k_scale;     // [H][C]
+  const float* v_scale;
+  const float* rope_q0;     // table row of position q_pos0
+  int n_q, H, C;
+  int n_current;
+  int64_t newest_slot;      // slot of the newest valid token
+  int64_t n_valid;          // valid slots
+  int q_first, q_block, k_first, k_block;
+  float score_scale_log2;   // softmax_scale * log2(e)
+  float bias_log2;          // history_bias * log2(e)
+  unsigned int* timeouts;   // device counter of waits that gave up
+};
+
+// Device address of the library's wait-timeout counter on the current device.
+unsigned int* timeout_counter();
+
+int launch_write(const WriteArgs& a, int D, int in_dtype, cudaStream_t s);
+int launch_rotate(const RotateArgs& a, int D, cudaStream_t s);
+// tmaps: two 128-byte CUtensorMap images (K codes, V codes), 64-byte aligned.
+int launch_attention(const AttnArgs& a, int D, const void* tmap_k, const void* tmap_v,
+                     cudaStream_t s);
+
+}  // namespace kvring

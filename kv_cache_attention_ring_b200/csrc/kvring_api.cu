@@ -1,0 +1,294 @@
+// kvring_api.cu -- the C ABI declared in include/kvring.h: argument and state validation,
+// ring-head arithmetic, the host-built RoPE table, TMA descriptor encoding, launches.
+//
+// Ring semantics follow "Runway Characters: Serving a 57B Video Diffusion Transformer for
+// Real-Time Conversation" (abstract: a ring cache written once per token, a delta rotation
+// when positions reset).  Every check happens here, before anything is enqueued; the
+// kernels assume validated arguments.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <string.h>
+
+#include "../../include/kvring.h"
+#include "internal.h"
+
+namespace kvring {
+__device__ unsigned int g_wait_timeouts = 0;
+
+unsigned int* timeout_counter() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_wait_timeouts) != cudaSuccess) return nullptr;
+  return static_cast<unsigned int*>(p);
+}
+}
+
+using namespace kvring;
+
+namespace {
+
+constexpr uint64_t kMagic = 0x6B7672696E673031ull;  // "kvring01"
+constexpr int kOpaqueTmapK = 0;                     // uint64 index of the K tensor map
+constexpr int kOpaqueTmapV = 16;                    // uint64 index of the V tensor map
+constexpr int kOpaqueMagic = 32;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t mod_c(int64_t a, int64_t c) {
+  int64_t r = a % c;
+  return r < 0 ? r + c : r;
+}
+
+// (cos, sin) of p * theta_i, theta_i = base^(-2i/D), binary64 angle, rounded to binary32.
+void rope_angles(int64_t p, int D, double base, float* out /* [D/2][2] */) {
+  for (int i = 0; i < D / 2; ++i) {
+    const double theta_i = pow(base, -(2.0 * (double)i) / (double)D);
+    const double angle = (double)p * theta_i;
+    out[2 * i] = (float)cos(angle);
+    out[2 * i + 1] = (float)sin(angle);
+  }
+}
+
+int check_ring(const kv_ring_t* kv) {
+  if (!kv) return KV_EINVAL;
+  if (!kv->initialized || kv->opaque[kOpaqueMagic] != kMagic) return KV_ESTATE;
+  const int64_t C = kv->capacity;
+  if (kv->write_slot < 0 || kv->write_slot >= C || kv->live < 0 || kv->live > C ||
+      kv->pending < 0 || kv->pending > C)
+    return KV_ESTATE;
+  return KV_OK;
+}
+
+int64_t valid_slots(const kv_ring_t* kv) {
+  const int64_t v = kv->live + kv->pending;
+  return v > kv->capacity ? kv->capacity : v;
+}
+
+bool in_table(const kv_ring_t* kv, int64_t p_first, int64_t p_last) {
+  return p_first >= kv->rope_pos_min && p_last <= kv->rope_pos_max && p_first <= p_last;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 3-D map over codes [H][C][D] bytes; box = D bytes x 128 slots x 1 head, no swizzle.
+// Slots >= C read as zero.
+int encode_codes_map(void* base, int H, int C, int D, uint64_t* dst) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return KV_ECUDA;
+  alignas(64) CUtensorMap m;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)C, (cuuint64_t)H};
+  const cuuint64_t strides[2] = {(cuuint64_t)D, (cuuint64_t)C * (cuuint64_t)D};
+  const cuuint32_t box[3] = {(cuuint32_t)D, 128u, 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return KV_ECUDA;
+  static_assert(sizeof(CUtensorMap) == 128, "CUtensorMap is 128 bytes");
+  memcpy(dst, &m, sizeof(m));
+  return KV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kv_status_string(int status) {
+  switch (status) {
+    case KV_OK: return "ok";
+    case KV_EINVAL: return "invalid argument (null pointer, shape, dtype, flag or alignment)";
+    case KV_ERANGE: return "count or position out of range of the ring or the RoPE table";
+    case KV_EUNSUPPORTED: return "unsupported configuration (head_dim or device)";
+    case KV_ECUDA: return "CUDA runtime or driver call failed";
+    case KV_ESTATE: return "ring not initialised or its state is inconsistent";
+    default: return "unknown status";
+  }
+}
+
+int kv_rope_table_build(float* host_out, int64_t pos_min, int64_t pos_max, int head_dim,
+                        double base) {
+  if (!host_out || head_dim <= 0 || (head_dim & 1) || pos_max < pos_min || !(base > 0.0))
+    return KV_EINVAL;
+  for (int64_t p = pos_min; p <= pos_max; ++p)
+    rope_angles(p, head_dim, base, host_out + (size_t)(p - pos_min) * head_dim);
+  return KV_OK;
+}
+
+int kv_ring_init(kv_ring_t* kv) {
+  if (!kv) return KV_EINVAL;
+  kv->initialized = 0;
+  if (kv->capacity < 1 || kv->n_heads < 1) return KV_EINVAL;
+  if (kv->head_dim != 64 && kv->head_dim != 128) return KV_EUNSUPPORTED;
+  if (!kv->k_codes || !kv->v_codes || !kv->k_scale || !kv->v_scale || !kv->slot_pos ||
+      !kv->rope_table)
+    return KV_EINVAL;
+  if (!aligned16(kv->k_codes) || !aligned16(kv->v_codes) || !aligned16(kv->rope_table))
+    return KV_EINVAL;
+  if (kv->rope_pos_max < kv->rope_pos_min || !(kv->rope_base > 0.0)) return KV_EINVAL;
+  if ((int64_t)kv->capacity * kv->n_heads > (int64_t)1 << 31) return KV_ERANGE;
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KV_ECUDA;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return KV_ECUDA;
+  if (major != 10 || minor != 0) return KV_EUNSUPPORTED;
+  int rc = encode_codes_map(kv->k_codes, kv->n_heads, kv->capacity, kv->head_dim,
+                            kv->opaque + kOpaqueTmapK);
+  if (rc) return rc;
+  rc = encode_codes_map(kv->v_codes, kv->n_heads, kv->capacity, kv->head_dim,
+                        kv->opaque + kOpaqueTmapV);
+  if (rc) return rc;
+  kv->opaque[kOpaqueMagic] = kMagic;
+  kv->write_slot = 0;
+  kv->live = 0;
+  kv->pending = 0;
+  kv->initialized = 1;
+  return KV_OK;
+}
+
+int kv_ring_commit(kv_ring_t* kv) {
+  int rc = check_ring(kv);
+  if (rc) return rc;
+  const int64_t C = kv->capacity;
+  kv->write_slot = mod_c(kv->write_slot + kv->pending, C);
+  kv->live = kv->live + kv->pending > C ? C : kv->live + kv->pending;
+  kv->next_pos += kv->pending;
+  kv->pending = 0;
+  return KV_OK;
+}
+
+int kv_ring_write(kv_ring_t* kv, const void* k, const void* v, int in_dtype, int n_tokens,
+                  uint32_t flags, void* stream) {
+  int rc = check_ring(kv);
+  if (rc) return rc;
+  if (!k || !v || !aligned16(k) || !aligned16(v)) return KV_EINVAL;
+  if (in_dtype != KV_DTYPE_BF16 && in_dtype != KV_DTYPE_FP32) return KV_EINVAL;
+  if (flags & ~KV_COMMIT) return KV_EINVAL;
+  if (n_tokens < 1 || n_tokens > kv->capacity) return KV_ERANGE;
+  if (n_tokens < kv->pending) return KV_ESTATE;  // a rewrite must cover the pending chunk
+  const int64_t p0 = kv->next_pos, p1 = kv->next_pos + n_tokens - 1;
+  if (!in_table(kv, p0, p1) || p0 < INT32_MIN || p1 > INT32_MAX) return KV_ERANGE;
+  WriteArgs a;
+  a.k = k;
+  a.v = v;
+  a.kc = kv->k_codes;
+  a.vc = kv->v_codes;
+  a.ks = kv->k_scale;
+  a.vs = kv->v_scale;
+  a.slot_pos = kv->slot_pos;
+  a.rope_row0 = kv->rope_table + (size_t)(p0 - kv->rope_pos_min) * kv->head_dim;
+  a.n = n_tokens;
+  a.H = kv->n_heads;
+  a.C = kv->capacity;
+  a.w = kv->write_slot;
+  a.pos0 = p0;
+  rc = launch_write(a, kv->head_dim, in_dtype, static_cast<cudaStream_t>(stream));
+  if (rc) return rc;
+  kv->pending = n_tokens;
+  if (flags & KV_COMMIT) return kv_ring_commit(kv);
+  return KV_OK;
+}
+
+int kv_ring_delta_rotate(kv_ring_t* kv, int64_t delta, void* stream) {
+  int rc = check_ring(kv);
+  if (rc) return rc;
+  const int64_t nv = valid_slots(kv);
+  const int64_t committed = nv - kv->pending;              // history still in the ring
+  const int64_t lo = kv->next_pos - committed + delta;     // oldest valid position after
+  const int64_t hi = kv->next_pos + (kv->pending > 0 ? kv->pending - 1 : 0) + delta;
+  if (delta < INT32_MIN || delta > INT32_MAX || lo < INT32_MIN || hi > INT32_MAX)
+    return KV_ERANGE;
+  if (nv > 0) {
+    RotateArgs a;
+    a.kc = kv->k_codes;
+    a.ks = kv->k_scale;
+    a.slot_pos = kv->slot_pos;
+    a.H = kv->n_heads;
+    a.C = kv->capacity;
+    a.first_slot = mod_c(kv->write_slot + kv->pending - nv, kv->capacity);
+    a.count = nv;
+    a.delta = (int32_t)delta;
+    rope_angles(delta, kv->head_dim, kv->rope_base, a.cs);
+    rc = launch_rotate(a, kv->head_dim, static_cast<cudaStream_t>(stream));
+    if (rc) return rc;
+  }
+  kv->next_pos += delta;
+  return KV_OK;
+}
+
+int chunk_attention(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
+                    int n_current, const kv_block_mask_t* mask, const kv_cache_bias_t* bias,
+                    float softmax_scale, void* out, float* lse, uint32_t flags, void* stream) {
+  int rc = check_ring(kv);
+  if (rc) return rc;
+  if (flags != 0) return KV_EINVAL;
+  if (n_q < 0 || n_current < 0) return KV_EINVAL;
+  if (n_q == 0) return KV_OK;
+  if (!q || !out || !aligned16(q) || !aligned16(out)) return KV_EINVAL;
+  if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return KV_EINVAL;
+  const float b = bias ? bias->history_bias : 0.f;
+  if (isnan(b) || b == INFINITY) return KV_EINVAL;
+  kv_block_mask_t m = {1 << 30, 1 << 30, 1 << 30, 1 << 30};
+  if (mask) {
+    if (mask->q_first_len < 1 || mask->q_block_len < 1 || mask->k_first_len < 1 ||
+        mask->k_block_len < 1)
+      return KV_EINVAL;
+    m = *mask;
+  }
+  const int64_t nv = valid_slots(kv);
+  if (n_current > nv) return KV_ERANGE;
+  if (!in_table(kv, q_pos0, q_pos0 + n_q - 1)) return KV_ERANGE;
+  if ((int64_t)n_q * kv->n_heads > ((int64_t)1 << 31)) return KV_ERANGE;
+  AttnArgs a;
+  a.q = static_cast<const uint16_t*>(q);
+  a.out = static_cast<uint16_t*>(out);
+  a.lse = lse;
+  a.k_scale = kv->k_scale;
+  a.v_scale = kv->v_scale;
+  a.rope_q0 = kv->rope_table + (size_t)(q_pos0 - kv->rope_pos_min) * kv->head_dim;
+  a.n_q = n_q;
+  a.H = kv->n_heads;
+  a.C = kv->capacity;
+  a.n_current = n_current;
+  a.newest_slot = mod_c(kv->write_slot + kv->pending - 1, kv->capacity);
+  a.n_valid = nv;
+  a.q_first = m.q_first_len;
+  a.q_block = m.q_block_len;
+  a.k_first = m.k_first_len;
+  a.k_block = m.k_block_len;
+  const float log2e = 1.4426950408889634f;
+  a.score_scale_log2 = softmax_scale * log2e;
+  a.bias_log2 = b * log2e;
+  a.timeouts = timeout_counter();
+  if (!a.timeouts) return KV_ECUDA;
+  return launch_attention(a, kv->head_dim, kv->opaque + kOpaqueTmapK,
+                          kv->opaque + kOpaqueTmapV, static_cast<cudaStream_t>(stream));
+}
+
+int kv_wait_timeout_count(uint32_t* host_count) {
+  if (!host_count) return KV_EINVAL;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, kvring::g_wait_timeouts, sizeof(v)) != cudaSuccess)
+    return KV_ECUDA;
+  *host_count = v;
+  return KV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,82 @@
+"""Shared helpers of the GPU parity tests: run the same seeded stream through the CUDA
+path (C ABI) and through the oracle, and compare."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import kv_cache_attention_ring_b200 as kv
+from kv_cache_attention_ring_b200 import inputs
+
+# Attention acceptance (max-abs and relative L2 against the fp64 oracle evaluated on the
+# same dequantised FP8 values).
+ATOL = 2e-2
+REL_L2 = 5e-3
+LSE_ATOL = 2e-3
+
+
+def to_dev(t: torch.Tensor) -> torch.Tensor:
+    return t.contiguous().cuda()
+
+
+def assert_ring_equal(ring: kv.KvRing, o, slots=None, what=""):
+    """Bit-exact comparison of codes, scales, slot positions and state integers."""
+    torch.cuda.synchronize()
+    assert ring.state() == o.state(), (what, ring.state(), o.state())
+    if slots is None:
+        kc, vc = ring.k_codes.cpu().numpy(), ring.v_codes.cpu().numpy()
+        ks, vs = ring.k_scale.cpu().numpy(), ring.v_scale.cpu().numpy()
+        sp = ring.slot_pos.cpu().numpy()
+        ok_kc, ok_vc = o.kc, o.vc
+        ok_ks, ok_vs, ok_sp = o.ks, o.vs, o.slot_pos
+    else:
+        idx = torch.as_tensor(np.asarray(slots), dtype=torch.long, device="cuda")
+        kc = ring.k_codes[:, idx].cpu().numpy()
+        vc = ring.v_codes[:, idx].cpu().numpy()
+        ks = ring.k_scale[:, idx].cpu().numpy()
+        vs = ring.v_scale[:, idx].cpu().numpy()
+        sp = ring.slot_pos[idx].cpu().numpy()
+        s = np.asarray(slots)
+        ok_kc, ok_vc, ok_ks, ok_vs, ok_sp = o.kc[:, s], o.vc[:, s], o.ks[:, s], o.vs[:, s], o.slot_pos[s]
+    bad = np.argwhere(kc != ok_kc)
+    assert bad.size == 0, (what, "k codes differ", bad[:5].tolist(), kc[tuple(bad[0])],
+                           ok_kc[tuple(bad[0])])
+    assert (vc == ok_vc).all(), (what, "v codes differ")
+    assert (ks.view(np.uint32) == ok_ks.view(np.uint32)).all(), (what, "k scales differ")
+    assert (vs.view(np.uint32) == ok_vs.view(np.uint32)).all(), (what, "v scales differ")
+    assert (sp == ok_sp).all(), (what, "slot positions differ")
+
+
+def valid_slots(o) -> list[int]:
+    nv = min(o.live + o.pending, o.C)
+    return [o.slot_of_age(a) for a in range(nv)]
+
+
+def assert_attention_close(out, lse, ref_out, ref_lse, rows=None, what=""):
+    """out: GPU bf16 [n_q][H][D]; lse: GPU fp32 [H][n_q]; refs from the oracle for `rows`."""
+    torch.cuda.synchronize()
+    o = out.float().cpu().numpy().astype(np.float64)
+    l = None if lse is None else lse.cpu().numpy().astype(np.float64)
+    if rows is not None:
+        o = o[np.asarray(rows)]
+        if l is not None:
+            l = l[:, np.asarray(rows)]
+    assert np.isfinite(o).all(), (what, "non-finite output")
+    err = np.abs(o - ref_out)
+    rel = np.linalg.norm(o - ref_out) / max(np.linalg.norm(ref_out), 1e-30)
+    assert err.max() <= ATOL, (what, "max abs", float(err.max()))
+    assert rel <= REL_L2, (what, "rel L2", float(rel))
+    if l is not None:
+        fin = np.isfinite(ref_lse)
+        assert (np.isfinite(l) == fin).all(), (what, "lse finiteness")
+        assert (l[~fin] == ref_lse[~fin]).all()
+        assert np.abs(l[fin] - ref_lse[fin]).max(initial=0) <= LSE_ATOL, (what, "lse")
+    return float(err.max()), float(rel)
+
+
+def sample_rows(n_q: int, k: int, seed: int) -> np.ndarray:
+    """Seeded sample of query rows that always includes tile edges and the last row."""
+    rng = np.random.default_rng(seed)
+    fixed = [0, 1, 127, 128, 129, n_q // 2, n_q - 2, n_q - 1]
+    rest = rng.choice(n_q, size=min(k, n_q), replace=False)
+    return np.unique(np.clip(np.concatenate([fixed, rest]), 0, n_q - 1)).astype(np.int32)

@@ -1,0 +1,146 @@
+"""Host-side checks of the C ABI that need no GPU: exports, status strings, the RoPE
+table, and argument/state validation that returns before anything is enqueued."""
+import ctypes
+import re
+
+import numpy as np
+import pytest
+
+import kv_cache_attention_ring_b200 as kv
+from kv_cache_attention_ring_b200 import build
+
+MAGIC = 0x6B7672696E673031
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return kv.lib()
+
+
+def _declared():
+    src = open(build.os.path.join(build.HERE, "..", "include", "kvring.h")).read()
+    return re.findall(r"^KV_API\s+[\w\s\*]+?\b(\w+)\(", src, re.M)
+
+
+def test_library_exports_every_declared_symbol(L):
+    names = _declared()
+    assert sorted(names) == sorted(kv.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code in (0, -1, -2, -3, -4, -5):
+        assert kv.kv_status_string(code) and "unknown" not in kv.kv_status_string(code)
+    assert "unknown" in kv.kv_status_string(-99)
+
+
+def test_rope_table_matches_oracle_angles(L, orc):
+    tab = kv.kv_rope_table_build(-130, 300, 64)
+    for p in (-130, -1, 0, 1, 255, 300):
+        c, s = orc.rope_cs(p, 64)
+        assert (tab[p + 130, :, 0].view(np.uint32) == c.view(np.uint32)).all()
+        assert (tab[p + 130, :, 1].view(np.uint32) == s.view(np.uint32)).all()
+    with pytest.raises(kv.KvError):
+        kv.kv_rope_table_build(5, 4, 64)
+
+
+def _fake_ring(C=256, H=2, D=64, pmin=0, pmax=4096):
+    s = kv.kv_ring_t()
+    s.capacity, s.n_heads, s.head_dim = C, H, D
+    for f in ("k_codes", "v_codes", "k_scale", "v_scale", "slot_pos", "rope_table"):
+        setattr(s, f, 0x100000)             # never dereferenced on these paths
+    s.rope_pos_min, s.rope_pos_max, s.rope_base = pmin, pmax, 10000.0
+    s.initialized = 1
+    s.opaque[32] = MAGIC
+    return s
+
+
+def test_init_validation_without_gpu(L):
+    s = kv.kv_ring_t()
+    assert L.kv_ring_init(None) == kv.KV_EINVAL
+    assert L.kv_ring_init(ctypes.byref(s)) == kv.KV_EINVAL          # zero capacity
+    s = _fake_ring(D=96)
+    assert L.kv_ring_init(ctypes.byref(s)) == kv.KV_EUNSUPPORTED
+    s = _fake_ring()
+    s.k_codes = 0
+    assert L.kv_ring_init(ctypes.byref(s)) == kv.KV_EINVAL
+    s = _fake_ring()
+    s.k_codes = 0x100001                                             # misaligned
+    assert L.kv_ring_init(ctypes.byref(s)) == kv.KV_EINVAL
+    s = _fake_ring()
+    assert L.kv_ring_init(ctypes.byref(s)) in (kv.KV_ECUDA, kv.KV_EUNSUPPORTED)  # no GPU here
+    assert s.initialized == 0
+
+
+def test_calls_on_uninitialised_ring_are_refused(L):
+    s = kv.kv_ring_t()
+    assert L.kv_ring_commit(ctypes.byref(s)) == kv.KV_ESTATE
+    assert L.kv_ring_write(ctypes.byref(s), 16, 16, 1, 1, 0, None) == kv.KV_ESTATE
+    assert L.kv_ring_delta_rotate(ctypes.byref(s), 3, None) == kv.KV_ESTATE
+    assert L.chunk_attention(ctypes.byref(s), 16, 1, 0, 0, None, None, 1.0, 16, None, 0,
+                             None) == kv.KV_ESTATE
+
+
+def test_write_validation_before_launch(L):
+    s = _fake_ring()
+    r = ctypes.byref(s)
+    assert L.kv_ring_write(r, 16, 16, 1, 257, 0, None) == kv.KV_ERANGE   # n > C
+    assert L.kv_ring_write(r, 16, 16, 1, 0, 0, None) == kv.KV_ERANGE
+    assert L.kv_ring_write(r, 16, 16, 3, 8, 0, None) == kv.KV_EINVAL     # dtype
+    assert L.kv_ring_write(r, 16, 16, 1, 8, 4, None) == kv.KV_EINVAL     # flag
+    assert L.kv_ring_write(r, 17, 16, 1, 8, 0, None) == kv.KV_EINVAL     # misaligned
+    assert L.kv_ring_write(r, None, 16, 1, 8, 0, None) == kv.KV_EINVAL
+    s.next_pos = 4090                                                    # past the table
+    assert L.kv_ring_write(r, 16, 16, 1, 8, 0, None) == kv.KV_ERANGE
+    s.next_pos = 0
+    s.pending = 32
+    assert L.kv_ring_write(r, 16, 16, 1, 16, 0, None) == kv.KV_ESTATE    # shorter rewrite
+    assert s.pending == 32
+
+
+def test_commit_matches_the_oracle_ring_arithmetic(L, orc):
+    s = _fake_ring(C=100)
+    o = orc.OracleRing(100, 1, 64)
+    for n in (30, 30, 30, 30, 7, 100, 1, 99):
+        s.pending = n
+        o._s.pending = n
+        assert L.kv_ring_commit(ctypes.byref(s)) == kv.KV_OK
+        o.commit()
+        assert (s.write_slot, s.live, s.pending, s.next_pos) == o.state()
+    s.live = 101
+    assert L.kv_ring_commit(ctypes.byref(s)) == kv.KV_ESTATE
+
+
+def test_delta_rotate_host_logic(L):
+    s = _fake_ring()
+    r = ctypes.byref(s)
+    s.next_pos = 500
+    assert L.kv_ring_delta_rotate(r, -128, None) == kv.KV_OK           # empty ring: no launch
+    assert s.next_pos == 372
+    assert L.kv_ring_delta_rotate(r, 2 ** 31, None) == kv.KV_ERANGE
+    assert L.kv_ring_delta_rotate(r, -(2 ** 31) - 400, None) == kv.KV_ERANGE
+    assert s.next_pos == 372
+
+
+def test_attention_validation_before_launch(L):
+    s = _fake_ring()
+    s.live = 64
+    r = ctypes.byref(s)
+    ok_args = (r, 16, 8, 0, 8, None, None, 0.125, 16, None)
+    assert L.chunk_attention(*ok_args[:1], 16, 0, 0, 0, None, None, 0.125, 16, None, 0,
+                             None) == kv.KV_OK                            # n_q = 0: no launch
+    assert L.chunk_attention(*ok_args, 1, None) == kv.KV_EINVAL           # flags
+    assert L.chunk_attention(r, 16, 8, 0, 65, None, None, 0.125, 16, None, 0,
+                             None) == kv.KV_ERANGE                        # n_current > valid
+    assert L.chunk_attention(r, 16, 8, 4090, 8, None, None, 0.125, 16, None, 0,
+                             None) == kv.KV_ERANGE                        # q positions
+    assert L.chunk_attention(r, 16, 8, 0, 8, None, None, 0.0, 16, None, 0,
+                             None) == kv.KV_EINVAL                        # scale
+    bad = kv.kv_cache_bias_t(float("nan"))
+    assert L.chunk_attention(r, 16, 8, 0, 8, None, ctypes.byref(bad), 0.125, 16, None, 0,
+                             None) == kv.KV_EINVAL
+    m = kv.kv_block_mask_t(0, 1, 1, 1)
+    assert L.chunk_attention(r, 16, 8, 0, 8, ctypes.byref(m), None, 0.125, 16, None, 0,
+                             None) == kv.KV_EINVAL
