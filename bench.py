@@ -1,0 +1,496 @@
+#!/usr/bin/env python
+"""Benchmark of the ring KV-cache attention hot path on B200.
+
+Workload (one "step"): the Runway-shaped chunk step -- 60 rings x 4 denoising passes =
+240 calls, each call a ring write of 757 new bf16 tokens (RoPE + e4m3 quantisation into
+a 5,788-slot ring, 40 heads x 128) followed by chunk attention of the 757 new queries
+over the whole ring (token-causal inside the new chunk, cache bias 0); the chunk is
+committed on the last pass.  Shapes from "Runway Characters: Serving a 57B Video
+Diffusion Transformer for Real-Time Conversation", abstract.  Inputs are seeded
+synthetic N(0,1)/sqrt(128) bf16 tensors, distinct for every ring and pass (5.6 GB, far
+above the 126 MB L2), resident in HBM before timing.
+
+Reported: value = microseconds per call (write + attention) over the whole step; per
+kernel averages from separate event-timed graphs of the same launches; the delta
+rotation timed on the long-stream shape (32,768 slots x 40 heads); the roofline of the
+attention kernel; an end-to-end number through the C ABI from pinned host buffers;
+and the fp64 CPU oracle timed on a bounded sample of the same workload.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "chunk-attn µs/call & % FP8 tensor peak; KV-write/rotate GB/s & % HBM"
+UNIT = "us/call"
+RINGS, PASSES = 60, 4
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "chunk_attn_traffic.txt")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"],
+                    bf16_sus=p.get("bf16_tflops_sustained", p["bf16_tflops"]), src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def attn_pairs_token_causal(n_new: int, C: int) -> int:
+    """Unmasked (query, key) pairs per head of one call: every history slot plus the
+    causal triangle of the new chunk."""
+    return n_new * (C - n_new) + n_new * (n_new + 1) // 2
+
+
+def write_bytes(n: int, H: int, D: int, in_bytes: int = 2) -> int:
+    """Algorithmic bytes of a ring write: K and V inputs read, codes, scales written."""
+    return n * H * (2 * D * in_bytes + 2 * D + 8)
+
+
+def rotate_bytes(slots: int, H: int, D: int) -> int:
+    return slots * H * 2 * (D + 4)
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def traffic_for(kernel_src: str):
+    """Per-launch DRAM bytes of the attention kernel from the committed ncu summary, or
+    None when the kernel source changed since the counters were taken."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = dict(line.split("=", 1) for line in f.read().split("\n") if "=" in line)
+        with open(kernel_src, "rb") as f:
+            h = hashlib.sha256(f.read()).hexdigest()[:16]
+        if rec.get("source_sha256_16", "").strip() != h:
+            return None
+        return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+class RunwayStep:
+    """60 full rings and the per-(ring, pass) inputs of one chunk step, on one GPU."""
+
+    def __init__(self, torch, kv, inputs, dev, seed: int):
+        self.torch, self.kv = torch, kv
+        w = inputs.RUNWAY
+        self.w = w
+        H, D, C, n = w.H, w.D, w.C, w.n
+        self.table = torch.from_numpy(kv.kv_rope_table_build(0, 64 * n, D)).to(dev)
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed)
+        sc = w.in_scale
+
+        def rnd():
+            return (torch.randn((n, H, D), generator=g, device=dev) * sc).to(torch.bfloat16)
+
+        self.rings = []
+        pre_k, pre_v = rnd(), rnd()
+        for r in range(RINGS):
+            ring = kv.KvRing(C, H, D, 0, 64 * n, device=dev, rope_table=self.table)
+            for _ in range(math.ceil(C / n)):          # fill: steady state, ring full
+                kv.kv_ring_write(ring, pre_k, pre_v, commit=True)
+            self.rings.append(ring)
+        self.q = [[rnd() for _ in range(PASSES)] for _ in range(RINGS)]
+        self.k = [[rnd() for _ in range(PASSES)] for _ in range(RINGS)]
+        self.v = [[rnd() for _ in range(PASSES)] for _ in range(RINGS)]
+        self.out = [torch.empty((n, H, D), dtype=torch.bfloat16, device=dev) for _ in range(RINGS)]
+        self.mask = (1, 1, 1, 1)
+        torch.cuda.synchronize()
+
+    def launch(self, parts=("write", "attn")):
+        kv, n = self.kv, self.w.n
+        for p in range(PASSES):
+            for r, ring in enumerate(self.rings):
+                if "write" in parts:
+                    kv.kv_ring_write(ring, self.k[r][p], self.v[r][p], commit=(p == PASSES - 1))
+                if "attn" in parts:
+                    kv.chunk_attention(ring, self.q[r][p], self._q_pos(ring, p, parts), n,
+                                       self.mask, 0.0, out=self.out[r], want_lse=False)
+
+    def _q_pos(self, ring, p, parts):
+        # the new chunk starts at next_pos while pending, and at next_pos - n once committed
+        if "write" in parts and p == PASSES - 1:
+            return ring.next_pos - self.w.n
+        return ring.next_pos
+
+    def graph(self, parts):
+        torch = self.torch
+        self.launch(parts)                   # eager warm-up outside capture
+        torch.cuda.synchronize()
+        states = [tuple(r.state()) for r in self.rings]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            self.launch(parts)
+        torch.cuda.synchronize()
+        for r, st in zip(self.rings, states):   # the graph replays this exact step
+            r.s.write_slot, r.s.live, r.s.pending, r.s.next_pos = st
+        return g
+
+
+def timed(torch, fn, reps: int, stream) -> float:
+    """Milliseconds per rep, CUDA events on the launching stream, synchronised both sides."""
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def max_over_ranks(torch, dist, x: float) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rotate_timing(torch, kv, inputs, dev, reps: int = 20) -> dict:
+    """Delta rotation of a full 32,768-slot x 40-head ring (the long-stream shape)."""
+    w = inputs.STRESS
+    ring = kv.KvRing(w.C, w.H, w.D, -4 * w.C, 4 * w.C, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(5)
+    for _ in range(w.C // w.n):
+        k = torch.randn((w.n, w.H, w.D), generator=g, device=dev).to(torch.bfloat16)
+        kv.kv_ring_write(ring, k, k, commit=True)
+    stream = torch.cuda.current_stream()
+    sign = [1]
+
+    def one():
+        kv.kv_ring_delta_rotate(ring, 7 * sign[0])
+        sign[0] = -sign[0]
+
+    for _ in range(3):
+        one()
+    ms = timed(torch, one, reps, stream)
+    nbytes = rotate_bytes(w.C, w.H, w.D)
+    del ring
+    return {"us_per_launch": ms * 1e3, "bytes_per_launch": nbytes,
+            "gbs": nbytes / (ms * 1e-3) / 1e9}
+
+
+def e2e_timing(torch, kv, step: RunwayStep, steps: int, stream) -> dict:
+    """Same step through the public API from pinned host buffers: every call copies its
+    q, k, v host->device and its output device->host inside the timed region."""
+    n_sets = 8
+    host = []
+    for s in range(n_sets):
+        host.append([[step.q[s][p].cpu().pin_memory(), step.k[s][p].cpu().pin_memory(),
+                      step.v[s][p].cpu().pin_memory()] for p in range(PASSES)])
+    dq = torch.empty_like(step.q[0][0])
+    dk = torch.empty_like(step.k[0][0])
+    dv = torch.empty_like(step.v[0][0])
+    outs = [torch.empty(step.out[0].shape, dtype=torch.bfloat16).pin_memory() for _ in range(n_sets)]
+    n = step.w.n
+
+    def one_step():
+        for p in range(PASSES):
+            for r, ring in enumerate(step.rings):
+                hq, hk, hv = host[r % n_sets][p]
+                dq.copy_(hq, non_blocking=True)
+                dk.copy_(hk, non_blocking=True)
+                dv.copy_(hv, non_blocking=True)
+                last = p == PASSES - 1
+                kv.kv_ring_write(ring, dk, dv, commit=last)
+                kv.chunk_attention(ring, dq, ring.next_pos - (n if last else 0), n, step.mask,
+                                   0.0, out=step.out[r], want_lse=False)
+                outs[r % n_sets].copy_(step.out[r], non_blocking=True)
+
+    one_step()
+    ms = timed(torch, one_step, steps, stream)
+    h2d = RINGS * PASSES * 3 * dq.numel() * dq.element_size()
+    d2h = RINGS * PASSES * step.out[0].numel() * 2
+    return {"ms_per_step": ms, "h2d": h2d, "d2h": d2h}
+
+
+class CpuBaseline:
+    """The fp64 oracle on the Runway shape: a full 5,788-slot ring (prefilled once), then
+    per sample one full 757-token x 40-head write plus attention of a seeded sample of
+    query rows (all 40 heads); attention time is scaled by 757/rows (rows are
+    independent, so the work scales exactly)."""
+
+    def __init__(self):
+        from kv_cache_attention_ring_b200 import inputs
+        from oracle import oracle
+        self.w = w = inputs.RUNWAY
+        self.o = oracle.OracleRing(w.C, w.H, w.D)
+        for ch in range(math.ceil(w.C / w.n)):
+            _, k, v = inputs.chunk_qkv(w, ch)
+            self.o.write(inputs.as_f32(k), inputs.as_f32(v), commit=True)
+        q, k, v = inputs.chunk_qkv(w, 99)
+        self.qf, self.kf, self.vf = inputs.as_f32(q), inputs.as_f32(k), inputs.as_f32(v)
+        self.rng = np.random.default_rng(0)
+        self.rows = None
+
+    def calibrate(self, target_s: float) -> int:
+        probe = np.sort(self.rng.choice(self.w.n, 8, replace=False))
+        t0 = time.perf_counter()
+        self.o.attention(self.qf, self.o.next_pos, self.w.n, (1, 1, 1, 1), 0.0, rows=probe)
+        per_row = (time.perf_counter() - t0) / len(probe)
+        self.rows = int(max(8, min(self.w.n, target_s / max(per_row, 1e-6))))
+        return self.rows
+
+    def sample(self) -> dict:
+        w, o = self.w, self.o
+        t0 = time.perf_counter()
+        o.write(self.kf, self.vf)
+        t_write = time.perf_counter() - t0
+        rows = np.sort(self.rng.choice(w.n, self.rows, replace=False))
+        t0 = time.perf_counter()
+        o.attention(self.qf, o.next_pos, w.n, (1, 1, 1, 1), 0.0, rows=rows)
+        t_attn = time.perf_counter() - t0
+        per_call_s = t_write + t_attn * w.n / self.rows
+        cores = int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
+        return {"value": per_call_s * 1e6, "unit": UNIT, "cores": cores, "kind": "oracle",
+                "sample": f"one full 757-token x 40-head write + attention of {self.rows} "
+                          f"seeded query rows x 40 heads over 5,788 slots, attention scaled "
+                          f"x{w.n}/{self.rows}",
+                "write_s": t_write, "attn_s": t_attn}
+
+
+def config_block(extra=None) -> dict:
+    c = {"workload": "runway_chunk_step: 60 rings x 4 passes = 240 x (ring write of 757 "
+                     "bf16 tokens + chunk attention over a 5,788-slot e4m3 ring), H=40, D=128, "
+                     "token-causal new chunk, cache_bias 0",
+         "calls_per_step": RINGS * PASSES, "heads": 40, "head_dim": 128, "ring_slots": 5788,
+         "new_tokens": 757, "l2": "inputs 5.6 GB + rings 3.7 GB per GPU, far above L2; no flush"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+def run_reference(args, rank: int, world: int):
+    """fp64 CPU oracle on the host cores (bounded sample per step)."""
+    if rank != 0:
+        return
+    cpu = CpuBaseline()
+    cpu.calibrate(target_s=4.0)
+    steps, base = [], None
+    for i in range(args.warmup + args.steps):
+        r = cpu.sample()
+        if i >= args.warmup:
+            steps.append(r["value"])
+            base = r
+    value = float(np.median(steps))
+    cb = dict(base)
+    cb["value"] = value
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": value * RINGS * PASSES / 1e3, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_block({"reference": "fp64 C oracle (OpenMP), bounded sample per "
+                                                 "step, scaled to a full call"}),
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    os.environ.setdefault("OMP_NUM_THREADS", str(len(os.sched_getaffinity(0))))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    import kv_cache_attention_ring_b200 as kv
+    from kv_cache_attention_ring_b200 import inputs
+    kv.lib()
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    peaks = load_peaks()
+
+    step = RunwayStep(torch, kv, inputs, dev, seed=1000 + 2 + rank)
+    g_full = step.graph(("write", "attn"))
+    g_attn = step.graph(("attn",))
+    g_write = step.graph(("write",))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(3, args.warmup)):
+        g_full.replay()
+    barrier()
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        g_full.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms_step = a.elapsed_time(b) / args.steps
+    barrier()
+    # per-kernel averages: the same launches, split into attention-only / write-only graphs
+    ms_attn = timed(torch, g_attn.replay, args.steps, stream) / (RINGS * PASSES)
+    ms_write = timed(torch, g_write.replay, args.steps, stream) / (RINGS * PASSES)
+    clk = clocks.stop()
+    ms_step = max_over_ranks(torch, dist, ms_step)
+    ms_attn = max_over_ranks(torch, dist, ms_attn)
+    ms_write = max_over_ranks(torch, dist, ms_write)
+    rot = rotate_timing(torch, kv, inputs, dev)
+    rot_us = max_over_ranks(torch, dist, rot["us_per_launch"])
+    e2e = e2e_timing(torch, kv, step, args.e2e_steps, stream)
+    e2e_ms = max_over_ranks(torch, dist, e2e["ms_per_step"])
+    timeouts = kv.kv_wait_timeout_count()
+    del g_full, g_attn, g_write
+
+    w = inputs.RUNWAY
+    calls = RINGS * PASSES * world
+    value = ms_step * 1e3 / (RINGS * PASSES * world)   # whole-job us per call
+    flop = 4 * w.D * attn_pairs_token_causal(w.n, w.C) * w.H
+    attn_tflops = flop / (ms_attn * 1e-3) / 1e12
+    wbytes = write_bytes(w.n, w.H, w.D)
+    write_gbs = wbytes / (ms_write * 1e-3) / 1e9
+    fp8_peak = 2.0 * peaks["bf16"]                       # nominal fp8:bf16 = 2:1
+    src = os.path.join(ROOT, "kv_cache_attention_ring_b200", "csrc", "chunk_attn.cu")
+    traffic = traffic_for(src)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 MMA on e4m3 cache (fp32 accumulate); write/rotate f32->e4m3",
+        "data": "synthetic",
+        "config": config_block({"parallelism": f"replicas{world}" if world > 1 else "1 GPU"}),
+        "attention": {"us_per_call": ms_attn * 1e3, "gflop_per_call": flop / 1e9,
+                      "tflops": attn_tflops,
+                      "frac_bf16_sustained": attn_tflops / peaks["bf16_sus"],
+                      "frac_fp8_dense": attn_tflops / fp8_peak,
+                      "fp8_peak_tflops": fp8_peak,
+                      "fp8_peak_note": f"{peaks['src']} bf16 burst x 2 (nominal ratio)"},
+        "write": {"us_per_call": ms_write * 1e3, "bytes_per_call": wbytes, "gbs": write_gbs,
+                  "frac_hbm": write_gbs / peaks["hbm"]},
+        "rotate": {"shape": "32768 slots x 40 heads x 128", "us_per_launch": rot_us,
+                   "bytes_per_launch": rot["bytes_per_launch"],
+                   "gbs": rot["bytes_per_launch"] / (rot_us * 1e-6) / 1e9,
+                   "frac_hbm": rot["bytes_per_launch"] / (rot_us * 1e-6) / 1e9 / peaks["hbm"]},
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peaks["bf16_sus"],
+                     "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16_sus"],
+                     "traffic": traffic, "kernel": "chunk_attn_kernel<128>",
+                     "peak_note": f"{peaks['src']} bf16 sustained (kernel timed inside a "
+                                  f"long graph); the contraction is bf16 x bf16 -> fp32"},
+        "e2e": {"value": e2e_ms * 1e3 / (RINGS * PASSES), "unit": UNIT,
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+        "gpu_launches": 2 * RINGS * PASSES * args.steps,
+        "clocks": clk,
+        "wait_timeouts": timeouts,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = CpuBaseline()
+        cpu.calibrate(target_s=12.0)
+        line["cpu_baseline"] = cpu.sample()
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

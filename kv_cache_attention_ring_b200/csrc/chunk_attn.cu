@@ -287,22 +287,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           mloc = fmaxf(mloc, s);
         }
       }
-      // lazy rescale: move the reference max only when it grows by more than 2^8
-      if (mloc > m_run + kRescaleLog2 || (m_run == -INFINITY && mloc > -INFINITY)) {
-        const float alpha = ex2(m_run - mloc);   // 0 when m_run = -inf
-        if (m_run != -INFINITY) {
-          l_run *= alpha;
+      // lazy rescale: move the reference max only when it grows by more than 2^8.
+      // tcgen05.ld/st are warp-collective, so the warp rescales together when any of its
+      // rows needs it (alpha = 1 for the others).
+      const bool move = mloc > m_run + kRescaleLog2 || (m_run == -INFINITY && mloc > -INFINITY);
+      const bool scale_o = move && m_run != -INFINITY;
+      const float alpha = scale_o ? ex2(m_run - mloc) : 1.f;
+      if (__any_sync(0xffffffffu, scale_o)) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(t_o + 32 * c, o);
-            tmem_wait_ld();
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(t_o + 32 * c, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-            tmem_st32(t_o + 32 * c, o);
-          }
-          tmem_wait_st();
+          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+          tmem_st32(t_o + 32 * c, o);
         }
+        tmem_wait_st();
+      }
+      if (move) {
+        l_run *= alpha;
         m_run = mloc;
       }
       const float mref = (m_run == -INFINITY) ? 0.f : m_run;
@@ -349,9 +353,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
   }
 
-  // ---- epilogue
-  if (gi < a.n_q) {
-    uint16_t* dst = a.out + ((size_t)gi * a.H + h) * D;
+  // ---- epilogue (TMEM loads by every lane: they are warp-collective)
+  {
+    const bool row_ok = gi < a.n_q;
+    uint16_t* dst = a.out + ((size_t)(row_ok ? gi : 0) * a.H + h) * D;
     const float inv_l = (ok && l_run > 0.f) ? 1.f / l_run : 0.f;
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
@@ -365,11 +370,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) x0 = x1 = __uint_as_float(0x7FC00000u);
         pk[j] = pack_bf16x2(x0, x1);
       }
-      uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+      if (row_ok) {
+        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) d4[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        for (int j = 0; j < 4; ++j)
+          d4[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+      }
     }
-    if (a.lse) {
+    if (row_ok && a.lse) {
       float v = (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
       if (!ok) v = __uint_as_float(0x7FC00000u);
       a.lse[(size_t)h * a.n_q + gi] = v;
