@@ -28,9 +28,10 @@ using namespace kvring;
 namespace {
 
 constexpr uint64_t kMagic = 0x6B7672696E673031ull;  // "kvring01"
-constexpr int kOpaqueTmapK = 0;                     // uint64 index of the K tensor map
-constexpr int kOpaqueTmapV = 16;                    // uint64 index of the V tensor map
-constexpr int kOpaqueMagic = 32;
+constexpr int kOpaqueTmapK = 0;                     // K codes, no swizzle
+constexpr int kOpaqueTmapV = 16;                    // V codes, no swizzle
+constexpr int kOpaqueTmapKsw = 32;                  // K codes, 128-byte swizzle (D = 128)
+constexpr int kOpaqueMagic = 48;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -87,9 +88,10 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D map over codes [H][C][D] bytes; box = D bytes x 128 slots x 1 head, no swizzle.
-// Slots >= C read as zero.
-int encode_codes_map(void* base, int H, int C, int D, uint64_t* dst) {
+// 3-D map over codes [H][C][D] bytes; box = D bytes x 128 slots x 1 head.  Slots >= C
+// read as zero.  swizzle128: rows land in shared memory with the 128-byte swizzle the
+// tensor core expects for a K-major operand (requires D = 128).
+int encode_codes_map(void* base, int H, int C, int D, uint64_t* dst, bool swizzle128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return KV_ECUDA;
   alignas(64) CUtensorMap m;
@@ -98,7 +100,8 @@ int encode_codes_map(void* base, int H, int C, int D, uint64_t* dst) {
   const cuuint32_t box[3] = {(cuuint32_t)D, 128u, 1u};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
   CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return KV_ECUDA;
   static_assert(sizeof(CUtensorMap) == 128, "CUtensorMap is 128 bytes");
@@ -150,11 +153,16 @@ int kv_ring_init(kv_ring_t* kv) {
     return KV_ECUDA;
   if (major != 10 || minor != 0) return KV_EUNSUPPORTED;
   int rc = encode_codes_map(kv->k_codes, kv->n_heads, kv->capacity, kv->head_dim,
-                            kv->opaque + kOpaqueTmapK);
+                            kv->opaque + kOpaqueTmapK, false);
   if (rc) return rc;
   rc = encode_codes_map(kv->v_codes, kv->n_heads, kv->capacity, kv->head_dim,
-                        kv->opaque + kOpaqueTmapV);
+                        kv->opaque + kOpaqueTmapV, false);
   if (rc) return rc;
+  if (kv->head_dim == 128) {
+    rc = encode_codes_map(kv->k_codes, kv->n_heads, kv->capacity, kv->head_dim,
+                          kv->opaque + kOpaqueTmapKsw, true);
+    if (rc) return rc;
+  }
   kv->opaque[kOpaqueMagic] = kMagic;
   kv->write_slot = 0;
   kv->live = 0;
@@ -279,7 +287,8 @@ int chunk_attention(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
   a.timeouts = timeout_counter();
   if (!a.timeouts) return KV_ECUDA;
   return launch_attention(a, kv->head_dim, kv->opaque + kOpaqueTmapK,
-                          kv->opaque + kOpaqueTmapV, static_cast<cudaStream_t>(stream));
+                          kv->opaque + kOpaqueTmapV, kv->opaque + kOpaqueTmapKsw,
+                          static_cast<cudaStream_t>(stream));
 }
 
 int kv_wait_timeout_count(uint32_t* host_count) {
