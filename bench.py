@@ -50,6 +50,10 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rings", type=int, default=RINGS,
+                    help="rings per step (60 = the Runway step; fewer for profiler captures)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the rotate, end-to-end and CPU legs (profiler captures)")
     return ap.parse_args()
 
 
@@ -157,8 +161,9 @@ def traffic_for(kernel_src: str):
 class RunwayStep:
     """60 full rings and the per-(ring, pass) inputs of one chunk step, on one GPU."""
 
-    def __init__(self, torch, kv, inputs, dev, seed: int):
+    def __init__(self, torch, kv, inputs, dev, seed: int, rings: int = RINGS):
         self.torch, self.kv = torch, kv
+        self.n_rings = rings
         w = inputs.RUNWAY
         self.w = w
         H, D, C, n = w.H, w.D, w.C, w.n
@@ -172,15 +177,15 @@ class RunwayStep:
 
         self.rings = []
         pre_k, pre_v = rnd(), rnd()
-        for r in range(RINGS):
+        for r in range(rings):
             ring = kv.KvRing(C, H, D, 0, 64 * n, device=dev, rope_table=self.table)
             for _ in range(math.ceil(C / n)):          # fill: steady state, ring full
                 kv.kv_ring_write(ring, pre_k, pre_v, commit=True)
             self.rings.append(ring)
-        self.q = [[rnd() for _ in range(PASSES)] for _ in range(RINGS)]
-        self.k = [[rnd() for _ in range(PASSES)] for _ in range(RINGS)]
-        self.v = [[rnd() for _ in range(PASSES)] for _ in range(RINGS)]
-        self.out = [torch.empty((n, H, D), dtype=torch.bfloat16, device=dev) for _ in range(RINGS)]
+        self.q = [[rnd() for _ in range(PASSES)] for _ in range(rings)]
+        self.k = [[rnd() for _ in range(PASSES)] for _ in range(rings)]
+        self.v = [[rnd() for _ in range(PASSES)] for _ in range(rings)]
+        self.out = [torch.empty((n, H, D), dtype=torch.bfloat16, device=dev) for _ in range(rings)]
         self.mask = (1, 1, 1, 1)
         torch.cuda.synchronize()
 
@@ -288,8 +293,8 @@ def e2e_timing(torch, kv, step: RunwayStep, steps: int, stream) -> dict:
 
     one_step()
     ms = timed(torch, one_step, steps, stream)
-    h2d = RINGS * PASSES * 3 * dq.numel() * dq.element_size()
-    d2h = RINGS * PASSES * step.out[0].numel() * 2
+    h2d = step.n_rings * PASSES * 3 * dq.numel() * dq.element_size()
+    d2h = step.n_rings * PASSES * step.out[0].numel() * 2
     return {"ms_per_step": ms, "h2d": h2d, "d2h": d2h}
 
 
@@ -403,7 +408,8 @@ def main():
     stream = torch.cuda.current_stream()
     peaks = load_peaks()
 
-    step = RunwayStep(torch, kv, inputs, dev, seed=1000 + 2 + rank)
+    step = RunwayStep(torch, kv, inputs, dev, seed=1000 + 2 + rank, rings=args.rings)
+    R = args.rings
     g_full = step.graph(("write", "attn"))
     g_attn = step.graph(("attn",))
     g_write = step.graph(("write",))
@@ -428,22 +434,26 @@ def main():
     ms_step = a.elapsed_time(b) / args.steps
     barrier()
     # per-kernel averages: the same launches, split into attention-only / write-only graphs
-    ms_attn = timed(torch, g_attn.replay, args.steps, stream) / (RINGS * PASSES)
-    ms_write = timed(torch, g_write.replay, args.steps, stream) / (RINGS * PASSES)
+    ms_attn = timed(torch, g_attn.replay, args.steps, stream) / (R * PASSES)
+    ms_write = timed(torch, g_write.replay, args.steps, stream) / (R * PASSES)
     clk = clocks.stop()
     ms_step = max_over_ranks(torch, dist, ms_step)
     ms_attn = max_over_ranks(torch, dist, ms_attn)
     ms_write = max_over_ranks(torch, dist, ms_write)
-    rot = rotate_timing(torch, kv, inputs, dev)
+    if args.no_extras:
+        rot = {"us_per_launch": float("nan"), "bytes_per_launch": 0}
+        e2e = {"ms_per_step": float("nan"), "h2d": 0, "d2h": 0}
+    else:
+        rot = rotate_timing(torch, kv, inputs, dev)
+        e2e = e2e_timing(torch, kv, step, args.e2e_steps, stream)
     rot_us = max_over_ranks(torch, dist, rot["us_per_launch"])
-    e2e = e2e_timing(torch, kv, step, args.e2e_steps, stream)
     e2e_ms = max_over_ranks(torch, dist, e2e["ms_per_step"])
     timeouts = kv.kv_wait_timeout_count()
     del g_full, g_attn, g_write
 
     w = inputs.RUNWAY
-    calls = RINGS * PASSES * world
-    value = ms_step * 1e3 / (RINGS * PASSES * world)   # whole-job us per call
+    value = ms_step * 1e3 / (R * PASSES)              # us per call (each rank: R*4 calls)
+    value = value / world                              # whole job: world x the calls
     flop = 4 * w.D * attn_pairs_token_causal(w.n, w.C) * w.H
     attn_tflops = flop / (ms_attn * 1e-3) / 1e12
     wbytes = write_bytes(w.n, w.H, w.D)
@@ -457,7 +467,8 @@ def main():
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16 MMA on e4m3 cache (fp32 accumulate); write/rotate f32->e4m3",
         "data": "synthetic",
-        "config": config_block({"parallelism": f"replicas{world}" if world > 1 else "1 GPU"}),
+        "config": config_block({"parallelism": f"replicas{world}" if world > 1 else "1 GPU",
+                                "rings": R, "calls_per_step": R * PASSES}),
         "attention": {"us_per_call": ms_attn * 1e3, "gflop_per_call": flop / 1e9,
                       "tflops": attn_tflops,
                       "frac_bf16_sustained": attn_tflops / peaks["bf16_sus"],
@@ -475,13 +486,13 @@ def main():
                      "traffic": traffic, "kernel": "chunk_attn_kernel<128>",
                      "peak_note": f"{peaks['src']} bf16 sustained (kernel timed inside a "
                                   f"long graph); the contraction is bf16 x bf16 -> fp32"},
-        "e2e": {"value": e2e_ms * 1e3 / (RINGS * PASSES), "unit": UNIT,
+        "e2e": {"value": e2e_ms * 1e3 / (R * PASSES) / world, "unit": UNIT,
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
-        "gpu_launches": 2 * RINGS * PASSES * args.steps,
+        "gpu_launches": 2 * R * PASSES * args.steps,
         "clocks": clk,
         "wait_timeouts": timeouts,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.no_extras:
         cpu = CpuBaseline()
         cpu.calibrate(target_s=12.0)
         line["cpu_baseline"] = cpu.sample()

@@ -13,16 +13,20 @@
 //    conversion of K).  The rotated bf16 query row is split exactly into
 //    q = r * (hi + lo), hi, lo e4m3, r a power of two (8 significant bits = 4 + 4), so
 //    S' = hi.K + lo.K is one f32 accumulation of 2*D/32 kind::f8f6f4 MMAs and
-//    s = r * ks * scale * S' (+ bias).
-//  * P.V runs in bf16: V codes are converted (exactly) to bf16 in shared memory by four
-//    converter warps; P = p * vs (bf16) is written to tensor memory over the S columns
-//    it came from and read from there as the A operand.
+//    s = r * ks * scale * S' (+ bias).  r is per query row, so a row's result never
+//    depends on other rows (later blocks cannot change earlier ones, bit for bit).
+//  * P.V runs in bf16: four converter warps turn V codes into bf16(e4m3(vc) * vs) in
+//    shared memory (one bf16 rounding, 2^-9 relative); P = bf16(p) is written to tensor
+//    memory over the S columns it came from and read from there as the A operand.
+//  * Softmax: two passes over the S tile in TMEM (row maximum, then 2^(t - m)), with
+//    paired fp32 instructions (f32x2) so the exponentials on the MUFU unit set the pace.
 //  * Tensor memory (512 columns): S0/P0 [0,128), S1/P1 [128,256), O0 [256,384),
 //    O1 [384,512).  MMA issue order per key tile j:
 //      S0(j) PV1(j-1) S1(j) PV0(j)
 //    so softmax of tile g overlaps the tensor core working on the other tile.
-//  * Warps: 0 TMA producer, 1 MMA issuer, 2-5 V converters + per-key info, 6-9 softmax
-//    of tile 0, 10-13 softmax of tile 1 (thread = query row = TMEM lane).
+//  * Warps: 0 TMA producer, 1 MMA issuer, 2-3 V converters + per-key info, 4-7 softmax
+//    of tile 0, 8-11 softmax of tile 1 (thread = query row = TMEM lane).  12 warps leave
+//    168 registers per thread, enough to hold a whole 128-column S row.
 //  * Online softmax in log2 units with lazy rescale of O (only when the row maximum
 //    grows by more than 8, i.e. a factor 256); the final O / l is exact regardless.
 //  * Keys are visited in physical slot order in 128-slot tiles; the ring wrap costs
@@ -47,8 +51,9 @@ constexpr int NK = 3;                   // K code stages
 constexpr int NV = 2;                   // V code stages
 constexpr int NB = 2;                   // V bf16 buffers
 constexpr int NI = 4;                   // per-key info stages
-constexpr int kThreads = 14 * 32;
-constexpr int kWarpTma = 0, kWarpMma = 1, kWarpConv = 2, kWarpSoft = 6;
+constexpr int kThreads = 12 * 32;
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpConv = 2, kWarpSoft = 4;
+constexpr int kConvThreads = 64;
 constexpr uint32_t kPanel = 128u * 128u;   // one 128-row x 128-byte swizzled panel
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kInvalidTok = 0x7FFFFFFF;
@@ -57,7 +62,6 @@ struct Info {             // per key slot of one tile
   float kscl[BN];         // ks * softmax_scale * log2(e); 0 for invalid slots
   float kb[BN];           // additive log2 logit: bias (history), 0 (current), -inf (invalid)
   int ktok[BN];           // -1 history, token index (current), kInvalidTok (invalid)
-  float vscl[BN];         // vs; 0 for invalid slots
   int flag[4];            // per converter warp: tile holds current or invalid keys
 };
 
@@ -71,7 +75,8 @@ struct Layout {
   static constexpr uint32_t bars = info + NI * sizeof(Info);    // mbarriers
   static constexpr int kNumBars = 2 * NK + 2 * NV + 2 * NB + 2 * NI + 2 + 2 + 1;
   static constexpr uint32_t misc = bars + 8 * kNumBars;         // tmem addr, abort flag
-  static constexpr uint32_t bytes = misc + 16 + 1024;           // + alignment slack
+  static constexpr uint32_t vsc = misc + 16;                    // float[BN]: converters only
+  static constexpr uint32_t bytes = vsc + 4 * BN + 1024;        // + alignment slack
 };
 static_assert(Layout::bytes <= 232448, "shared memory budget");
 
@@ -104,26 +109,22 @@ __device__ __forceinline__ float e4m3_value(uint32_t code) {
   return f16x2_to_float2(e4m3x2_to_f16x2((uint16_t)code)).x;
 }
 
-__device__ __forceinline__ bool tile_valid(int64_t t, int64_t C, int64_t newest, int64_t nv) {
+__device__ __forceinline__ bool tile_valid(int t, int C, int newest, int nv) {
   if (nv <= 0) return false;
   if (nv >= C) return true;
-  const int64_t a = t * BN, b = min(C, a + BN);
-  int64_t first = newest - nv + 1;
+  const int a = t * BN, b = min(C, a + BN);
+  int first = newest - nv + 1;
   if (first >= 0) return a <= newest && b > first;
   first += C;
   return (b > first) || (a <= newest);
 }
 
 // Next physical tile index >= t holding a valid slot (n_tiles if none).
-__device__ __forceinline__ int64_t next_tile(int64_t t, int64_t n_tiles, int64_t C,
-                                             int64_t newest, int64_t nv) {
+__device__ __forceinline__ int next_tile(int t, int n_tiles, int C, int newest, int nv) {
   while (t < n_tiles && !tile_valid(t, C, newest, nv)) ++t;
   return t;
 }
 
-// Rotate query row gi at position q_pos0 + gi, round to bf16, split exactly into
-// r * (hi + lo) with e4m3 hi/lo and a power-of-two r; write hi/lo into the swizzled
-// K-major operand rows.  Returns r (0 rows beyond n_q give r = 1 and zero codes).
 // bf16-rounded rotation of 8 consecutive elements (chunk c) of query row gi.
 __device__ __forceinline__ void q_rot8(const AttnArgs& a, int gi, int h, int c, float (&y)[8]) {
   const uint4 raw = __ldg(reinterpret_cast<const uint4*>(a.q + ((size_t)gi * a.H + h) * D) + c);
@@ -144,31 +145,31 @@ __device__ __forceinline__ void q_rot8(const AttnArgs& a, int gi, int h, int c, 
   }
 }
 
-// Rotate query row gi at position q_pos0 + gi, round to bf16, split exactly into
-// r * (hi + lo) with e4m3 hi/lo and a power-of-two r; write hi/lo into the swizzled
-// K-major operand rows.  Returns r.  Rows beyond n_q get zero codes and r = 1.
-__device__ __forceinline__ float q_prologue(const AttnArgs& a, int gi, int h, uint8_t* qhi,
-                                            uint8_t* qlo, int row) {
-  const bool live = gi < a.n_q;
+// Exponent k of the smallest power of two r = 2^k with max|bf16(RoPE(q_gi))| / r <= 448
+// (448 = 1.75 * 2^8).  Rows beyond n_q or all-zero rows return INT_MIN.
+__device__ __forceinline__ int q_exponent(const AttnArgs& a, int gi, int h) {
+  if (gi >= a.n_q) return INT_MIN;
   float amax = 0.f;
-  if (live) {
 #pragma unroll 4
-    for (int c = 0; c < D / 8; ++c) {
-      float y[8];
-      q_rot8(a, gi, h, c, y);
+  for (int c = 0; c < D / 8; ++c) {
+    float y[8];
+    q_rot8(a, gi, h, c, y);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(y[e]));
-    }
+    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(y[e]));
   }
-  // smallest power of two r with amax / r <= 448 (448 = 1.75 * 2^8), clamped to normals
-  int k = 0;
-  if (amax > 0.f && isfinite(amax)) {
-    int e;
-    const float m = frexpf(amax, &e);        // amax = m * 2^e, m in [0.5, 1)
-    k = (e - 1) - 8 + (m > 0.875f ? 1 : 0);
-    k = max(-126, min(127, k));
-  }
-  const float r = ldexpf(1.f, k), inv_r = ldexpf(1.f, -k);
+  if (!(amax > 0.f) || !isfinite(amax)) return INT_MIN;
+  int e;
+  const float m = frexpf(amax, &e);          // amax = m * 2^e, m in [0.5, 1)
+  return (e - 1) - 8 + (m > 0.875f ? 1 : 0);
+}
+
+// Split bf16(RoPE(q_gi)) / 2^k exactly into e4m3 hi + lo (4 + 4 significant bits; exact
+// for elements within 2^10 of the tile's largest) and write both into the swizzled
+// K-major operand rows.  Rows beyond n_q get zero codes.
+__device__ __forceinline__ void q_split(const AttnArgs& a, int gi, int h, int k, uint8_t* qhi,
+                                        uint8_t* qlo, int row) {
+  const bool live = gi < a.n_q;
+  const float inv_r = ldexpf(1.f, -k);
 #pragma unroll 2
   for (int c = 0; c < D / 16; ++c) {
     float y[16];
@@ -204,7 +205,6 @@ __device__ __forceinline__ float q_prologue(const AttnArgs& a, int gi, int h, ui
     *reinterpret_cast<uint4*>(qhi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
     *reinterpret_cast<uint4*>(qlo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
   }
-  return r;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -221,8 +221,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.y;
   const int q0 = blockIdx.x * BM;
-  const int64_t C = a.C;
-  const int64_t n_tiles = (C + BN - 1) / BN;
+  const int C = a.C;
+  const int n_tiles = (C + BN - 1) / BN;
+  const int newest = (int)a.newest_slot, n_valid = (int)a.n_valid;
 
   if (warp == 0) {
     tmem_alloc(tmem_slot, 512);
@@ -230,9 +231,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid == 32) {
     for (int s = 0; s < NK; ++s) { mbar_init(bars.kfull(s), 1); mbar_init(bars.kempty(s), 1); }
-    for (int s = 0; s < NV; ++s) { mbar_init(bars.vfull(s), 1); mbar_init(bars.vempty(s), 128); }
-    for (int s = 0; s < NB; ++s) { mbar_init(bars.vbfull(s), 128); mbar_init(bars.vbempty(s), 1); }
-    for (int s = 0; s < NI; ++s) { mbar_init(bars.ifull(s), 128); mbar_init(bars.iempty(s), 256); }
+    for (int s = 0; s < NV; ++s) { mbar_init(bars.vfull(s), 1); mbar_init(bars.vempty(s), kConvThreads); }
+    for (int s = 0; s < NB; ++s) { mbar_init(bars.vbfull(s), kConvThreads); mbar_init(bars.vbempty(s), 1); }
+    for (int s = 0; s < NI; ++s) { mbar_init(bars.ifull(s), kConvThreads); mbar_init(bars.iempty(s), 256); }
     for (int g = 0; g < 2; ++g) { mbar_init(bars.sfull(g), 1); mbar_init(bars.pfull(g), 128); }
     mbar_init(bars.ofinal(), 1);
     *abort_flag = 0;
@@ -244,12 +245,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // Q prologue by the softmax warps: thread = query row = TMEM lane
-  const int g = (warp - kWarpSoft) >> 2;                 // softmax tile (valid for warps 6..13)
+  const int g = (warp - kWarpSoft) >> 2;                 // softmax tile (valid for warps 4..11)
   const int row_in_tile = 32 * (warp & 3) + lane;        // TMEM lane of this thread
   const int gi = q0 + 128 * g + row_in_tile;
+  // per-row power-of-two query scale r = 2^k
   float rowmul = 1.f;
-  if (warp >= kWarpSoft)
-    rowmul = q_prologue(a, gi, h, sm + Layout::qhi, sm + Layout::qlo, 128 * g + row_in_tile);
+  if (warp >= kWarpSoft) {
+    int k = q_exponent(a, gi, h);
+    k = (k == INT_MIN) ? 0 : max(-126, min(127, k));
+    q_split(a, gi, h, k, sm + Layout::qhi, sm + Layout::qlo, 128 * g + row_in_tile);
+    rowmul = ldexpf(1.f, k);
+  }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -266,8 +272,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kWarpTma) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int64_t t = next_tile(0, n_tiles, C, a.newest_slot, a.n_valid);
-      for (int j = 0; t < n_tiles; ++j, t = next_tile(t + 1, n_tiles, C, a.newest_slot, a.n_valid)) {
+      int t = next_tile(0, n_tiles, C, newest, n_valid);
+      for (int j = 0; t < n_tiles; ++j, t = next_tile(t + 1, n_tiles, C, newest, n_valid)) {
         const int sk = j % NK, rk = j / NK;
         if (rk > 0 && !wait(bars.kempty(sk), (rk - 1) & 1)) break;
         mbar_arrive_expect_tx(bars.kfull(sk), BN * D);
@@ -308,8 +314,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       int j = 0;
       bool ok = true;
-      for (int64_t t = next_tile(0, n_tiles, C, a.newest_slot, a.n_valid); t < n_tiles;
-           t = next_tile(t + 1, n_tiles, C, a.newest_slot, a.n_valid), ++j) {
+      for (int t = next_tile(0, n_tiles, C, newest, n_valid); t < n_tiles;
+           t = next_tile(t + 1, n_tiles, C, newest, n_valid), ++j) {
         const int sk = j % NK;
         if (!(ok = wait(bars.kfull(sk), (j / NK) & 1))) break;
         tc_fence_after();
@@ -339,24 +345,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < kWarpSoft) {
     // ------------------------------------------------------------ converters + key info
-    const int ct = tid - 32 * kWarpConv;          // 0..127
-    int j = 0;
-    for (int64_t t = next_tile(0, n_tiles, C, a.newest_slot, a.n_valid); t < n_tiles;
-         t = next_tile(t + 1, n_tiles, C, a.newest_slot, a.n_valid), ++j) {
+    // 64 threads; thread ct owns keys ct and ct + 64 of every tile.  The K/V scales of the
+    // next tile are loaded while the current tile's V codes are converted.
+    const int ct = tid - 32 * kWarpConv;          // 0..63
+    float* vsc = reinterpret_cast<float*>(sm + Layout::vsc);   // V scales of the tile
+    auto load_scales = [&](int tt, float (&ks)[2], float (&vs)[2]) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int slot = tt * BN + ct + 64 * e;
+        const bool in_ring = tt < n_tiles && slot < C;
+        ks[e] = in_ring ? __ldg(a.k_scale + (size_t)h * C + slot) : 0.f;
+        vs[e] = in_ring ? __ldg(a.v_scale + (size_t)h * C + slot) : 0.f;
+      }
+    };
+    float pks[2], pvs[2];
+    int t = next_tile(0, n_tiles, C, newest, n_valid);
+    load_scales(t, pks, pvs);
+    for (int j = 0; t < n_tiles; ++j) {
+      const int t_next = next_tile(t + 1, n_tiles, C, newest, n_valid);
       const int si = j % NI;
       bool ok = j < NI || wait(bars.iempty(si), ((j / NI) - 1) & 1);
-      if (!named_bar_and(1, 128, ok)) break;       // uniform decision across converters
+      if (!named_bar_and(1, kConvThreads, ok)) break;   // uniform decision across converters
       Info& in = info[si];
-      {
-        const int64_t slot = t * BN + ct;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int key = ct + 64 * e;
+        const int slot = t * BN + key;
         float ksv = 0.f, kbv = -INFINITY, vsv = 0.f;
         int tok = kInvalidTok;
         if (slot < C) {
-          int64_t age = a.newest_slot - slot;
+          int age = newest - slot;
           if (age < 0) age += C;
-          if (age < a.n_valid) {
-            ksv = a.k_scale[(size_t)h * C + slot] * a.score_scale_log2;
-            vsv = a.v_scale[(size_t)h * C + slot];
+          if (age < n_valid) {
+            ksv = pks[e] * a.score_scale_log2;
+            vsv = pvs[e];
             if (age < a.n_current) {
               kbv = 0.f;
               tok = (int)(a.n_current - 1 - age);
@@ -366,25 +388,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        in.kscl[ct] = ksv;
-        in.kb[ct] = kbv;
-        in.ktok[ct] = tok;
-        in.vscl[ct] = vsv;
+        in.kscl[key] = ksv;
+        in.kb[key] = kbv;
+        in.ktok[key] = tok;
+        vsc[key] = vsv;
         const unsigned special = __ballot_sync(0xffffffffu, tok != -1);
-        if (lane == 0) in.flag[ct >> 5] = special != 0;
+        if (lane == 0) in.flag[2 * e + (ct >> 5)] = special != 0;
       }
-      named_bar(1, 128);                               // info of this tile complete
+      load_scales(t_next, pks, pvs);                   // prefetch for the next tile
+      named_bar(1, kConvThreads);                      // info of this tile complete
       mbar_arrive(bars.ifull(si));
       const int sv = j % NV, b = j % NB;
       ok = wait(bars.vfull(sv), (j / NV) & 1);
       ok = ok && (j < NB || wait(bars.vbempty(b), ((j / NB) - 1) & 1));
-      if (!named_bar_and(2, 128, ok)) break;
+      if (!named_bar_and(2, kConvThreads, ok)) break;
       const uint8_t* vc = sm + Layout::vcode + sv * BN * D;
       uint8_t* vb = sm + Layout::vbf + b * 2 * kPanel;
 #pragma unroll 4
-      for (int idx = ct; idx < BN * D / 16; idx += 128) {
+      for (int idx = ct; idx < BN * D / 16; idx += kConvThreads) {
         const int row = idx >> 3, c = idx & 7;
         uint4 cv = *reinterpret_cast<const uint4*>(vc + row * D + 16 * c);
+        const float vsr = vsc[row];                    // 0 for invalid slots
         if (in.ktok[row] == kInvalidTok) cv = make_uint4(0u, 0u, 0u, 0u);
         const uint32_t w[4] = {cv.x, cv.y, cv.z, cv.w};
         uint32_t o[8];
@@ -392,8 +416,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 4; ++i) {
           const float2 lo = f16x2_to_float2(e4m3x2_to_f16x2((uint16_t)(w[i] & 0xFFFFu)));
           const float2 hi = f16x2_to_float2(e4m3x2_to_f16x2((uint16_t)(w[i] >> 16)));
-          o[2 * i] = pack_bf16x2(lo.x, lo.y);
-          o[2 * i + 1] = pack_bf16x2(hi.x, hi.y);
+          o[2 * i] = pack_bf16x2(lo.x * vsr, lo.y * vsr);
+          o[2 * i + 1] = pack_bf16x2(hi.x * vsr, hi.y * vsr);
         }
         *reinterpret_cast<uint4*>(vb + sw128_offset(row, 16 * c, kPanel)) =
             make_uint4(o[0], o[1], o[2], o[3]);
@@ -403,6 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       mbar_arrive(bars.vbfull(b));
       mbar_arrive(bars.vempty(sv));
+      t = t_next;
     }
   } else {
     // ------------------------------------------------------------ softmax of tile g
@@ -417,47 +442,102 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     float m_run = -INFINITY, l_run = 0.f;
     int j = 0;
-    for (int64_t t = next_tile(0, n_tiles, C, a.newest_slot, a.n_valid); t < n_tiles;
-         t = next_tile(t + 1, n_tiles, C, a.newest_slot, a.n_valid), ++j) {
+    for (int t = next_tile(0, n_tiles, C, newest, n_valid); t < n_tiles;
+         t = next_tile(t + 1, n_tiles, C, newest, n_valid), ++j) {
       const int si = j % NI;
       bool ok = wait(bars.sfull(g), j & 1) && wait(bars.ifull(si), (j / NI) & 1);
       if (!__all_sync(0xffffffffu, ok)) break;     // TMEM access below is warp-collective
       tc_fence_after();
       const Info& in = info[si];
+      const float* kscl = in.kscl;
+      const uint64_t r2 = f2_pack(rowmul, rowmul);
       const bool special = (in.flag[0] | in.flag[1] | in.flag[2] | in.flag[3]) != 0;
-      // pass 1: row maximum of this tile (log2 units)
-      float mloc = -INFINITY;
+      // the whole 128-column S row of this thread: one load, one wait
+      uint32_t sr[128];
+      tmem_ld128(t_s, sr);
+      tmem_wait_ld();
+      // pass 1, in place: fast tiles keep u = S * kscl, masked tiles t = u * r + kb (or
+      // -inf); track the row maximum.  Pass 2 then needs no per-key data.
+      float m0 = -INFINITY, m1 = -INFINITY;
+      const float4* k4 = reinterpret_cast<const float4*>(kscl);
       if (!special) {
-        float umax = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t raw[32];
-          tmem_ld32(t_s + 32 * c, raw);
-          tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 32; ++k) umax = fmaxf(umax, __uint_as_float(raw[k]) * in.kscl[32 * c + k]);
+        for (int q = 0; q < 32; ++q) {
+          const float4 ks = k4[q];
+          float u0, u1, u2, u3;
+          f2_unpack(f2_mul(f2_pack(__uint_as_float(sr[4 * q]), __uint_as_float(sr[4 * q + 1])),
+                           f2_pack(ks.x, ks.y)), u0, u1);
+          f2_unpack(f2_mul(f2_pack(__uint_as_float(sr[4 * q + 2]), __uint_as_float(sr[4 * q + 3])),
+                           f2_pack(ks.z, ks.w)), u2, u3);
+          sr[4 * q] = __float_as_uint(u0);
+          sr[4 * q + 1] = __float_as_uint(u1);
+          sr[4 * q + 2] = __float_as_uint(u2);
+          sr[4 * q + 3] = __float_as_uint(u3);
+          m0 = max3f(m0, u0, u1);
+          m1 = max3f(m1, u2, u3);
         }
-        mloc = fmaf(umax, rowmul, a.bias_log2);
       } else {
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t raw[32];
-          tmem_ld32(t_s + 32 * c, raw);
-          tmem_wait_ld();
+        const float4* b4 = reinterpret_cast<const float4*>(in.kb);
+        const int4* t4 = reinterpret_cast<const int4*>(in.ktok);
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const int key = 32 * c + k;
-            const float tv = fmaf(__uint_as_float(raw[k]) * in.kscl[key], rowmul, in.kb[key]);
-            mloc = fmaxf(mloc, in.ktok[key] < lim ? tv : -INFINITY);
-          }
+        for (int q = 0; q < 32; ++q) {
+          const float4 ks = k4[q], kb = b4[q];
+          const int4 tk = t4[q];
+          float u0, u1, u2, u3;
+          f2_unpack(f2_fma(f2_mul(f2_pack(__uint_as_float(sr[4 * q]), __uint_as_float(sr[4 * q + 1])),
+                                  f2_pack(ks.x, ks.y)), r2, f2_pack(kb.x, kb.y)), u0, u1);
+          f2_unpack(f2_fma(f2_mul(f2_pack(__uint_as_float(sr[4 * q + 2]), __uint_as_float(sr[4 * q + 3])),
+                                  f2_pack(ks.z, ks.w)), r2, f2_pack(kb.z, kb.w)), u2, u3);
+          u0 = tk.x < lim ? u0 : -INFINITY;
+          u1 = tk.y < lim ? u1 : -INFINITY;
+          u2 = tk.z < lim ? u2 : -INFINITY;
+          u3 = tk.w < lim ? u3 : -INFINITY;
+          sr[4 * q] = __float_as_uint(u0);
+          sr[4 * q + 1] = __float_as_uint(u1);
+          sr[4 * q + 2] = __float_as_uint(u2);
+          sr[4 * q + 3] = __float_as_uint(u3);
+          m0 = max3f(m0, u0, u1);
+          m1 = max3f(m1, u2, u3);
         }
       }
-      // lazy rescale of O (warp-collective TMEM access; alpha = 1 for rows that keep m)
+      const float mloc = special ? fmaxf(m0, m1) : fmaf(fmaxf(m0, m1), rowmul, a.bias_log2);
+      // lazy reference maximum: move m only when the tile maximum exceeds it by more than
+      // 2^8; O is rescaled after pass 2 (the S row is no longer live then)
       const bool move = mloc > m_run + kRescaleLog2 || (m_run == -INFINITY && mloc > -INFINITY);
       const bool scale_o = move && m_run != -INFINITY;
       const float alpha = scale_o ? ex2(m_run - mloc) : 1.f;
-      if (__any_sync(0xffffffffu, scale_o)) {
+      if (move) {
+        l_run *= alpha;
+        m_run = mloc;
+      }
+      // pass 2: p = 2^(t - m); P = bf16(p) written over the S columns (S is in registers)
+      const float mref = (m_run == -INFINITY) ? 0.f : m_run;
+      // fast tiles: t - m = u * r + (bias - m); masked tiles: t - m = t * 1 + (-m)
+      const float off = special ? -mref : a.bias_log2 - mref;
+      const uint64_t mul2 = special ? f2_pack(1.f, 1.f) : r2;
+      const uint64_t off2 = f2_pack(off, off);
+      uint64_t sum01 = f2_pack(0.f, 0.f), sum23 = sum01;
 #pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8) {
+          const int q = 8 * c + q8;
+          float t0, t1, t2, t3;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[4 * q]), __uint_as_float(sr[4 * q + 1])), mul2,
+                           off2), t0, t1);
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[4 * q + 2]), __uint_as_float(sr[4 * q + 3])), mul2,
+                           off2), t2, t3);
+          const float p0 = ex2(t0), p1 = ex2(t1), p2 = ex2(t2), p3 = ex2(t3);   // 2^-inf = 0
+          sum01 = f2_add(sum01, f2_pack(p0, p1));
+          sum23 = f2_add(sum23, f2_pack(p2, p3));
+          pk[2 * q8] = pack_bf16x2(p0, p1);
+          pk[2 * q8 + 1] = pack_bf16x2(p2, p3);
+        }
+        tmem_st16(t_s + 16 * c, pk);
+      }
+      if (__any_sync(0xffffffffu, scale_o)) {      // warp-collective TMEM access
+#pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
           tmem_ld32(t_o + 32 * c, o);
@@ -467,51 +547,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st32(t_o + 32 * c, o);
         }
       }
-      if (move) {
-        l_run *= alpha;
-        m_run = mloc;
-      }
-      // pass 2: p = 2^(t - m), P = p * vs (bf16) over the S columns already consumed
-      const float mref = (m_run == -INFINITY) ? 0.f : m_run;
-      float lsum = 0.f;
-      if (!special) {
-        const float off = a.bias_log2 - mref;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t raw[32], pk[16];
-          tmem_ld32(t_s + 32 * c, raw);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const int key = 32 * c + 2 * k;
-            const float p0 = ex2(fmaf(__uint_as_float(raw[2 * k]) * in.kscl[key], rowmul, off));
-            const float p1 = ex2(fmaf(__uint_as_float(raw[2 * k + 1]) * in.kscl[key + 1], rowmul, off));
-            lsum += p0 + p1;
-            pk[k] = pack_bf16x2(p0 * in.vscl[key], p1 * in.vscl[key + 1]);
-          }
-          tmem_st16(t_s + 16 * c, pk);
-        }
-      } else {
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t raw[32], pk[16];
-          tmem_ld32(t_s + 32 * c, raw);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            float pp[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int key = 32 * c + 2 * k + e;
-              const float tv = fmaf(__uint_as_float(raw[2 * k + e]) * in.kscl[key], rowmul, in.kb[key]);
-              pp[e] = in.ktok[key] < lim ? ex2(tv - mref) : 0.f;
-            }
-            lsum += pp[0] + pp[1];
-            pk[k] = pack_bf16x2(pp[0] * in.vscl[32 * c + 2 * k], pp[1] * in.vscl[32 * c + 2 * k + 1]);
-          }
-          tmem_st16(t_s + 16 * c, pk);
-        }
-      }
+      float s0, s1, s2, s3;
+      f2_unpack(sum01, s0, s1);
+      f2_unpack(sum23, s2, s3);
+      const float lsum = (s0 + s1) + (s2 + s3);
       l_run += lsum;
       tmem_wait_st();
       tc_fence_before();
