@@ -110,7 +110,7 @@ typedef struct kv_ring {
   int64_t rope_pos_min;      /* first position held by rope_table */
   int64_t rope_pos_max;      /* last position held by rope_table */
   double rope_base;          /* base used to build the table (for the delta rotation) */
-  uint64_t opaque[64];       /* library-owned: encoded TMA descriptors of the caches */
+  uint64_t opaque[96];       /* library-owned: encoded TMA descriptors of the caches */
 } kv_ring_t;
 
 /* Block-causal mask of the current chunk ("Stream LTX", section "Training": a block is

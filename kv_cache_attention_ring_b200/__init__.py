@@ -45,7 +45,7 @@ class kv_ring_t(ctypes.Structure):
                 ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
                 ("slot_pos", ctypes.c_void_p), ("rope_table", ctypes.c_void_p),
                 ("rope_pos_min", ctypes.c_int64), ("rope_pos_max", ctypes.c_int64),
-                ("rope_base", ctypes.c_double), ("opaque", ctypes.c_uint64 * 64)]
+                ("rope_base", ctypes.c_double), ("opaque", ctypes.c_uint64 * 96)]
 
 
 class kv_block_mask_t(ctypes.Structure):

@@ -412,8 +412,8 @@ int launch_d(const AttnArgs& a, const void* tk, const void* tv, cudaStream_t s) 
 }  // namespace
 
 int launch_attention(const AttnArgs& a, int D, const void* tmap_k, const void* tmap_v,
-                     const void* tmap_k_sw128, cudaStream_t s) {
-  if (D == 128) return launch_attention_sm100_d128(a, tmap_k_sw128, tmap_v, s);
+                     const void* tmap_k_sw128, const void* tmap_v_sw128, cudaStream_t s) {
+  if (D == 128) return launch_attention_sm100_d128(a, tmap_k_sw128, tmap_v_sw128, s);
   return launch_d<64>(a, tmap_k, tmap_v, s);
 }
 

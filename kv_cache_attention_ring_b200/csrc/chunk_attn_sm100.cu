@@ -8,29 +8,30 @@
 //   s_ij = softmax_scale * <bf16(RoPE(q_i)), e4m3(kc_j) * ks_j> + [j history] * bias,
 //   out_i = sum_j softmax_j(s_i) * e4m3(vc_j) * vs_j.
 //
-// Design (one CTA = 256 query rows of one head = two 128-row tiles g = 0, 1):
+// Design (one CTA = 256 query rows of one head = two 128-row tiles g = 0, 1; keys in
+// tiles of 64 slots):
 //  * Q.K^T runs on the FP8 tensor core directly on the cached e4m3 K codes (no
 //    conversion of K).  The rotated bf16 query row is split exactly into
 //    q = r * (hi + lo), hi, lo e4m3, r a power of two (8 significant bits = 4 + 4), so
 //    S' = hi.K + lo.K is one f32 accumulation of 2*D/32 kind::f8f6f4 MMAs and
 //    s = r * ks * scale * S' (+ bias).  r is per query row, so a row's result never
 //    depends on other rows (later blocks cannot change earlier ones, bit for bit).
-//  * P.V runs in bf16: four converter warps turn V codes into bf16(e4m3(vc) * vs) in
+//  * P.V runs in bf16: two converter warps turn V codes into bf16(e4m3(vc) * vs) in
 //    shared memory (one bf16 rounding, 2^-9 relative); P = bf16(p) is written to tensor
 //    memory over the S columns it came from and read from there as the A operand.
-//  * Softmax: two passes over the S tile in TMEM (row maximum, then 2^(t - m)), with
-//    paired fp32 instructions (f32x2) so the exponentials on the MUFU unit set the pace.
-//  * Tensor memory (512 columns): S0/P0 [0,128), S1/P1 [128,256), O0 [256,384),
-//    O1 [384,512).  MMA issue order per key tile j:
-//      S0(j) PV1(j-1) S1(j) PV0(j)
-//    so softmax of tile g overlaps the tensor core working on the other tile.
+//  * Tensor memory (512 columns): tile g owns two S/P buffers of 64 columns,
+//    [128g, 128g+64) and [128g+64, 128g+128), and O_g = [256+128g, 384+128g).  The MMA
+//    issuer runs one key tile ahead: S_g(j+1) is computed into the other buffer while
+//    the softmax of tile g works on S_g(j); issue order S0(j+1) S1(j+1) PV0(j) PV1(j).
 //  * Warps: 0 TMA producer, 1 MMA issuer, 2-3 V converters + per-key info, 4-7 softmax
-//    of tile 0, 8-11 softmax of tile 1 (thread = query row = TMEM lane).  12 warps leave
-//    168 registers per thread, enough to hold a whole 128-column S row.
-//  * Online softmax in log2 units with lazy rescale of O (only when the row maximum
-//    grows by more than 8, i.e. a factor 256); the final O / l is exact regardless.
-//  * Keys are visited in physical slot order in 128-slot tiles; the ring wrap costs
-//    nothing (attention does not depend on key order once bias and mask are per key).
+//    of tile 0, 8-11 softmax of tile 1 (thread = query row = TMEM lane).
+//  * Softmax in log2 units with paired fp32 instructions (f32x2): the 64-column S row
+//    sits in registers; pass 1 scales it in place and finds the maximum, pass 2 takes
+//    2^(t - m).  The reference maximum m moves lazily (only when the tile maximum
+//    exceeds it by more than 8, a factor 256); O is then rescaled in tensor memory after
+//    the previous P.V has completed.  out = O / l is exact regardless of m.
+//  * Keys are visited in physical slot order; the ring wrap costs nothing (attention
+//    does not depend on key order once bias and mask are per key).
 // Every mbarrier wait is bounded (about a second); on a timeout the CTA abandons the
 // work, writes NaN to its rows and exits.
 #include <cuda.h>
@@ -46,15 +47,15 @@ namespace {
 
 constexpr int D = 128;
 constexpr int BM = 256;                 // query rows per CTA
-constexpr int BN = 128;                 // key slots per tile
-constexpr int NK = 3;                   // K code stages
-constexpr int NV = 2;                   // V code stages
+constexpr int BN = 64;                  // key slots per tile
+constexpr int NK = 4;                   // K code stages
+constexpr int NV = 4;                   // V code stages
 constexpr int NB = 2;                   // V bf16 buffers
 constexpr int NI = 4;                   // per-key info stages
 constexpr int kThreads = 12 * 32;
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpConv = 2, kWarpSoft = 4;
-constexpr int kConvThreads = 64;
-constexpr uint32_t kPanel = 128u * 128u;   // one 128-row x 128-byte swizzled panel
+constexpr int kConvThreads = 64;        // one converter thread per key slot of a tile
+constexpr uint32_t kVPanel = BN * 128u;  // bytes of one 64-column bf16 panel of V (64 rows)
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kInvalidTok = 0x7FFFFFFF;
 
@@ -62,23 +63,25 @@ struct Info {             // per key slot of one tile
   float kscl[BN];         // ks * softmax_scale * log2(e); 0 for invalid slots
   float kb[BN];           // additive log2 logit: bias (history), 0 (current), -inf (invalid)
   int ktok[BN];           // -1 history, token index (current), kInvalidTok (invalid)
-  int flag[4];            // per converter warp: tile holds current or invalid keys
+  int flag[2];            // per converter warp: tile holds current or invalid keys
+  int pad[2];
 };
 
 struct Layout {
   static constexpr uint32_t qhi = 0;                            // e4m3 [256][128], sw128
   static constexpr uint32_t qlo = qhi + BM * D;
-  static constexpr uint32_t kbuf = qlo + BM * D;                // NK x e4m3 [128][128], sw128
-  static constexpr uint32_t vcode = kbuf + NK * BN * D;         // NV x e4m3 [128][128]
+  static constexpr uint32_t kbuf = qlo + BM * D;                // NK x e4m3 [64][128], sw128
+  static constexpr uint32_t vcode = kbuf + NK * BN * D;         // NV x e4m3 [64][128], sw128
   static constexpr uint32_t vbf = vcode + NV * BN * D;          // NB x bf16 2 panels, sw128
-  static constexpr uint32_t info = vbf + NB * 2 * kPanel;       // NI x Info
+  static constexpr uint32_t info = vbf + NB * 2 * kVPanel;      // NI x Info
   static constexpr uint32_t bars = info + NI * sizeof(Info);    // mbarriers
-  static constexpr int kNumBars = 2 * NK + 2 * NV + 2 * NB + 2 * NI + 2 + 2 + 1;
+  static constexpr int kNumBars = 2 * NK + 2 * NV + 2 * NB + 2 * NI + 4 + 4 + 2 + 1;
   static constexpr uint32_t misc = bars + 8 * kNumBars;         // tmem addr, abort flag
-  static constexpr uint32_t vsc = misc + 16;                    // float[BN]: converters only
-  static constexpr uint32_t bytes = vsc + 4 * BN + 1024;        // + alignment slack
+  static constexpr uint32_t bytes = misc + 16 + 1024;           // + alignment slack
 };
 static_assert(Layout::bytes <= 232448, "shared memory budget");
+static_assert(Layout::kbuf % 1024 == 0 && Layout::vcode % 1024 == 0 && Layout::vbf % 1024 == 0,
+              "swizzled operands need 1024-byte alignment");
 
 struct Bars {
   uint64_t* b;
@@ -90,9 +93,13 @@ struct Bars {
   __device__ uint64_t* vbempty(int s) { return b + 2 * NK + 2 * NV + NB + s; }
   __device__ uint64_t* ifull(int s) { return b + 2 * NK + 2 * NV + 2 * NB + s; }
   __device__ uint64_t* iempty(int s) { return b + 2 * NK + 2 * NV + 2 * NB + NI + s; }
-  __device__ uint64_t* sfull(int g) { return b + 2 * NK + 2 * NV + 2 * NB + 2 * NI + g; }
-  __device__ uint64_t* pfull(int g) { return b + 2 * NK + 2 * NV + 2 * NB + 2 * NI + 2 + g; }
-  __device__ uint64_t* ofinal() { return b + 2 * NK + 2 * NV + 2 * NB + 2 * NI + 4; }
+  // buffer `buf` of tile g holds S (sfull) / holds P (pfull); the P.V of tile g has
+  // completed (pvdone); all MMAs are done (ofinal).  P-ready is per buffer because the
+  // softmax may finish tile j+1 before the MMA issuer has consumed tile j's signal.
+  __device__ uint64_t* sfull(int g, int buf) { return b + 2 * (NK + NV + NB + NI) + 2 * g + buf; }
+  __device__ uint64_t* pfull(int g, int buf) { return b + 2 * (NK + NV + NB + NI) + 4 + 2 * g + buf; }
+  __device__ uint64_t* pvdone(int g) { return b + 2 * (NK + NV + NB + NI) + 8 + g; }
+  __device__ uint64_t* ofinal() { return b + 2 * (NK + NV + NB + NI) + 10; }
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -109,17 +116,19 @@ __device__ __forceinline__ float e4m3_value(uint32_t code) {
   return f16x2_to_float2(e4m3x2_to_f16x2((uint16_t)code)).x;
 }
 
+// Does tile t (slots [t*BN, t*BN+BN)) hold a valid slot?  Valid slots are the nv slots
+// ending at `newest` (mod C).
 __device__ __forceinline__ bool tile_valid(int t, int C, int newest, int nv) {
   if (nv <= 0) return false;
   if (nv >= C) return true;
   const int a = t * BN, b = min(C, a + BN);
   int first = newest - nv + 1;
   if (first >= 0) return a <= newest && b > first;
-  first += C;
+  first += C;  // wrapped: [first, C) and [0, newest]
   return (b > first) || (a <= newest);
 }
 
-// Next physical tile index >= t holding a valid slot (n_tiles if none).
+// Next tile index >= t holding a valid slot (n_tiles if none).
 __device__ __forceinline__ int next_tile(int t, int n_tiles, int C, int newest, int nv) {
   while (t < n_tiles && !tile_valid(t, C, newest, nv)) ++t;
   return t;
@@ -164,7 +173,7 @@ __device__ __forceinline__ int q_exponent(const AttnArgs& a, int gi, int h) {
 }
 
 // Split bf16(RoPE(q_gi)) / 2^k exactly into e4m3 hi + lo (4 + 4 significant bits; exact
-// for elements within 2^10 of the tile's largest) and write both into the swizzled
+// for elements within 2^10 of the row's largest) and write both into the swizzled
 // K-major operand rows.  Rows beyond n_q get zero codes.
 __device__ __forceinline__ void q_split(const AttnArgs& a, int gi, int h, int k, uint8_t* qhi,
                                         uint8_t* qlo, int row) {
@@ -234,7 +243,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < NV; ++s) { mbar_init(bars.vfull(s), 1); mbar_init(bars.vempty(s), kConvThreads); }
     for (int s = 0; s < NB; ++s) { mbar_init(bars.vbfull(s), kConvThreads); mbar_init(bars.vbempty(s), 1); }
     for (int s = 0; s < NI; ++s) { mbar_init(bars.ifull(s), kConvThreads); mbar_init(bars.iempty(s), 256); }
-    for (int g = 0; g < 2; ++g) { mbar_init(bars.sfull(g), 1); mbar_init(bars.pfull(g), 128); }
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(bars.sfull(g, 0), 1);
+      mbar_init(bars.sfull(g, 1), 1);
+      mbar_init(bars.pfull(g, 0), 128);
+      mbar_init(bars.pfull(g, 1), 128);
+      mbar_init(bars.pvdone(g), 1);
+    }
     mbar_init(bars.ofinal(), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -244,11 +259,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmv);
   }
 
-  // Q prologue by the softmax warps: thread = query row = TMEM lane
-  const int g = (warp - kWarpSoft) >> 2;                 // softmax tile (valid for warps 4..11)
+  // Q prologue by the softmax warps: thread = query row = TMEM lane; per-row scale r = 2^k
+  const int g = (warp - kWarpSoft) >> 2;                 // softmax tile (warps 4..11)
   const int row_in_tile = 32 * (warp & 3) + lane;        // TMEM lane of this thread
   const int gi = q0 + 128 * g + row_in_tile;
-  // per-row power-of-two query scale r = 2^k
   float rowmul = 1.f;
   if (warp >= kWarpSoft) {
     int k = q_exponent(a, gi, h);
@@ -277,11 +291,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sk = j % NK, rk = j / NK;
         if (rk > 0 && !wait(bars.kempty(sk), (rk - 1) & 1)) break;
         mbar_arrive_expect_tx(bars.kfull(sk), BN * D);
-        tma_load_3d(sm + Layout::kbuf + sk * BN * D, &tmk, bars.kfull(sk), 0, (int)(t * BN), h);
+        tma_load_3d(sm + Layout::kbuf + sk * BN * D, &tmk, bars.kfull(sk), 0, t * BN, h);
         const int sv = j % NV, rv = j / NV;
         if (rv > 0 && !wait(bars.vempty(sv), (rv - 1) & 1)) break;
         mbar_arrive_expect_tx(bars.vfull(sv), BN * D);
-        tma_load_3d(sm + Layout::vcode + sv * BN * D, &tmv, bars.vfull(sv), 0, (int)(t * BN), h);
+        tma_load_3d(sm + Layout::vcode + sv * BN * D, &tmv, bars.vfull(sv), 0, t * BN, h);
       }
     }
   } else if (warp == kWarpMma) {
@@ -291,8 +305,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t sQhi = smem_u32(sm + Layout::qhi), sQlo = smem_u32(sm + Layout::qlo);
       const uint32_t sK = smem_u32(sm + Layout::kbuf), sV = smem_u32(sm + Layout::vbf);
-      auto issue_s = [&](int gg, int sk) {
-        const uint32_t d = tmem + 128 * gg;
+      // S_g = Q_g K^T into buffer buf of tile g (hi and lo halves of Q accumulate)
+      auto issue_s = [&](int gg, int buf, int sk) {
+        const uint32_t d = tmem + 128 * gg + 64 * buf;
         const uint32_t kb = sK + sk * BN * D;
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk)
@@ -303,62 +318,69 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_mma_f8_ss(d, smem_desc_sw128(sQlo + gg * 128 * D + kk * 32, 16, 1024),
                        smem_desc_sw128(kb + kk * 32, 16, 1024), idS, 1);
       };
-      auto issue_pv = [&](int gg, int b, uint32_t acc) {
+      // O_g (+)= P_g V with P_g read from tensor memory (buffer buf)
+      auto issue_pv = [&](int gg, int buf, int vbi, uint32_t acc) {
         const uint32_t d = tmem + 256 + 128 * gg;
-        const uint32_t p = tmem + 128 * gg;
-        const uint32_t vb = sV + b * 2 * kPanel;
+        const uint32_t p = tmem + 128 * gg + 64 * buf;
+        const uint32_t vb = sV + vbi * 2 * kVPanel;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          tc_mma_f16_ts(d, p + 8 * kk, smem_desc_sw128(vb + kk * 2048, kPanel, 1024), idO,
+          tc_mma_f16_ts(d, p + 8 * kk, smem_desc_sw128(vb + kk * 2048, kVPanel, 1024), idO,
                         acc | (kk > 0));
       };
       int j = 0;
       bool ok = true;
-      for (int t = next_tile(0, n_tiles, C, newest, n_valid); t < n_tiles;
-           t = next_tile(t + 1, n_tiles, C, newest, n_valid), ++j) {
-        const int sk = j % NK;
-        if (!(ok = wait(bars.kfull(sk), (j / NK) & 1))) break;
-        tc_fence_after();
-        issue_s(0, sk);
-        tc_commit(bars.sfull(0));
-        if (j > 0) {
-          if (!(ok = wait(bars.pfull(1), (j - 1) & 1))) break;
+      int t = next_tile(0, n_tiles, C, newest, n_valid);
+      if (t < n_tiles) {
+        ok = wait(bars.kfull(0), 0);
+        if (ok) {
           tc_fence_after();
-          issue_pv(1, (j - 1) % NB, (j - 1) > 0);
-          tc_commit(bars.vbempty((j - 1) % NB));
+          issue_s(0, 0, 0);
+          tc_commit(bars.sfull(0, 0));
+          issue_s(1, 0, 0);
+          tc_commit(bars.sfull(1, 0));
+          tc_commit(bars.kempty(0));
         }
-        issue_s(1, sk);
-        tc_commit(bars.sfull(1));
-        tc_commit(bars.kempty(sk));
-        if (!(ok = wait(bars.vbfull(j % NB), (j / NB) & 1))) break;
-        if (!(ok = wait(bars.pfull(0), j & 1))) break;
-        tc_fence_after();
-        issue_pv(0, j % NB, j > 0);
       }
-      if (ok && j > 0 && wait(bars.pfull(1), (j - 1) & 1)) {
+      for (; ok && t < n_tiles; ++j) {
+        const int t_next = next_tile(t + 1, n_tiles, C, newest, n_valid);
+        if (t_next < n_tiles) {                        // S of the next tile, one ahead
+          const int jn = j + 1, sk = jn % NK;
+          if (!(ok = wait(bars.kfull(sk), (jn / NK) & 1))) break;
+          tc_fence_after();
+          issue_s(0, jn & 1, sk);
+          tc_commit(bars.sfull(0, jn & 1));
+          issue_s(1, jn & 1, sk);
+          tc_commit(bars.sfull(1, jn & 1));
+          tc_commit(bars.kempty(sk));
+        }
+        if (!(ok = wait(bars.vbfull(j % NB), (j / NB) & 1))) break;
+        if (!(ok = wait(bars.pfull(0, j & 1), (j >> 1) & 1))) break;
         tc_fence_after();
-        issue_pv(1, (j - 1) % NB, (j - 1) > 0);
-        tc_commit(bars.vbempty((j - 1) % NB));
+        issue_pv(0, j & 1, j % NB, j > 0);
+        tc_commit(bars.pvdone(0));
+        if (!(ok = wait(bars.pfull(1, j & 1), (j >> 1) & 1))) break;
+        tc_fence_after();
+        issue_pv(1, j & 1, j % NB, j > 0);
+        tc_commit(bars.pvdone(1));
+        tc_commit(bars.vbempty(j % NB));
+        t = t_next;
       }
       if (j > 0) tc_commit(bars.ofinal());
       else mbar_arrive(bars.ofinal());
     }
   } else if (warp < kWarpSoft) {
     // ------------------------------------------------------------ converters + key info
-    // 64 threads; thread ct owns keys ct and ct + 64 of every tile.  The K/V scales of the
-    // next tile are loaded while the current tile's V codes are converted.
+    // 64 threads; thread ct owns key slot ct of every tile: its info, its V row (bf16,
+    // scale folded in).  The scales of the next tile are loaded while this one converts.
     const int ct = tid - 32 * kWarpConv;          // 0..63
-    float* vsc = reinterpret_cast<float*>(sm + Layout::vsc);   // V scales of the tile
-    auto load_scales = [&](int tt, float (&ks)[2], float (&vs)[2]) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int slot = tt * BN + ct + 64 * e;
-        const bool in_ring = tt < n_tiles && slot < C;
-        ks[e] = in_ring ? __ldg(a.k_scale + (size_t)h * C + slot) : 0.f;
-        vs[e] = in_ring ? __ldg(a.v_scale + (size_t)h * C + slot) : 0.f;
-      }
+    auto load_scales = [&](int tt, float& ks, float& vs) {
+      const int slot = tt * BN + ct;
+      const bool in_ring = tt < n_tiles && slot < C;
+      ks = in_ring ? __ldg(a.k_scale + (size_t)h * C + slot) : 0.f;
+      vs = in_ring ? __ldg(a.v_scale + (size_t)h * C + slot) : 0.f;
     };
-    float pks[2], pvs[2];
+    float pks, pvs;
     int t = next_tile(0, n_tiles, C, newest, n_valid);
     load_scales(t, pks, pvs);
     for (int j = 0; t < n_tiles; ++j) {
@@ -367,61 +389,59 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = j < NI || wait(bars.iempty(si), ((j / NI) - 1) & 1);
       if (!named_bar_and(1, kConvThreads, ok)) break;   // uniform decision across converters
       Info& in = info[si];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int key = ct + 64 * e;
-        const int slot = t * BN + key;
-        float ksv = 0.f, kbv = -INFINITY, vsv = 0.f;
-        int tok = kInvalidTok;
-        if (slot < C) {
-          int age = newest - slot;
-          if (age < 0) age += C;
-          if (age < n_valid) {
-            ksv = pks[e] * a.score_scale_log2;
-            vsv = pvs[e];
-            if (age < a.n_current) {
-              kbv = 0.f;
-              tok = (int)(a.n_current - 1 - age);
-            } else {
-              kbv = a.bias_log2;
-              tok = -1;
-            }
+      const int slot = t * BN + ct;
+      float ksv = 0.f, kbv = -INFINITY, vsv = 0.f;
+      int tok = kInvalidTok;
+      if (slot < C) {
+        int age = newest - slot;
+        if (age < 0) age += C;
+        if (age < n_valid) {
+          ksv = pks * a.score_scale_log2;
+          vsv = pvs;
+          if (age < a.n_current) {
+            kbv = 0.f;
+            tok = a.n_current - 1 - age;
+          } else {
+            kbv = a.bias_log2;
+            tok = -1;
           }
         }
-        in.kscl[key] = ksv;
-        in.kb[key] = kbv;
-        in.ktok[key] = tok;
-        vsc[key] = vsv;
-        const unsigned special = __ballot_sync(0xffffffffu, tok != -1);
-        if (lane == 0) in.flag[2 * e + (ct >> 5)] = special != 0;
       }
+      in.kscl[ct] = ksv;
+      in.kb[ct] = kbv;
+      in.ktok[ct] = tok;
+      const unsigned special = __ballot_sync(0xffffffffu, tok != -1);
+      if (lane == 0) in.flag[ct >> 5] = special != 0;
       load_scales(t_next, pks, pvs);                   // prefetch for the next tile
-      named_bar(1, kConvThreads);                      // info of this tile complete
       mbar_arrive(bars.ifull(si));
       const int sv = j % NV, b = j % NB;
       ok = wait(bars.vfull(sv), (j / NV) & 1);
       ok = ok && (j < NB || wait(bars.vbempty(b), ((j / NB) - 1) & 1));
       if (!named_bar_and(2, kConvThreads, ok)) break;
-      const uint8_t* vc = sm + Layout::vcode + sv * BN * D;
-      uint8_t* vb = sm + Layout::vbf + b * 2 * kPanel;
-#pragma unroll 4
-      for (int idx = ct; idx < BN * D / 16; idx += kConvThreads) {
-        const int row = idx >> 3, c = idx & 7;
-        uint4 cv = *reinterpret_cast<const uint4*>(vc + row * D + 16 * c);
-        const float vsr = vsc[row];                    // 0 for invalid slots
-        if (in.ktok[row] == kInvalidTok) cv = make_uint4(0u, 0u, 0u, 0u);
+      // V row ct: 8 chunks of 16 codes (128-byte swizzled) -> bf16(code * vs)
+      const uint8_t* vc = sm + Layout::vcode + sv * BN * D + ct * 128;
+      uint8_t* vb = sm + Layout::vbf + b * 2 * kVPanel;
+      const bool dead = tok == kInvalidTok;
+      const uint64_t vs2 = f2_pack(vsv, vsv);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 cv = *reinterpret_cast<const uint4*>(vc + ((c ^ (ct & 7)) << 4));
+        if (dead) cv = make_uint4(0u, 0u, 0u, 0u);
         const uint32_t w[4] = {cv.x, cv.y, cv.z, cv.w};
         uint32_t o[8];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
+          float a0, a1, b0, b1;
           const float2 lo = f16x2_to_float2(e4m3x2_to_f16x2((uint16_t)(w[i] & 0xFFFFu)));
           const float2 hi = f16x2_to_float2(e4m3x2_to_f16x2((uint16_t)(w[i] >> 16)));
-          o[2 * i] = pack_bf16x2(lo.x * vsr, lo.y * vsr);
-          o[2 * i + 1] = pack_bf16x2(hi.x * vsr, hi.y * vsr);
+          f2_unpack(f2_mul(f2_pack(lo.x, lo.y), vs2), a0, a1);
+          f2_unpack(f2_mul(f2_pack(hi.x, hi.y), vs2), b0, b1);
+          o[2 * i] = pack_bf16x2(a0, a1);
+          o[2 * i + 1] = pack_bf16x2(b0, b1);
         }
-        *reinterpret_cast<uint4*>(vb + sw128_offset(row, 16 * c, kPanel)) =
+        *reinterpret_cast<uint4*>(vb + sw128_offset(ct, 16 * c, kVPanel)) =
             make_uint4(o[0], o[1], o[2], o[3]);
-        *reinterpret_cast<uint4*>(vb + sw128_offset(row, 16 * c + 8, kPanel)) =
+        *reinterpret_cast<uint4*>(vb + sw128_offset(ct, 16 * c + 8, kVPanel)) =
             make_uint4(o[4], o[5], o[6], o[7]);
       }
       fence_proxy_async_smem();
@@ -432,7 +452,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax of tile g
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    const uint32_t t_s = tmem + lane_base + 128 * g;           // S_g / P_g
     const uint32_t t_o = tmem + lane_base + 256 + 128 * g;     // O_g
     int lim;                                                   // visible current keys: tok < lim
     {
@@ -440,29 +459,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t l = (int64_t)a.k_first + qb * (int64_t)a.k_block;
       lim = (int)(l < (int64_t)a.n_current ? l : (int64_t)a.n_current);
     }
+    const uint64_t r2 = f2_pack(rowmul, rowmul);
     float m_run = -INFINITY, l_run = 0.f;
     int j = 0;
     for (int t = next_tile(0, n_tiles, C, newest, n_valid); t < n_tiles;
          t = next_tile(t + 1, n_tiles, C, newest, n_valid), ++j) {
-      const int si = j % NI;
-      bool ok = wait(bars.sfull(g), j & 1) && wait(bars.ifull(si), (j / NI) & 1);
+      const int si = j % NI, buf = j & 1;
+      const uint32_t t_s = tmem + lane_base + 128 * g + 64 * buf;   // S_g(j) / P_g(j)
+      bool ok = wait(bars.sfull(g, buf), (j >> 1) & 1) && wait(bars.ifull(si), (j / NI) & 1);
       if (!__all_sync(0xffffffffu, ok)) break;     // TMEM access below is warp-collective
       tc_fence_after();
       const Info& in = info[si];
-      const float* kscl = in.kscl;
-      const uint64_t r2 = f2_pack(rowmul, rowmul);
-      const bool special = (in.flag[0] | in.flag[1] | in.flag[2] | in.flag[3]) != 0;
-      // the whole 128-column S row of this thread: one load, one wait
-      uint32_t sr[128];
-      tmem_ld128(t_s, sr);
+      const bool special = (in.flag[0] | in.flag[1]) != 0;
+      uint32_t sr[64];
+      {
+        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t (*)[32]>(sr);
+        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t (*)[32]>(sr + 32);
+        tmem_ld32(t_s, lo);
+        tmem_ld32(t_s + 32, hi);
+      }
       tmem_wait_ld();
-      // pass 1, in place: fast tiles keep u = S * kscl, masked tiles t = u * r + kb (or
-      // -inf); track the row maximum.  Pass 2 then needs no per-key data.
+      // pass 1, in place: t = S * kscl (* r + bias later) for fast tiles, masked t for the
+      // others; row maximum of the tile
+      const float4* k4 = reinterpret_cast<const float4*>(in.kscl);
       float m0 = -INFINITY, m1 = -INFINITY;
-      const float4* k4 = reinterpret_cast<const float4*>(kscl);
       if (!special) {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
+        for (int q = 0; q < 16; ++q) {
           const float4 ks = k4[q];
           float u0, u1, u2, u3;
           f2_unpack(f2_mul(f2_pack(__uint_as_float(sr[4 * q]), __uint_as_float(sr[4 * q + 1])),
@@ -480,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float4* b4 = reinterpret_cast<const float4*>(in.kb);
         const int4* t4 = reinterpret_cast<const int4*>(in.ktok);
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
+        for (int q = 0; q < 16; ++q) {
           const float4 ks = k4[q], kb = b4[q];
           const int4 tk = t4[q];
           float u0, u1, u2, u3;
@@ -502,23 +525,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float mloc = special ? fmaxf(m0, m1) : fmaf(fmaxf(m0, m1), rowmul, a.bias_log2);
       // lazy reference maximum: move m only when the tile maximum exceeds it by more than
-      // 2^8; O is rescaled after pass 2 (the S row is no longer live then)
-      const bool move = mloc > m_run + kRescaleLog2 || (m_run == -INFINITY && mloc > -INFINITY);
-      const bool scale_o = move && m_run != -INFINITY;
-      const float alpha = scale_o ? ex2(m_run - mloc) : 1.f;
-      if (move) {
-        l_run *= alpha;
-        m_run = mloc;
-      }
-      // pass 2: p = 2^(t - m); P = bf16(p) written over the S columns (S is in registers)
+      // 2^8 (rows of a tile may differ; everything below is per row)
+      const float m_old = m_run;
+      const bool move = mloc > m_old + kRescaleLog2 || (m_old == -INFINITY && mloc > -INFINITY);
+      if (move) m_run = mloc;
       const float mref = (m_run == -INFINITY) ? 0.f : m_run;
-      // fast tiles: t - m = u * r + (bias - m); masked tiles: t - m = t * 1 + (-m)
+      // pass 2: p = 2^(t - m); P = bf16(p) over the S columns of tensor memory
       const float off = special ? -mref : a.bias_log2 - mref;
       const uint64_t mul2 = special ? f2_pack(1.f, 1.f) : r2;
       const uint64_t off2 = f2_pack(off, off);
       uint64_t sum01 = f2_pack(0.f, 0.f), sum23 = sum01;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int q8 = 0; q8 < 8; ++q8) {
@@ -536,7 +554,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st16(t_s + 16 * c, pk);
       }
-      if (__any_sync(0xffffffffu, scale_o)) {      // warp-collective TMEM access
+      float s0, s1, s2, s3;
+      f2_unpack(sum01, s0, s1);
+      f2_unpack(sum23, s2, s3);
+      const bool scale_o = move && m_old != -INFINITY;
+      const float alpha = scale_o ? ex2(m_old - m_run) : 1.f;
+      l_run = l_run * alpha + ((s0 + s1) + (s2 + s3));
+      // rescale O_g once the previous P.V of this tile has landed (rare; warp-collective)
+      if (__any_sync(0xffffffffu, scale_o)) {
+        ok = wait(bars.pvdone(g), (j - 1) & 1);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -547,14 +575,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st32(t_o + 32 * c, o);
         }
       }
-      float s0, s1, s2, s3;
-      f2_unpack(sum01, s0, s1);
-      f2_unpack(sum23, s2, s3);
-      const float lsum = (s0 + s1) + (s2 + s3);
-      l_run += lsum;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bars.pfull(g));
+      mbar_arrive(bars.pfull(g, buf));
       mbar_arrive(bars.iempty(si));
     }
     // ------------------------------------------------------------ epilogue
@@ -564,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool any = j > 0;
     uint16_t* dst = a.out + ((size_t)(row_ok ? gi : 0) * a.H + h) * D;
     const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
-#pragma unroll
+#pragma unroll 1
     for (int c = 0; c < D / 32; ++c) {
       uint32_t o[32];
       if (any) {
@@ -602,8 +625,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-int launch_attention_sm100_d128(const AttnArgs& a, const void* tmap_k_sw128, const void* tmap_v,
-                                cudaStream_t s) {
+int launch_attention_sm100_d128(const AttnArgs& a, const void* tmap_k_sw128,
+                                const void* tmap_v_sw128, cudaStream_t s) {
   static bool configured = false;
   if (!configured) {
     if (cudaFuncSetAttribute(chunk_attn_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -613,7 +636,7 @@ int launch_attention_sm100_d128(const AttnArgs& a, const void* tmap_k_sw128, con
   }
   CUtensorMap mk, mv;
   memcpy(&mk, tmap_k_sw128, sizeof(mk));
-  memcpy(&mv, tmap_v, sizeof(mv));
+  memcpy(&mv, tmap_v_sw128, sizeof(mv));
   dim3 grid((a.n_q + BM - 1) / BM, a.H);
   chunk_attn_sm100_kernel<<<grid, kThreads, Layout::bytes, s>>>(mk, mv, a);
   return cudaPeekAtLastError() == cudaSuccess ? KV_OK : KV_ECUDA;

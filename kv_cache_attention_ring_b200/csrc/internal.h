@@ -53,11 +53,11 @@ unsigned int* timeout_counter();
 
 int launch_write(const WriteArgs& a, int D, int in_dtype, cudaStream_t s);
 int launch_rotate(const RotateArgs& a, int D, cudaStream_t s);
-// tmaps: 128-byte CUtensorMap images of the K codes, the V codes (no swizzle) and the
-// K codes with the 128-byte swizzle (D = 128 only).
+// tmaps: 128-byte CUtensorMap images of the K and V codes without swizzle and with the
+// 128-byte swizzle (the latter for D = 128 only).
 int launch_attention(const AttnArgs& a, int D, const void* tmap_k, const void* tmap_v,
-                     const void* tmap_k_sw128, cudaStream_t s);
+                     const void* tmap_k_sw128, const void* tmap_v_sw128, cudaStream_t s);
 int launch_attention_sm100_d128(const AttnArgs& a, const void* tmap_k_sw128,
-                                const void* tmap_v, cudaStream_t s);
+                                const void* tmap_v_sw128, cudaStream_t s);
 
 }  // namespace kvring

@@ -31,7 +31,8 @@ constexpr uint64_t kMagic = 0x6B7672696E673031ull;  // "kvring01"
 constexpr int kOpaqueTmapK = 0;                     // K codes, no swizzle
 constexpr int kOpaqueTmapV = 16;                    // V codes, no swizzle
 constexpr int kOpaqueTmapKsw = 32;                  // K codes, 128-byte swizzle (D = 128)
-constexpr int kOpaqueMagic = 48;
+constexpr int kOpaqueTmapVsw = 48;                  // V codes, 128-byte swizzle (D = 128)
+constexpr int kOpaqueMagic = 64;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -88,16 +89,17 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D map over codes [H][C][D] bytes; box = D bytes x 128 slots x 1 head.  Slots >= C
-// read as zero.  swizzle128: rows land in shared memory with the 128-byte swizzle the
-// tensor core expects for a K-major operand (requires D = 128).
-int encode_codes_map(void* base, int H, int C, int D, uint64_t* dst, bool swizzle128) {
+// 3-D map over codes [H][C][D] bytes; box = D bytes x box_rows slots x 1 head.  Slots
+// >= C read as zero.  swizzle128: rows land in shared memory with the 128-byte swizzle
+// the tensor core expects for a K-major operand (requires D = 128).
+int encode_codes_map(void* base, int H, int C, int D, uint64_t* dst, bool swizzle128,
+                     unsigned box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return KV_ECUDA;
   alignas(64) CUtensorMap m;
   const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)C, (cuuint64_t)H};
   const cuuint64_t strides[2] = {(cuuint64_t)D, (cuuint64_t)C * (cuuint64_t)D};
-  const cuuint32_t box[3] = {(cuuint32_t)D, 128u, 1u};
+  const cuuint32_t box[3] = {(cuuint32_t)D, box_rows, 1u};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
   CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -153,14 +155,17 @@ int kv_ring_init(kv_ring_t* kv) {
     return KV_ECUDA;
   if (major != 10 || minor != 0) return KV_EUNSUPPORTED;
   int rc = encode_codes_map(kv->k_codes, kv->n_heads, kv->capacity, kv->head_dim,
-                            kv->opaque + kOpaqueTmapK, false);
+                            kv->opaque + kOpaqueTmapK, false, 128u);
   if (rc) return rc;
   rc = encode_codes_map(kv->v_codes, kv->n_heads, kv->capacity, kv->head_dim,
-                        kv->opaque + kOpaqueTmapV, false);
+                        kv->opaque + kOpaqueTmapV, false, 128u);
   if (rc) return rc;
-  if (kv->head_dim == 128) {
+  if (kv->head_dim == 128) {   // 64-slot boxes for the head_dim-128 attention kernel
     rc = encode_codes_map(kv->k_codes, kv->n_heads, kv->capacity, kv->head_dim,
-                          kv->opaque + kOpaqueTmapKsw, true);
+                          kv->opaque + kOpaqueTmapKsw, true, 64u);
+    if (rc) return rc;
+    rc = encode_codes_map(kv->v_codes, kv->n_heads, kv->capacity, kv->head_dim,
+                          kv->opaque + kOpaqueTmapVsw, true, 64u);
     if (rc) return rc;
   }
   kv->opaque[kOpaqueMagic] = kMagic;
@@ -288,7 +293,7 @@ int chunk_attention(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
   if (!a.timeouts) return KV_ECUDA;
   return launch_attention(a, kv->head_dim, kv->opaque + kOpaqueTmapK,
                           kv->opaque + kOpaqueTmapV, kv->opaque + kOpaqueTmapKsw,
-                          static_cast<cudaStream_t>(stream));
+                          kv->opaque + kOpaqueTmapVsw, static_cast<cudaStream_t>(stream));
 }
 
 int kv_wait_timeout_count(uint32_t* host_count) {

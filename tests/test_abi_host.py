@@ -53,7 +53,7 @@ def _fake_ring(C=256, H=2, D=64, pmin=0, pmax=4096):
         setattr(s, f, 0x100000)             # never dereferenced on these paths
     s.rope_pos_min, s.rope_pos_max, s.rope_base = pmin, pmax, 10000.0
     s.initialized = 1
-    s.opaque[48] = MAGIC
+    s.opaque[64] = MAGIC
     return s
 
 
