@@ -8,31 +8,28 @@
 //   s_ij = softmax_scale * <bf16(RoPE(q_i)), e4m3(kc_j) * ks_j> + [j history] * bias,
 //   out_i = sum_j softmax_j(s_i) * e4m3(vc_j) * vs_j.
 //
-// Design (one CTA = 128 query rows of one head; keys in tiles of 128 slots):
+// Design (one CTA = 256 query rows of one head = two 128-row tiles g = 0, 1; keys in
+// tiles of 64 slots):
 //  * Q.K^T runs on the FP8 tensor core directly on the cached e4m3 K codes (no
 //    conversion of K).  The rotated bf16 query row is split exactly into
 //    q = r * (hi + lo), hi, lo e4m3, r a power of two (8 significant bits = 4 + 4), so
 //    S' = hi.K + lo.K is one f32 accumulation of 2*D/32 kind::f8f6f4 MMAs and
 //    s = r * ks * scale * S' (+ bias).  r is per query row, so a row's result never
 //    depends on other rows (later blocks cannot change earlier ones, bit for bit).
-//  * P.V runs in bf16: four converter warps turn V codes into bf16(e4m3(vc) * vs) in
-//    shared memory (one bf16 rounding, 2^-9 relative); P = bf16(p) is written to its own
-//    tensor-memory buffer and read from there as the A operand.
-//  * Tensor memory (512 columns): S buffers [0,128) [128,256), P buffers [256,320)
-//    [320,384), O [384,512).  The MMA issuer keeps S(j+1) computing while the softmax
-//    works on S(j); issue order ... PV(j) S(j+2) PV(j+1) ...  Both MMAs have N = 128, so
-//    each operand byte read from shared memory feeds 128 columns.  S stays intact while
-//    its P is produced, so a softmax pass can be redone.
-//  * Warps: 0 TMA producer, 1 MMA issuer, 2-5 V converters + per-key info (thread = key
-//    slot), 6-9 softmax (thread = query row = TMEM lane).
-//  * Softmax in log2 units with paired fp32 instructions (f32x2).  Tiles whose keys are
-//    all valid history, once the row has a reference maximum m: one pass, 64 columns at a
-//    time, p = 2^(t - m) against the running m; if some t exceeds m by more than 8 (a
-//    factor 256) the tile is redone exactly.  First, masked (current-chunk, invalid or
-//    mixed) and redone tiles: an exact two-pass (row maximum, then 2^(t - m)) in
-//    32-column pieces with the mask.  m moves lazily (only when the tile maximum exceeds
-//    it by more than 8); O is then rescaled in tensor memory after the previous P.V has
-//    completed.  out = O / l is exact regardless of m.
+//  * P.V runs in bf16: two converter warps turn V codes into bf16(e4m3(vc) * vs) in
+//    shared memory (one bf16 rounding, 2^-9 relative); P = bf16(p) is written to tensor
+//    memory over the S columns it came from and read from there as the A operand.
+//  * Tensor memory (512 columns): tile g owns two S/P buffers of 64 columns,
+//    [128g, 128g+64) and [128g+64, 128g+128), and O_g = [256+128g, 384+128g).  The MMA
+//    issuer runs one key tile ahead: S_g(j+1) is computed into the other buffer while
+//    the softmax of tile g works on S_g(j); issue order S0(j+1) S1(j+1) PV0(j) PV1(j).
+//  * Warps: 0 TMA producer, 1 MMA issuer, 2-3 V converters + per-key info, 4-7 softmax
+//    of tile 0, 8-11 softmax of tile 1 (thread = query row = TMEM lane).
+//  * Softmax in log2 units with paired fp32 instructions (f32x2): the 64-column S row
+//    sits in registers; pass 1 scales it in place and finds the maximum, pass 2 takes
+//    2^(t - m).  The reference maximum m moves lazily (only when the tile maximum
+//    exceeds it by more than 8, a factor 256); O is then rescaled in tensor memory after
+//    the previous P.V has completed.  out = O / l is exact regardless of m.
 //  * Keys are visited in physical slot order; the ring wrap costs nothing (attention
 //    does not depend on key order once bias and mask are per key).
 // Every mbarrier wait is bounded (about a second); on a timeout the CTA abandons the
@@ -49,17 +46,16 @@ namespace kvring {
 namespace {
 
 constexpr int D = 128;
-constexpr int BM = 128;                 // query rows per CTA
-constexpr int BN = 128;                 // key slots per tile
-constexpr int NS = 2;                   // S buffers and P buffers in tensor memory
-constexpr int NK = 3;                   // K code stages
-constexpr int NV = 3;                   // V code stages
+constexpr int BM = 256;                 // query rows per CTA
+constexpr int BN = 64;                  // key slots per tile
+constexpr int NK = 4;                   // K code stages
+constexpr int NV = 4;                   // V code stages
 constexpr int NB = 2;                   // V bf16 buffers
 constexpr int NI = 4;                   // per-key info stages
-constexpr int kThreads = 10 * 32;
-constexpr int kWarpTma = 0, kWarpMma = 1, kWarpConv = 2, kWarpSoft = 6;
-constexpr int kConvThreads = 128;       // one converter thread per key slot of a tile
-constexpr uint32_t kVPanel = BN * 128u;  // bytes of one 64-column bf16 panel of V
+constexpr int kThreads = 12 * 32;
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpConv = 2, kWarpSoft = 4;
+constexpr int kConvThreads = 64;        // one converter thread per key slot of a tile
+constexpr uint32_t kVPanel = BN * 128u;  // bytes of one 64-column bf16 panel of V (64 rows)
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kInvalidTok = 0x7FFFFFFF;
 
@@ -67,19 +63,19 @@ struct Info {             // per key slot of one tile
   float kscl[BN];         // ks * softmax_scale * log2(e); 0 for invalid slots
   float kb[BN];           // additive log2 logit: bias (history), 0 (current), -inf (invalid)
   int ktok[BN];           // -1 history, token index (current), kInvalidTok (invalid)
-  int flag[4];            // per converter warp: tile holds current or invalid keys
-  float kext[8];          // per converter warp: max kscl [0, 4) and min kscl [4, 8)
+  int flag[2];            // per converter warp: tile holds current or invalid keys
+  int pad[2];
 };
 
 struct Layout {
-  static constexpr uint32_t qhi = 0;                            // e4m3 [128][128], sw128
+  static constexpr uint32_t qhi = 0;                            // e4m3 [256][128], sw128
   static constexpr uint32_t qlo = qhi + BM * D;
-  static constexpr uint32_t kbuf = qlo + BM * D;                // NK x e4m3 [128][128], sw128
-  static constexpr uint32_t vcode = kbuf + NK * BN * D;         // NV x e4m3 [128][128], sw128
+  static constexpr uint32_t kbuf = qlo + BM * D;                // NK x e4m3 [64][128], sw128
+  static constexpr uint32_t vcode = kbuf + NK * BN * D;         // NV x e4m3 [64][128], sw128
   static constexpr uint32_t vbf = vcode + NV * BN * D;          // NB x bf16 2 panels, sw128
   static constexpr uint32_t info = vbf + NB * 2 * kVPanel;      // NI x Info
   static constexpr uint32_t bars = info + NI * sizeof(Info);    // mbarriers
-  static constexpr int kNumBars = 2 * NK + 2 * NV + 2 * NB + 2 * NI + 2 * NS + 2;
+  static constexpr int kNumBars = 2 * NK + 2 * NV + 2 * NB + 2 * NI + 4 + 4 + 2 + 1;
   static constexpr uint32_t misc = bars + 8 * kNumBars;         // tmem addr, abort flag
   static constexpr uint32_t bytes = misc + 16 + 1024;           // + alignment slack
 };
@@ -97,13 +93,13 @@ struct Bars {
   __device__ uint64_t* vbempty(int s) { return b + 2 * NK + 2 * NV + NB + s; }
   __device__ uint64_t* ifull(int s) { return b + 2 * NK + 2 * NV + 2 * NB + s; }
   __device__ uint64_t* iempty(int s) { return b + 2 * NK + 2 * NV + 2 * NB + NI + s; }
-  // buffer `buf` holds S (sfull) / holds P (pfull); the last P.V has completed
-  // (pvdone); all MMAs are done (ofinal).  P-ready is per buffer because the softmax may
-  // finish later tiles before the MMA issuer has consumed an earlier tile's signal.
-  __device__ uint64_t* sfull(int buf) { return b + 2 * (NK + NV + NB + NI) + buf; }
-  __device__ uint64_t* pfull(int buf) { return b + 2 * (NK + NV + NB + NI) + NS + buf; }
-  __device__ uint64_t* pvdone() { return b + 2 * (NK + NV + NB + NI) + 2 * NS; }
-  __device__ uint64_t* ofinal() { return b + 2 * (NK + NV + NB + NI) + 2 * NS + 1; }
+  // buffer `buf` of tile g holds S (sfull) / holds P (pfull); the P.V of tile g has
+  // completed (pvdone); all MMAs are done (ofinal).  P-ready is per buffer because the
+  // softmax may finish tile j+1 before the MMA issuer has consumed tile j's signal.
+  __device__ uint64_t* sfull(int g, int buf) { return b + 2 * (NK + NV + NB + NI) + 2 * g + buf; }
+  __device__ uint64_t* pfull(int g, int buf) { return b + 2 * (NK + NV + NB + NI) + 4 + 2 * g + buf; }
+  __device__ uint64_t* pvdone(int g) { return b + 2 * (NK + NV + NB + NI) + 8 + g; }
+  __device__ uint64_t* ofinal() { return b + 2 * (NK + NV + NB + NI) + 10; }
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -220,122 +216,6 @@ __device__ __forceinline__ void q_split(const AttnArgs& a, int gi, int h, int k,
   }
 }
 
-// One pass over a tile row whose keys are all valid history, against the running
-// maximum m: t' = S * kscl * r + (bias - m), p = 2^t', P = bf16(p) into the P buffer.
-// 64 columns per tensor-memory load.  Returns sum(p); *tmaxp = max t' (a redo is due if
-// it exceeds the lazy threshold).
-__device__ __forceinline__ float softmax_single_pass(const float* kscl, uint64_t r2, float off,
-                                                     uint32_t t_s, uint32_t t_p, float* tmaxp) {
-  const float4* k4 = reinterpret_cast<const float4*>(kscl);
-  const uint64_t off2 = f2_pack(off, off);
-  uint64_t sum01 = f2_pack(0.f, 0.f), sum23 = sum01;
-  float x0 = -INFINITY, x1 = -INFINITY;
-#pragma unroll 1
-  for (int hf = 0; hf < 2; ++hf) {
-    uint32_t sr[64];
-    {
-      uint32_t (&lo)[32] = *reinterpret_cast<uint32_t (*)[32]>(sr);
-      uint32_t (&hi)[32] = *reinterpret_cast<uint32_t (*)[32]>(sr + 32);
-      tmem_ld32(t_s + 64 * hf, lo);
-      tmem_ld32(t_s + 64 * hf + 32, hi);
-    }
-    tmem_wait_ld();
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      uint32_t pk[16];
-#pragma unroll
-      for (int q8 = 0; q8 < 8; ++q8) {
-        const int q = 8 * c + q8;                     // 4 keys: 64 * hf + 4 * q ...
-        const float4 ks = k4[16 * hf + q];
-        float t0, t1, t2, t3;
-        f2_unpack(f2_fma(f2_mul(f2_pack(__uint_as_float(sr[4 * q]), __uint_as_float(sr[4 * q + 1])),
-                                f2_pack(ks.x, ks.y)), r2, off2), t0, t1);
-        f2_unpack(f2_fma(f2_mul(f2_pack(__uint_as_float(sr[4 * q + 2]), __uint_as_float(sr[4 * q + 3])),
-                                f2_pack(ks.z, ks.w)), r2, off2), t2, t3);
-        x0 = max3f(x0, t0, t1);
-        x1 = max3f(x1, t2, t3);
-        const float p0 = ex2(t0), p1 = ex2(t1), p2 = ex2(t2), p3 = ex2(t3);
-        sum01 = f2_add(sum01, f2_pack(p0, p1));
-        sum23 = f2_add(sum23, f2_pack(p2, p3));
-        pk[2 * q8] = pack_bf16x2(p0, p1);
-        pk[2 * q8 + 1] = pack_bf16x2(p2, p3);
-      }
-      tmem_st16(t_p + 32 * hf + 16 * c, pk);
-    }
-  }
-  *tmaxp = fmaxf(x0, x1);
-  float s0, s1, s2, s3;
-  f2_unpack(sum01, s0, s1);
-  f2_unpack(sum23, s2, s3);
-  return (s0 + s1) + (s2 + s3);
-}
-
-// Exact two-pass over one tile row with the mask, 32 columns at a time: t = S * kscl * r
-// + kb for visible keys (-inf otherwise); the lazy reference moves to the tile maximum
-// when that exceeds m_old by more than 8 (or m_old is -inf).  P = bf16(2^(t - m)) into the
-// P buffer.  Returns sum(p); *move / *mref report the reference used.
-__device__ __forceinline__ float softmax_exact(const Info& in, int lim, uint64_t r2, float m_old,
-                                               uint32_t t_s, uint32_t t_p, bool* move,
-                                               float* mref) {
-  const float4* k4 = reinterpret_cast<const float4*>(in.kscl);
-  const float4* b4 = reinterpret_cast<const float4*>(in.kb);
-  const int4* t4 = reinterpret_cast<const int4*>(in.ktok);
-  float m0 = -INFINITY, m1 = -INFINITY;
-#pragma unroll 1
-  for (int c = 0; c < 4; ++c) {
-    uint32_t raw[32];
-    tmem_ld32(t_s + 32 * c, raw);
-    tmem_wait_ld();
-#pragma unroll
-    for (int q8 = 0; q8 < 8; ++q8) {
-      const int q = 8 * c + q8;
-      const float4 ks = k4[q], kb = b4[q];
-      const int4 tk = t4[q];
-      float u0, u1, u2, u3;
-      f2_unpack(f2_fma(f2_mul(f2_pack(__uint_as_float(raw[4 * q8]), __uint_as_float(raw[4 * q8 + 1])),
-                              f2_pack(ks.x, ks.y)), r2, f2_pack(kb.x, kb.y)), u0, u1);
-      f2_unpack(f2_fma(f2_mul(f2_pack(__uint_as_float(raw[4 * q8 + 2]), __uint_as_float(raw[4 * q8 + 3])),
-                              f2_pack(ks.z, ks.w)), r2, f2_pack(kb.z, kb.w)), u2, u3);
-      m0 = max3f(m0, tk.x < lim ? u0 : -INFINITY, tk.y < lim ? u1 : -INFINITY);
-      m1 = max3f(m1, tk.z < lim ? u2 : -INFINITY, tk.w < lim ? u3 : -INFINITY);
-    }
-  }
-  const float mloc = fmaxf(m0, m1);
-  *move = mloc > m_old + kRescaleLog2 || (m_old == -INFINITY && mloc > -INFINITY);
-  *mref = *move ? mloc : m_old;
-  const float mr0 = (*mref == -INFINITY) ? 0.f : *mref;
-  uint64_t sum01 = f2_pack(0.f, 0.f), sum23 = sum01;
-  const uint64_t neg = f2_pack(-mr0, -mr0);
-#pragma unroll 1
-  for (int c = 0; c < 4; ++c) {
-    uint32_t raw[32], pk[16];
-    tmem_ld32(t_s + 32 * c, raw);
-    tmem_wait_ld();
-#pragma unroll
-    for (int q8 = 0; q8 < 8; ++q8) {
-      const int q = 8 * c + q8;
-      const float4 ks = k4[q], kb = b4[q];
-      const int4 tk = t4[q];
-      float t0, t1, t2, t3;
-      f2_unpack(f2_add(f2_fma(f2_mul(f2_pack(__uint_as_float(raw[4 * q8]), __uint_as_float(raw[4 * q8 + 1])),
-                                     f2_pack(ks.x, ks.y)), r2, f2_pack(kb.x, kb.y)), neg), t0, t1);
-      f2_unpack(f2_add(f2_fma(f2_mul(f2_pack(__uint_as_float(raw[4 * q8 + 2]), __uint_as_float(raw[4 * q8 + 3])),
-                                     f2_pack(ks.z, ks.w)), r2, f2_pack(kb.z, kb.w)), neg), t2, t3);
-      const float p0 = tk.x < lim ? ex2(t0) : 0.f, p1 = tk.y < lim ? ex2(t1) : 0.f;
-      const float p2 = tk.z < lim ? ex2(t2) : 0.f, p3 = tk.w < lim ? ex2(t3) : 0.f;
-      sum01 = f2_add(sum01, f2_pack(p0, p1));
-      sum23 = f2_add(sum23, f2_pack(p2, p3));
-      pk[2 * q8] = pack_bf16x2(p0, p1);
-      pk[2 * q8 + 1] = pack_bf16x2(p2, p3);
-    }
-    tmem_st16(t_p + 16 * c, pk);
-  }
-  float s0, s1, s2, s3;
-  f2_unpack(sum01, s0, s1);
-  f2_unpack(sum23, s2, s3);
-  return (s0 + s1) + (s2 + s3);
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_attn_sm100_kernel(const __grid_constant__ CUtensorMap tmk,
                             const __grid_constant__ CUtensorMap tmv, const AttnArgs a) {
@@ -362,9 +242,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < NK; ++s) { mbar_init(bars.kfull(s), 1); mbar_init(bars.kempty(s), 1); }
     for (int s = 0; s < NV; ++s) { mbar_init(bars.vfull(s), 1); mbar_init(bars.vempty(s), kConvThreads); }
     for (int s = 0; s < NB; ++s) { mbar_init(bars.vbfull(s), kConvThreads); mbar_init(bars.vbempty(s), 1); }
-    for (int s = 0; s < NI; ++s) { mbar_init(bars.ifull(s), kConvThreads); mbar_init(bars.iempty(s), 128); }
-    for (int s = 0; s < NS; ++s) { mbar_init(bars.sfull(s), 1); mbar_init(bars.pfull(s), 128); }
-    mbar_init(bars.pvdone(), 1);
+    for (int s = 0; s < NI; ++s) { mbar_init(bars.ifull(s), kConvThreads); mbar_init(bars.iempty(s), 256); }
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(bars.sfull(g, 0), 1);
+      mbar_init(bars.sfull(g, 1), 1);
+      mbar_init(bars.pfull(g, 0), 128);
+      mbar_init(bars.pfull(g, 1), 128);
+      mbar_init(bars.pvdone(g), 1);
+    }
     mbar_init(bars.ofinal(), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -375,13 +260,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // Q prologue by the softmax warps: thread = query row = TMEM lane; per-row scale r = 2^k
-  const int row = 32 * (warp & 3) + lane;                // TMEM lane of this thread
-  const int gi = q0 + row;
+  const int g = (warp - kWarpSoft) >> 2;                 // softmax tile (warps 4..11)
+  const int row_in_tile = 32 * (warp & 3) + lane;        // TMEM lane of this thread
+  const int gi = q0 + 128 * g + row_in_tile;
   float rowmul = 1.f;
   if (warp >= kWarpSoft) {
     int k = q_exponent(a, gi, h);
     k = (k == INT_MIN) ? 0 : max(-126, min(127, k));
-    q_split(a, gi, h, k, sm + Layout::qhi, sm + Layout::qlo, row);
+    q_split(a, gi, h, k, sm + Layout::qhi, sm + Layout::qlo, 128 * g + row_in_tile);
     rowmul = ldexpf(1.f, k);
   }
   fence_proxy_async_smem();
@@ -419,55 +305,75 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t sQhi = smem_u32(sm + Layout::qhi), sQlo = smem_u32(sm + Layout::qlo);
       const uint32_t sK = smem_u32(sm + Layout::kbuf), sV = smem_u32(sm + Layout::vbf);
-      int T = 0;                                       // valid tiles
-      for (int t = next_tile(0, n_tiles, C, newest, n_valid); t < n_tiles;
-           t = next_tile(t + 1, n_tiles, C, newest, n_valid))
-        ++T;
-      // S = Q K^T into buffer `buf` (hi and lo halves of Q accumulate)
-      auto issue_s = [&](int jn) -> bool {
-        const int sk = jn % NK;
-        if (!wait(bars.kfull(sk), (jn / NK) & 1)) return false;
-        tc_fence_after();
-        const uint32_t d = tmem + 128 * (jn % NS);
+      // S_g = Q_g K^T into buffer buf of tile g (hi and lo halves of Q accumulate)
+      auto issue_s = [&](int gg, int buf, int sk) {
+        const uint32_t d = tmem + 128 * gg + 64 * buf;
         const uint32_t kb = sK + sk * BN * D;
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk)
-          tc_mma_f8_ss(d, smem_desc_sw128(sQhi + kk * 32, 16, 1024),
+          tc_mma_f8_ss(d, smem_desc_sw128(sQhi + gg * 128 * D + kk * 32, 16, 1024),
                        smem_desc_sw128(kb + kk * 32, 16, 1024), idS, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk)
-          tc_mma_f8_ss(d, smem_desc_sw128(sQlo + kk * 32, 16, 1024),
+          tc_mma_f8_ss(d, smem_desc_sw128(sQlo + gg * 128 * D + kk * 32, 16, 1024),
                        smem_desc_sw128(kb + kk * 32, 16, 1024), idS, 1);
-        tc_commit(bars.sfull(jn % NS));
-        tc_commit(bars.kempty(sk));
-        return true;
       };
-      bool ok = true;
-      for (int jn = 0; jn < NS && jn < T && ok; ++jn) ok = issue_s(jn);
-      int j = 0;
-      for (; ok && j < T; ++j) {
-        // O (+)= P V with P read from tensor memory
-        if (!(ok = wait(bars.vbfull(j % NB), (j / NB) & 1))) break;
-        if (!(ok = wait(bars.pfull(j % NS), (j / NS) & 1))) break;
-        tc_fence_after();
-        const uint32_t p = tmem + 256 + 64 * (j % NS);
-        const uint32_t vb = sV + (j % NB) * 2 * kVPanel;
+      // O_g (+)= P_g V with P_g read from tensor memory (buffer buf)
+      auto issue_pv = [&](int gg, int buf, int vbi, uint32_t acc) {
+        const uint32_t d = tmem + 256 + 128 * gg;
+        const uint32_t p = tmem + 128 * gg + 64 * buf;
+        const uint32_t vb = sV + vbi * 2 * kVPanel;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          tc_mma_f16_ts(tmem + 384, p + 8 * kk, smem_desc_sw128(vb + kk * 2048, kVPanel, 1024),
-                        idO, (j > 0) | (kk > 0));
-        tc_commit(bars.pvdone());
+          tc_mma_f16_ts(d, p + 8 * kk, smem_desc_sw128(vb + kk * 2048, kVPanel, 1024), idO,
+                        acc | (kk > 0));
+      };
+      int j = 0;
+      bool ok = true;
+      int t = next_tile(0, n_tiles, C, newest, n_valid);
+      if (t < n_tiles) {
+        ok = wait(bars.kfull(0), 0);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0, 0, 0);
+          tc_commit(bars.sfull(0, 0));
+          issue_s(1, 0, 0);
+          tc_commit(bars.sfull(1, 0));
+          tc_commit(bars.kempty(0));
+        }
+      }
+      for (; ok && t < n_tiles; ++j) {
+        const int t_next = next_tile(t + 1, n_tiles, C, newest, n_valid);
+        if (t_next < n_tiles) {                        // S of the next tile, one ahead
+          const int jn = j + 1, sk = jn % NK;
+          if (!(ok = wait(bars.kfull(sk), (jn / NK) & 1))) break;
+          tc_fence_after();
+          issue_s(0, jn & 1, sk);
+          tc_commit(bars.sfull(0, jn & 1));
+          issue_s(1, jn & 1, sk);
+          tc_commit(bars.sfull(1, jn & 1));
+          tc_commit(bars.kempty(sk));
+        }
+        if (!(ok = wait(bars.vbfull(j % NB), (j / NB) & 1))) break;
+        if (!(ok = wait(bars.pfull(0, j & 1), (j >> 1) & 1))) break;
+        tc_fence_after();
+        issue_pv(0, j & 1, j % NB, j > 0);
+        tc_commit(bars.pvdone(0));
+        if (!(ok = wait(bars.pfull(1, j & 1), (j >> 1) & 1))) break;
+        tc_fence_after();
+        issue_pv(1, j & 1, j % NB, j > 0);
+        tc_commit(bars.pvdone(1));
         tc_commit(bars.vbempty(j % NB));
-        if (j + NS < T) ok = issue_s(j + NS);           // S buffer of tile j is free
+        t = t_next;
       }
       if (j > 0) tc_commit(bars.ofinal());
       else mbar_arrive(bars.ofinal());
     }
   } else if (warp < kWarpSoft) {
     // ------------------------------------------------------------ converters + key info
-    // thread ct owns key slot ct of every tile: its info and its V row (bf16, scale folded
-    // in).  The scales of the next tile are loaded while this one converts.
-    const int ct = tid - 32 * kWarpConv;          // 0..127
+    // 64 threads; thread ct owns key slot ct of every tile: its info, its V row (bf16,
+    // scale folded in).  The scales of the next tile are loaded while this one converts.
+    const int ct = tid - 32 * kWarpConv;          // 0..63
     auto load_scales = [&](int tt, float& ks, float& vs) {
       const int slot = tt * BN + ct;
       const bool in_ring = tt < n_tiles && slot < C;
@@ -504,20 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       in.kscl[ct] = ksv;
       in.kb[ct] = kbv;
       in.ktok[ct] = tok;
-      {
-        const unsigned special = __ballot_sync(0xffffffffu, tok != -1);
-        float kx = ksv, kn = ksv;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          kx = fmaxf(kx, __shfl_xor_sync(0xffffffffu, kx, off));
-          kn = fminf(kn, __shfl_xor_sync(0xffffffffu, kn, off));
-        }
-        if (lane == 0) {
-          in.flag[ct >> 5] = special != 0;
-          in.kext[ct >> 5] = kx;
-          in.kext[4 + (ct >> 5)] = kn;
-        }
-      }
+      const unsigned special = __ballot_sync(0xffffffffu, tok != -1);
+      if (lane == 0) in.flag[ct >> 5] = special != 0;
       load_scales(t_next, pks, pvs);                   // prefetch for the next tile
       mbar_arrive(bars.ifull(si));
       const int sv = j % NV, b = j % NB;
@@ -556,9 +450,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       t = t_next;
     }
   } else {
-    // ------------------------------------------------------------ softmax (row = lane)
+    // ------------------------------------------------------------ softmax of tile g
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    const uint32_t t_o = tmem + lane_base + 384;               // O
+    const uint32_t t_o = tmem + lane_base + 256 + 128 * g;     // O_g
     int lim;                                                   // visible current keys: tok < lim
     {
       const int64_t qb = gi < a.q_first ? 0 : 1 + (int64_t)(gi - a.q_first) / a.q_block;
@@ -570,32 +464,105 @@ __global__ void __launch_bounds__(kThreads, 1)
     int j = 0;
     for (int t = next_tile(0, n_tiles, C, newest, n_valid); t < n_tiles;
          t = next_tile(t + 1, n_tiles, C, newest, n_valid), ++j) {
-      const int si = j % NI, buf = j % NS;
-      const uint32_t t_s = tmem + lane_base + 128 * buf;       // S(j)
-      const uint32_t t_p = tmem + lane_base + 256 + 64 * buf;  // P(j)
-      bool ok = wait(bars.sfull(buf), (j / NS) & 1) && wait(bars.ifull(si), (j / NI) & 1);
+      const int si = j % NI, buf = j & 1;
+      const uint32_t t_s = tmem + lane_base + 128 * g + 64 * buf;   // S_g(j) / P_g(j)
+      bool ok = wait(bars.sfull(g, buf), (j >> 1) & 1) && wait(bars.ifull(si), (j / NI) & 1);
       if (!__all_sync(0xffffffffu, ok)) break;     // TMEM access below is warp-collective
       tc_fence_after();
       const Info& in = info[si];
-      const bool special = (in.flag[0] | in.flag[1] | in.flag[2] | in.flag[3]) != 0;
-      const float m_old = m_run;
-      bool move = false;
-      float mref = m_old, lsum = 0.f;
-      // one pass against the running maximum when possible; exact otherwise or on overflow
-      bool exact = __any_sync(0xffffffffu, special || m_old == -INFINITY);
-      if (!exact) {
-        float tmaxp;
-        lsum = softmax_single_pass(in.kscl, r2, a.bias_log2 - m_old, t_s, t_p, &tmaxp);
-        exact = __any_sync(0xffffffffu, !(tmaxp <= kRescaleLog2));
+      const bool special = (in.flag[0] | in.flag[1]) != 0;
+      uint32_t sr[64];
+      {
+        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t (*)[32]>(sr);
+        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t (*)[32]>(sr + 32);
+        tmem_ld32(t_s, lo);
+        tmem_ld32(t_s + 32, hi);
       }
-      if (exact) lsum = softmax_exact(in, lim, r2, m_old, t_s, t_p, &move, &mref);
+      tmem_wait_ld();
+      // pass 1, in place: t = S * kscl (* r + bias later) for fast tiles, masked t for the
+      // others; row maximum of the tile
+      const float4* k4 = reinterpret_cast<const float4*>(in.kscl);
+      float m0 = -INFINITY, m1 = -INFINITY;
+      if (!special) {
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const float4 ks = k4[q];
+          float u0, u1, u2, u3;
+          f2_unpack(f2_mul(f2_pack(__uint_as_float(sr[4 * q]), __uint_as_float(sr[4 * q + 1])),
+                           f2_pack(ks.x, ks.y)), u0, u1);
+          f2_unpack(f2_mul(f2_pack(__uint_as_float(sr[4 * q + 2]), __uint_as_float(sr[4 * q + 3])),
+                           f2_pack(ks.z, ks.w)), u2, u3);
+          sr[4 * q] = __float_as_uint(u0);
+          sr[4 * q + 1] = __float_as_uint(u1);
+          sr[4 * q + 2] = __float_as_uint(u2);
+          sr[4 * q + 3] = __float_as_uint(u3);
+          m0 = max3f(m0, u0, u1);
+          m1 = max3f(m1, u2, u3);
+        }
+      } else {
+        const float4* b4 = reinterpret_cast<const float4*>(in.kb);
+        const int4* t4 = reinterpret_cast<const int4*>(in.ktok);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const float4 ks = k4[q], kb = b4[q];
+          const int4 tk = t4[q];
+          float u0, u1, u2, u3;
+          f2_unpack(f2_fma(f2_mul(f2_pack(__uint_as_float(sr[4 * q]), __uint_as_float(sr[4 * q + 1])),
+                                  f2_pack(ks.x, ks.y)), r2, f2_pack(kb.x, kb.y)), u0, u1);
+          f2_unpack(f2_fma(f2_mul(f2_pack(__uint_as_float(sr[4 * q + 2]), __uint_as_float(sr[4 * q + 3])),
+                                  f2_pack(ks.z, ks.w)), r2, f2_pack(kb.z, kb.w)), u2, u3);
+          u0 = tk.x < lim ? u0 : -INFINITY;
+          u1 = tk.y < lim ? u1 : -INFINITY;
+          u2 = tk.z < lim ? u2 : -INFINITY;
+          u3 = tk.w < lim ? u3 : -INFINITY;
+          sr[4 * q] = __float_as_uint(u0);
+          sr[4 * q + 1] = __float_as_uint(u1);
+          sr[4 * q + 2] = __float_as_uint(u2);
+          sr[4 * q + 3] = __float_as_uint(u3);
+          m0 = max3f(m0, u0, u1);
+          m1 = max3f(m1, u2, u3);
+        }
+      }
+      const float mloc = special ? fmaxf(m0, m1) : fmaf(fmaxf(m0, m1), rowmul, a.bias_log2);
+      // lazy reference maximum: move m only when the tile maximum exceeds it by more than
+      // 2^8 (rows of a tile may differ; everything below is per row)
+      const float m_old = m_run;
+      const bool move = mloc > m_old + kRescaleLog2 || (m_old == -INFINITY && mloc > -INFINITY);
+      if (move) m_run = mloc;
+      const float mref = (m_run == -INFINITY) ? 0.f : m_run;
+      // pass 2: p = 2^(t - m); P = bf16(p) over the S columns of tensor memory
+      const float off = special ? -mref : a.bias_log2 - mref;
+      const uint64_t mul2 = special ? f2_pack(1.f, 1.f) : r2;
+      const uint64_t off2 = f2_pack(off, off);
+      uint64_t sum01 = f2_pack(0.f, 0.f), sum23 = sum01;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8) {
+          const int q = 8 * c + q8;
+          float t0, t1, t2, t3;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[4 * q]), __uint_as_float(sr[4 * q + 1])), mul2,
+                           off2), t0, t1);
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[4 * q + 2]), __uint_as_float(sr[4 * q + 3])), mul2,
+                           off2), t2, t3);
+          const float p0 = ex2(t0), p1 = ex2(t1), p2 = ex2(t2), p3 = ex2(t3);   // 2^-inf = 0
+          sum01 = f2_add(sum01, f2_pack(p0, p1));
+          sum23 = f2_add(sum23, f2_pack(p2, p3));
+          pk[2 * q8] = pack_bf16x2(p0, p1);
+          pk[2 * q8 + 1] = pack_bf16x2(p2, p3);
+        }
+        tmem_st16(t_s + 16 * c, pk);
+      }
+      float s0, s1, s2, s3;
+      f2_unpack(sum01, s0, s1);
+      f2_unpack(sum23, s2, s3);
       const bool scale_o = move && m_old != -INFINITY;
-      const float alpha = scale_o ? ex2(m_old - mref) : 1.f;
-      if (move) m_run = mref;
-      l_run = l_run * alpha + lsum;
-      // rescale O once the previous P.V has landed (rare; warp-collective)
+      const float alpha = scale_o ? ex2(m_old - m_run) : 1.f;
+      l_run = l_run * alpha + ((s0 + s1) + (s2 + s3));
+      // rescale O_g once the previous P.V of this tile has landed (rare; warp-collective)
       if (__any_sync(0xffffffffu, scale_o)) {
-        ok = wait(bars.pvdone(), (j - 1) & 1);
+        ok = wait(bars.pvdone(g), (j - 1) & 1);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
 #pragma unroll 1
@@ -610,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bars.pfull(buf));
+      mbar_arrive(bars.pfull(g, buf));
       mbar_arrive(bars.iempty(si));
     }
     // ------------------------------------------------------------ epilogue

@@ -160,12 +160,12 @@ int kv_ring_init(kv_ring_t* kv) {
   rc = encode_codes_map(kv->v_codes, kv->n_heads, kv->capacity, kv->head_dim,
                         kv->opaque + kOpaqueTmapV, false, 128u);
   if (rc) return rc;
-  if (kv->head_dim == 128) {   // swizzled 128-slot boxes for the head_dim-128 kernel
+  if (kv->head_dim == 128) {   // swizzled 64-slot boxes for the head_dim-128 kernel
     rc = encode_codes_map(kv->k_codes, kv->n_heads, kv->capacity, kv->head_dim,
-                          kv->opaque + kOpaqueTmapKsw, true, 128u);
+                          kv->opaque + kOpaqueTmapKsw, true, 64u);
     if (rc) return rc;
     rc = encode_codes_map(kv->v_codes, kv->n_heads, kv->capacity, kv->head_dim,
-                          kv->opaque + kOpaqueTmapVsw, true, 128u);
+                          kv->opaque + kOpaqueTmapVsw, true, 64u);
     if (rc) return rc;
   }
   kv->opaque[kOpaqueMagic] = kMagic;

@@ -121,3 +121,32 @@ def chunk_qkv(w: Workload, chunk: int, pss: int = 0, n: int | None = None, strea
 def as_f32(t: torch.Tensor) -> np.ndarray:
     """Exact binary32 view of an input tensor (bf16 widens exactly)."""
     return t.to(torch.float32).numpy()
+
+
+def draw_torch(seed: int, shape, dist: str = "normal", scale: float = 1.0, dtype: str = "bf16",
+               device="cuda") -> torch.Tensor:
+    """Seeded tensor drawn by torch on `device` (fast for long streams).  Student-t(4) is
+    z0 / sqrt((z1^2 + z2^2 + z3^2 + z4^2) / 4) with independent normals z.  The same seed
+    on the same device gives the same tensor; copy it to the host for the oracle."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    if dist == "normal":
+        x = torch.randn(shape, generator=g, device=device)
+    elif dist == "student_t4":
+        z = torch.randn((5, *shape), generator=g, device=device)
+        x = z[0] / torch.sqrt((z[1:] ** 2).sum(0) / 4.0)
+    else:
+        raise ValueError(dist)
+    if scale != 1.0:
+        x = x * scale
+    return x.to(torch.bfloat16) if dtype == "bf16" else x.contiguous()
+
+
+def chunk_qkv_torch(w: Workload, chunk: int, pss: int = 0, device="cuda"):
+    """(q, k, v) of one chunk drawn on `device` with torch (see draw_torch)."""
+    wid = sum(map(ord, w.name))
+    shape = (w.n, w.H, w.D)
+    q = draw_torch(seed_of(wid, 7, chunk, pss, 1), shape, "normal", w.in_scale, w.in_dtype, device)
+    k = draw_torch(seed_of(wid, 7, chunk, pss, 2), shape, w.dist, w.in_scale, w.in_dtype, device)
+    v = draw_torch(seed_of(wid, 7, chunk, pss, 3), shape, w.dist, w.in_scale, w.in_dtype, device)
+    return q, k, v

@@ -90,29 +90,45 @@ def test_joint_audio_video_four_paths(orc):
 def test_long_stream_resets_and_bias_toggle(orc):
     """32,768-slot ring, 600 chunks of 1,024 (many wraparounds), a delta re-rotation of the
     whole cache every 50 chunks (positions return to 0..C-1), cache bias 0 <-> -4 every 10
-    chunks, Student-t(4) keys and values.  Attention is checked around the resets."""
+    chunks, Student-t(4) keys and values.  The GPU runs the whole stream.  At checkpoints the
+    oracle replays the last 40 chunks from the recorded ring head: 40 x 1,024 slots cover
+    the ring, so the replayed state equals the full stream's (including the resets in the
+    window); attention and ring state are compared there."""
     w = inputs.STRESS
     chunks, every = w.extra["chunks"], w.extra["reset_every"]
+    window = 40
+    assert window * w.n > w.C
     max_pos = w.C + every * w.n + w.n
     ring = kv.KvRing(w.C, w.H, w.D, 0, max_pos)
-    o = orc.OracleRing(w.C, w.H, w.D)
-    checked = {0, 1, 49, 50, 51, 299, 599}
+    checked = (49, 50, 51, 299, 599)
     rows = sample_rows(w.n, 8, seed=6)
+    heads = []          # ring head (write_slot, next_pos) before each chunk's write
+    resets = {}         # chunk -> delta applied after that chunk's commit
     for ch in range(chunks):
-        q, k, v = inputs.chunk_qkv(w, ch)
-        kv.kv_ring_write(ring, to_dev(k), to_dev(v))
-        o.write(inputs.as_f32(k), inputs.as_f32(v))
+        heads.append((ring.s.write_slot, ring.s.next_pos))
+        q, k, v = inputs.chunk_qkv_torch(w, ch)
+        kv.kv_ring_write(ring, k, v)
         if ch in checked:
             bias = w.biases[(ch // w.extra["bias_every"]) % 2]
-            out, lse = kv.chunk_attention(ring, to_dev(q), ring.next_pos, w.n, None, bias)
-            ro, rl = o.attention(inputs.as_f32(q), o.next_pos, w.n, cache_bias=bias, rows=rows)
+            out, lse = kv.chunk_attention(ring, q, ring.next_pos, w.n, None, bias)
+            o = orc.OracleRing(w.C, w.H, w.D)
+            first = max(0, ch - window)
+            o._s.write_slot, o._s.next_pos = heads[first]
+            for c2 in range(first, ch + 1):
+                _, k2, v2 = inputs.chunk_qkv_torch(w, c2)
+                o.write(inputs.as_f32(k2.cpu()), inputs.as_f32(v2.cpu()), commit=c2 < ch)
+                if c2 < ch and c2 in resets:
+                    o.delta_rotate(resets[c2])
+            assert (o.write_slot, o.next_pos) == (ring.s.write_slot, ring.s.next_pos)
+            slots = [o.slot_of_age(a) for a in range(w.C)]
+            assert_ring_equal(ring, o, slots=slots, what=f"stress ring at chunk {ch}")
+            ro, rl = o.attention(inputs.as_f32(q.cpu()), o.next_pos, w.n, cache_bias=bias,
+                                 rows=rows)
             assert_attention_close(out, lse, ro, rl, rows=rows, what=f"stress chunk {ch}")
-            assert_ring_equal(ring, o, what=f"stress ring at chunk {ch}")
         kv.kv_ring_commit(ring)
-        o.commit()
         if (ch + 1) % every == 0:
-            oldest = int(o.slot_pos[o.slot_of_age(min(o.live, w.C) - 1)])
+            oldest = int(ring.slot_pos[(ring.s.write_slot) % w.C].item())   # ring is full
             kv.kv_ring_delta_rotate(ring, -oldest)
-            o.delta_rotate(-oldest)
-    assert_ring_equal(ring, o, what="stress ring at the end")
+            resets[ch] = -oldest
+            assert int(ring.slot_pos.min().item()) == 0
     assert kv.kv_wait_timeout_count() == 0
