@@ -459,13 +459,14 @@ def main():
     wbytes = write_bytes(w.n, w.H, w.D)
     write_gbs = wbytes / (ms_write * 1e-3) / 1e9
     fp8_peak = 2.0 * peaks["bf16"]                       # nominal fp8:bf16 = 2:1
-    src = os.path.join(ROOT, "kv_cache_attention_ring_b200", "csrc", "chunk_attn.cu")
+    src = os.path.join(ROOT, "kv_cache_attention_ring_b200", "csrc", "chunk_attn_sm100.cu")
     traffic = traffic_for(src)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16 MMA on e4m3 cache (fp32 accumulate); write/rotate f32->e4m3",
+        "dtype": "e4m3 (Q hi+lo) x e4m3 K and f16 P x f16 V' MMAs, fp32 accumulate; "
+                 "write/rotate f32->e4m3",
         "data": "synthetic",
         "config": config_block({"parallelism": f"replicas{world}" if world > 1 else "1 GPU",
                                 "rings": R, "calls_per_step": R * PASSES}),
@@ -483,9 +484,11 @@ def main():
                    "frac_hbm": rot["bytes_per_launch"] / (rot_us * 1e-6) / 1e9 / peaks["hbm"]},
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peaks["bf16_sus"],
                      "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16_sus"],
-                     "traffic": traffic, "kernel": "chunk_attn_kernel<128>",
+                     "traffic": traffic, "kernel": "chunk_attn_sm100_kernel",
                      "peak_note": f"{peaks['src']} bf16 sustained (kernel timed inside a "
-                                  f"long graph); the contraction is bf16 x bf16 -> fp32"},
+                                  f"long graph); S = Q.K^T runs as two e4m3 MMAs (query "
+                                  f"hi + lo), as much tensor time as one bf16 MMA, and "
+                                  f"P.V is f16 (same rate), so the bf16 peak bounds 4*D flops/pair"},
         "e2e": {"value": e2e_ms * 1e3 / (R * PASSES) / world, "unit": UNIT,
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
         "gpu_launches": 2 * R * PASSES * args.steps,

@@ -183,6 +183,27 @@ KV_API int chunk_attention(const kv_ring_t* kv, const void* q, int n_q, int64_t 
                     int n_current, const kv_block_mask_t* mask, const kv_cache_bias_t* bias,
                     float softmax_scale, void* out, float* lse, uint32_t flags, void* stream);
 
+/* Bytes of workspace chunk_attention_split needs: n_splits * n_q * n_heads * (4*head_dim + 8).
+ * 0 for invalid arguments. */
+KV_API size_t chunk_attention_workspace_size(int n_q, int n_heads, int head_dim, int n_splits);
+
+/* chunk_attention with the keys split over n_splits (1..64) groups of consecutive valid
+ * tiles, for few queries over a long ring (e.g. the 25 audio latents of a 1 s block in
+ * "Stream LTX", section "Training", attending a 20-block video ring): every split keeps
+ * its own online softmax and writes an unnormalised fp32 partial (O, max, sum) into
+ * `workspace`; a second kernel merges the partials (max over splits, weights 2^(m_s - M))
+ * into out and lse.  Same result and contract as chunk_attention up to fp32 rounding.
+ * workspace: device, 16-byte aligned, caller-owned, at least
+ * chunk_attention_workspace_size(n_q, H, D, n_splits) bytes, contents need not be
+ * initialised; calls that share a workspace must be ordered on one stream.  head_dim 128
+ * only.  Errors: those of chunk_attention, KV_EINVAL (n_splits, workspace null or
+ * misaligned), KV_ERANGE (workspace too small), KV_EUNSUPPORTED (head_dim 64). */
+KV_API int chunk_attention_split(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
+                                 int n_current, const kv_block_mask_t* mask,
+                                 const kv_cache_bias_t* bias, float softmax_scale, void* out,
+                                 float* lse, int n_splits, void* workspace,
+                                 size_t workspace_bytes, uint32_t flags, void* stream);
+
 /* Static description of a status code.  Never NULL. */
 KV_API const char* kv_status_string(int status);
 

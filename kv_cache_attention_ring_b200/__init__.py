@@ -26,8 +26,8 @@ KV_DTYPE_BF16, KV_DTYPE_FP32 = 1, 2
 KV_COMMIT = 1
 
 EXPORTS = ("kv_rope_table_build", "kv_ring_init", "kv_ring_write", "kv_ring_commit",
-           "kv_ring_delta_rotate", "chunk_attention", "kv_status_string",
-           "kv_wait_timeout_count")
+           "kv_ring_delta_rotate", "chunk_attention", "chunk_attention_workspace_size",
+           "chunk_attention_split", "kv_status_string", "kv_wait_timeout_count")
 
 
 class KvError(RuntimeError):
@@ -79,6 +79,10 @@ def lib() -> ctypes.CDLL:
         L.kv_status_string.argtypes = [I]
         L.kv_status_string.restype = ctypes.c_char_p
         L.kv_wait_timeout_count.argtypes = [P]
+        L.chunk_attention_workspace_size.argtypes = [I, I, I, I]
+        L.chunk_attention_workspace_size.restype = ctypes.c_size_t
+        L.chunk_attention_split.argtypes = [P, P, I, I64, I, P, P, ctypes.c_float, P, P, I, P,
+                                            ctypes.c_size_t, ctypes.c_uint32, P]
         _lib = L
     return _lib
 
@@ -197,6 +201,39 @@ def chunk_attention(ring: KvRing, q, q_pos0: int, n_current: int, mask=None,
                                  float(softmax_scale), _ptr(out),
                                  None if lse is None else _ptr(lse), 0, _stream(stream)),
            "chunk_attention")
+    return out, lse
+
+
+def chunk_attention_workspace_size(n_q: int, n_heads: int, head_dim: int, n_splits: int) -> int:
+    return int(lib().chunk_attention_workspace_size(int(n_q), int(n_heads), int(head_dim),
+                                                    int(n_splits)))
+
+
+def chunk_attention_split(ring: KvRing, q, q_pos0: int, n_current: int, n_splits: int,
+                          workspace, mask=None, cache_bias: float = 0.0,
+                          softmax_scale: float | None = None, out=None, lse=None,
+                          want_lse: bool = True, stream=None):
+    """chunk_attention with the keys split over n_splits groups; `workspace` is a device
+    tensor of at least chunk_attention_workspace_size(...) bytes."""
+    import torch
+    assert q.is_cuda and q.dtype == torch.bfloat16 and q.is_contiguous()
+    n_q = int(q.shape[0])
+    assert q.shape == (n_q, ring.H, ring.D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((ring.H, n_q), dtype=torch.float32, device=q.device)
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(ring.D)
+    m = None if mask is None else kv_block_mask_t(*(int(x) for x in mask))
+    b = kv_cache_bias_t(float(cache_bias))
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().chunk_attention_split(ring.ref, _ptr(q), n_q, int(q_pos0), int(n_current),
+                                       None if m is None else ctypes.byref(m), ctypes.byref(b),
+                                       float(softmax_scale), _ptr(out),
+                                       None if lse is None else _ptr(lse), int(n_splits),
+                                       _ptr(workspace), nbytes, 0, _stream(stream)),
+           "chunk_attention_split")
     return out, lse
 
 

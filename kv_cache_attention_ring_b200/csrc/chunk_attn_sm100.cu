@@ -16,9 +16,11 @@
 //    S' = hi.K + lo.K is one f32 accumulation of 2*D/32 kind::f8f6f4 MMAs and
 //    s = r * ks * scale * S' (+ bias).  r is per query row, so a row's result never
 //    depends on other rows (later blocks cannot change earlier ones, bit for bit).
-//  * P.V runs in bf16: two converter warps turn V codes into bf16(e4m3(vc) * vs) in
-//    shared memory (one bf16 rounding, 2^-9 relative); P = bf16(p) is written to tensor
-//    memory over the S columns it came from and read from there as the A operand.
+//  * P.V runs in f16 (11 significant bits): a CTA first finds G, the smallest power of
+//    two at or above every V scale of its keys; two converter warps turn V codes into
+//    f16(e4m3(vc) * vs / G) in shared memory (|V'| <= 448, one f16 rounding, 2^-11
+//    relative); P = f16(p) (p <= 1) is written to tensor memory over the S columns it
+//    came from and read from there as the A operand; the epilogue multiplies O by G.
 //  * Tensor memory (512 columns): tile g owns two S/P buffers of 64 columns,
 //    [128g, 128g+64) and [128g+64, 128g+128), and O_g = [256+128g, 384+128g).  The MMA
 //    issuer runs one key tile ahead: S_g(j+1) is computed into the other buffer while
@@ -50,12 +52,12 @@ constexpr int BM = 256;                 // query rows per CTA
 constexpr int BN = 64;                  // key slots per tile
 constexpr int NK = 4;                   // K code stages
 constexpr int NV = 4;                   // V code stages
-constexpr int NB = 2;                   // V bf16 buffers
+constexpr int NB = 2;                   // V f16 buffers
 constexpr int NI = 4;                   // per-key info stages
 constexpr int kThreads = 12 * 32;
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpConv = 2, kWarpSoft = 4;
 constexpr int kConvThreads = 64;        // one converter thread per key slot of a tile
-constexpr uint32_t kVPanel = BN * 128u;  // bytes of one 64-column bf16 panel of V (64 rows)
+constexpr uint32_t kVPanel = BN * 128u;  // bytes of one 64-column f16 panel of V (64 rows)
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kInvalidTok = 0x7FFFFFFF;
 
@@ -72,15 +74,15 @@ struct Layout {
   static constexpr uint32_t qlo = qhi + BM * D;
   static constexpr uint32_t kbuf = qlo + BM * D;                // NK x e4m3 [64][128], sw128
   static constexpr uint32_t vcode = kbuf + NK * BN * D;         // NV x e4m3 [64][128], sw128
-  static constexpr uint32_t vbf = vcode + NV * BN * D;          // NB x bf16 2 panels, sw128
-  static constexpr uint32_t info = vbf + NB * 2 * kVPanel;      // NI x Info
+  static constexpr uint32_t vh = vcode + NV * BN * D;           // NB x f16 2 panels, sw128
+  static constexpr uint32_t info = vh + NB * 2 * kVPanel;      // NI x Info
   static constexpr uint32_t bars = info + NI * sizeof(Info);    // mbarriers
   static constexpr int kNumBars = 2 * NK + 2 * NV + 2 * NB + 2 * NI + 4 + 4 + 2 + 1;
-  static constexpr uint32_t misc = bars + 8 * kNumBars;         // tmem addr, abort flag
+  static constexpr uint32_t misc = bars + 8 * kNumBars;         // tmem addr, abort flag, G
   static constexpr uint32_t bytes = misc + 16 + 1024;           // + alignment slack
 };
 static_assert(Layout::bytes <= 232448, "shared memory budget");
-static_assert(Layout::kbuf % 1024 == 0 && Layout::vcode % 1024 == 0 && Layout::vbf % 1024 == 0,
+static_assert(Layout::kbuf % 1024 == 0 && Layout::vcode % 1024 == 0 && Layout::vh % 1024 == 0,
               "swizzled operands need 1024-byte alignment");
 
 struct Bars {
@@ -89,8 +91,8 @@ struct Bars {
   __device__ uint64_t* kempty(int s) { return b + NK + s; }
   __device__ uint64_t* vfull(int s) { return b + 2 * NK + s; }
   __device__ uint64_t* vempty(int s) { return b + 2 * NK + NV + s; }
-  __device__ uint64_t* vbfull(int s) { return b + 2 * NK + 2 * NV + s; }
-  __device__ uint64_t* vbempty(int s) { return b + 2 * NK + 2 * NV + NB + s; }
+  __device__ uint64_t* vhfull(int s) { return b + 2 * NK + 2 * NV + s; }
+  __device__ uint64_t* vhempty(int s) { return b + 2 * NK + 2 * NV + NB + s; }
   __device__ uint64_t* ifull(int s) { return b + 2 * NK + 2 * NV + 2 * NB + s; }
   __device__ uint64_t* iempty(int s) { return b + 2 * NK + 2 * NV + 2 * NB + NI + s; }
   // buffer `buf` of tile g holds S (sfull) / holds P (pfull); the P.V of tile g has
@@ -225,6 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   Bars bars{reinterpret_cast<uint64_t*>(sm + Layout::bars)};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Layout::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Layout::misc + 4);
+  uint32_t* vmax_bits = reinterpret_cast<uint32_t*>(sm + Layout::misc + 8);
   Info* info = reinterpret_cast<Info*>(sm + Layout::info);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -241,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 32) {
     for (int s = 0; s < NK; ++s) { mbar_init(bars.kfull(s), 1); mbar_init(bars.kempty(s), 1); }
     for (int s = 0; s < NV; ++s) { mbar_init(bars.vfull(s), 1); mbar_init(bars.vempty(s), kConvThreads); }
-    for (int s = 0; s < NB; ++s) { mbar_init(bars.vbfull(s), kConvThreads); mbar_init(bars.vbempty(s), 1); }
+    for (int s = 0; s < NB; ++s) { mbar_init(bars.vhfull(s), kConvThreads); mbar_init(bars.vhempty(s), 1); }
     for (int s = 0; s < NI; ++s) { mbar_init(bars.ifull(s), kConvThreads); mbar_init(bars.iempty(s), 256); }
     for (int g = 0; g < 2; ++g) {
       mbar_init(bars.sfull(g, 0), 1);
@@ -252,6 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bars.ofinal(), 1);
     *abort_flag = 0;
+    *vmax_bits = 0u;
     fence_mbar_init();
   }
   if (tid == 0) {
@@ -276,6 +280,48 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // this CTA's slice of the valid tiles (all of them unless split over keys)
+  int n_mine, t_first, t_last;
+  {
+    int T = 0;
+    for (int t = next_tile(0, n_tiles, C, newest, n_valid); t < n_tiles;
+         t = next_tile(t + 1, n_tiles, C, newest, n_valid))
+      ++T;
+    const int per = (T + (int)gridDim.z - 1) / (int)gridDim.z;
+    const int j0 = min(T, (int)blockIdx.z * per);
+    n_mine = min(T, j0 + per) - j0;
+    t_first = next_tile(0, n_tiles, C, newest, n_valid);
+    for (int k = 0; k < j0; ++k) t_first = next_tile(t_first + 1, n_tiles, C, newest, n_valid);
+    t_last = t_first;
+    for (int k = 1; k < n_mine; ++k) t_last = next_tile(t_last + 1, n_tiles, C, newest, n_valid);
+  }
+
+  // G = 2^e >= every V scale of this CTA's valid keys (converters + softmax warps; the
+  // TMA and MMA warps start meanwhile).  Non-negative floats order like their bits.
+  float vnorm = 1.f, vnorm_inv = 1.f;
+  if (warp >= kWarpConv) {
+    constexpr int kN = kThreads - 32 * kWarpConv;
+    float mx = 0.f;
+    if (n_mine > 0) {
+      const int lo = t_first * BN, hi = min(C, (t_last + 1) * BN);
+      const float* vsrow = a.v_scale + (size_t)h * C;
+#pragma unroll 6
+      for (int s = lo + tid - 32 * kWarpConv; s < hi; s += kN) {
+        int age = newest - s;
+        if (age < 0) age += C;
+        if (age < n_valid) mx = fmaxf(mx, __ldg(vsrow + s));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) atomicMax(vmax_bits, __float_as_uint(mx));
+    named_bar(3, kN);
+    // mx < 2^(b - 126) for biased exponent b; b clamped so that G and 1/G are normal
+    const int b = max(1, min(252, (int)((*vmax_bits >> 23) & 0xFFu)));
+    vnorm = __uint_as_float((uint32_t)(b + 1) << 23);
+    vnorm_inv = __uint_as_float((uint32_t)(253 - b) << 23);
+  }
+
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
     if (*abort_flag) return false;
     if (mbar_wait(bar, parity, a.timeouts)) return true;
@@ -286,8 +332,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kWarpTma) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int t = next_tile(0, n_tiles, C, newest, n_valid);
-      for (int j = 0; t < n_tiles; ++j, t = next_tile(t + 1, n_tiles, C, newest, n_valid)) {
+      int t = t_first;
+      for (int j = 0; j < n_mine; ++j, t = next_tile(t + 1, n_tiles, C, newest, n_valid)) {
         const int sk = j % NK, rk = j / NK;
         if (rk > 0 && !wait(bars.kempty(sk), (rk - 1) & 1)) break;
         mbar_arrive_expect_tx(bars.kfull(sk), BN * D);
@@ -302,9 +348,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_e4m3_f32(128, BN);
-      constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);
+      constexpr uint32_t idO = idesc_f16_f32(128, D, 0, 1);
       const uint32_t sQhi = smem_u32(sm + Layout::qhi), sQlo = smem_u32(sm + Layout::qlo);
-      const uint32_t sK = smem_u32(sm + Layout::kbuf), sV = smem_u32(sm + Layout::vbf);
+      const uint32_t sK = smem_u32(sm + Layout::kbuf), sV = smem_u32(sm + Layout::vh);
       // S_g = Q_g K^T into buffer buf of tile g (hi and lo halves of Q accumulate)
       auto issue_s = [&](int gg, int buf, int sk) {
         const uint32_t d = tmem + 128 * gg + 64 * buf;
@@ -330,8 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       int j = 0;
       bool ok = true;
-      int t = next_tile(0, n_tiles, C, newest, n_valid);
-      if (t < n_tiles) {
+      if (n_mine > 0) {
         ok = wait(bars.kfull(0), 0);
         if (ok) {
           tc_fence_after();
@@ -342,9 +387,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_commit(bars.kempty(0));
         }
       }
-      for (; ok && t < n_tiles; ++j) {
-        const int t_next = next_tile(t + 1, n_tiles, C, newest, n_valid);
-        if (t_next < n_tiles) {                        // S of the next tile, one ahead
+      for (; ok && j < n_mine; ++j) {
+        if (j + 1 < n_mine) {                          // S of the next tile, one ahead
           const int jn = j + 1, sk = jn % NK;
           if (!(ok = wait(bars.kfull(sk), (jn / NK) & 1))) break;
           tc_fence_after();
@@ -354,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_commit(bars.sfull(1, jn & 1));
           tc_commit(bars.kempty(sk));
         }
-        if (!(ok = wait(bars.vbfull(j % NB), (j / NB) & 1))) break;
+        if (!(ok = wait(bars.vhfull(j % NB), (j / NB) & 1))) break;
         if (!(ok = wait(bars.pfull(0, j & 1), (j >> 1) & 1))) break;
         tc_fence_after();
         issue_pv(0, j & 1, j % NB, j > 0);
@@ -363,16 +407,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         issue_pv(1, j & 1, j % NB, j > 0);
         tc_commit(bars.pvdone(1));
-        tc_commit(bars.vbempty(j % NB));
-        t = t_next;
+        tc_commit(bars.vhempty(j % NB));
       }
       if (j > 0) tc_commit(bars.ofinal());
       else mbar_arrive(bars.ofinal());
     }
   } else if (warp < kWarpSoft) {
     // ------------------------------------------------------------ converters + key info
-    // 64 threads; thread ct owns key slot ct of every tile: its info, its V row (bf16,
-    // scale folded in).  The scales of the next tile are loaded while this one converts.
+    // 64 threads; thread ct owns key slot ct of every tile: its info, its V row (f16,
+    // scale / G folded in).  The scales of the next tile are loaded while this one converts.
     const int ct = tid - 32 * kWarpConv;          // 0..63
     auto load_scales = [&](int tt, float& ks, float& vs) {
       const int slot = tt * BN + ct;
@@ -381,10 +424,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       vs = in_ring ? __ldg(a.v_scale + (size_t)h * C + slot) : 0.f;
     };
     float pks, pvs;
-    int t = next_tile(0, n_tiles, C, newest, n_valid);
-    load_scales(t, pks, pvs);
-    for (int j = 0; t < n_tiles; ++j) {
-      const int t_next = next_tile(t + 1, n_tiles, C, newest, n_valid);
+    int t = t_first;
+    load_scales(n_mine > 0 ? t : n_tiles, pks, pvs);
+    for (int j = 0; j < n_mine; ++j) {
+      const int t_next = j + 1 < n_mine ? next_tile(t + 1, n_tiles, C, newest, n_valid) : n_tiles;
       const int si = j % NI;
       bool ok = j < NI || wait(bars.iempty(si), ((j / NI) - 1) & 1);
       if (!named_bar_and(1, kConvThreads, ok)) break;   // uniform decision across converters
@@ -397,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (age < 0) age += C;
         if (age < n_valid) {
           ksv = pks * a.score_scale_log2;
-          vsv = pvs;
+          vsv = pvs * vnorm_inv;
           if (age < a.n_current) {
             kbv = 0.f;
             tok = a.n_current - 1 - age;
@@ -416,11 +459,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bars.ifull(si));
       const int sv = j % NV, b = j % NB;
       ok = wait(bars.vfull(sv), (j / NV) & 1);
-      ok = ok && (j < NB || wait(bars.vbempty(b), ((j / NB) - 1) & 1));
+      ok = ok && (j < NB || wait(bars.vhempty(b), ((j / NB) - 1) & 1));
       if (!named_bar_and(2, kConvThreads, ok)) break;
-      // V row ct: 8 chunks of 16 codes (128-byte swizzled) -> bf16(code * vs)
+      // V row ct: 8 chunks of 16 codes (128-byte swizzled) -> f16(code * vs / G)
       const uint8_t* vc = sm + Layout::vcode + sv * BN * D + ct * 128;
-      uint8_t* vb = sm + Layout::vbf + b * 2 * kVPanel;
+      uint8_t* vb = sm + Layout::vh + b * 2 * kVPanel;
       const bool dead = tok == kInvalidTok;
       const uint64_t vs2 = f2_pack(vsv, vsv);
 #pragma unroll
@@ -436,8 +479,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float2 hi = f16x2_to_float2(e4m3x2_to_f16x2((uint16_t)(w[i] >> 16)));
           f2_unpack(f2_mul(f2_pack(lo.x, lo.y), vs2), a0, a1);
           f2_unpack(f2_mul(f2_pack(hi.x, hi.y), vs2), b0, b1);
-          o[2 * i] = pack_bf16x2(a0, a1);
-          o[2 * i + 1] = pack_bf16x2(b0, b1);
+          o[2 * i] = pack_f16x2(a0, a1);
+          o[2 * i + 1] = pack_f16x2(b0, b1);
         }
         *reinterpret_cast<uint4*>(vb + sw128_offset(ct, 16 * c, kVPanel)) =
             make_uint4(o[0], o[1], o[2], o[3]);
@@ -445,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             make_uint4(o[4], o[5], o[6], o[7]);
       }
       fence_proxy_async_smem();
-      mbar_arrive(bars.vbfull(b));
+      mbar_arrive(bars.vhfull(b));
       mbar_arrive(bars.vempty(sv));
       t = t_next;
     }
@@ -462,8 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t r2 = f2_pack(rowmul, rowmul);
     float m_run = -INFINITY, l_run = 0.f;
     int j = 0;
-    for (int t = next_tile(0, n_tiles, C, newest, n_valid); t < n_tiles;
-         t = next_tile(t + 1, n_tiles, C, newest, n_valid), ++j) {
+    for (int t = t_first; j < n_mine; t = next_tile(t + 1, n_tiles, C, newest, n_valid), ++j) {
       const int si = j % NI, buf = j & 1;
       const uint32_t t_s = tmem + lane_base + 128 * g + 64 * buf;   // S_g(j) / P_g(j)
       bool ok = wait(bars.sfull(g, buf), (j >> 1) & 1) && wait(bars.ifull(si), (j / NI) & 1);
@@ -530,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool move = mloc > m_old + kRescaleLog2 || (m_old == -INFINITY && mloc > -INFINITY);
       if (move) m_run = mloc;
       const float mref = (m_run == -INFINITY) ? 0.f : m_run;
-      // pass 2: p = 2^(t - m); P = bf16(p) over the S columns of tensor memory
+      // pass 2: p = 2^(t - m); P = f16(p) over the S columns of tensor memory
       const float off = special ? -mref : a.bias_log2 - mref;
       const uint64_t mul2 = special ? f2_pack(1.f, 1.f) : r2;
       const uint64_t off2 = f2_pack(off, off);
@@ -549,8 +591,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float p0 = ex2(t0), p1 = ex2(t1), p2 = ex2(t2), p3 = ex2(t3);   // 2^-inf = 0
           sum01 = f2_add(sum01, f2_pack(p0, p1));
           sum23 = f2_add(sum23, f2_pack(p2, p3));
-          pk[2 * q8] = pack_bf16x2(p0, p1);
-          pk[2 * q8 + 1] = pack_bf16x2(p2, p3);
+          pk[2 * q8] = pack_f16x2(p0, p1);
+          pk[2 * q8 + 1] = pack_f16x2(p2, p3);
         }
         tmem_st16(t_s + 16 * c, pk);
       }
@@ -585,8 +627,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const bool row_ok = gi < a.n_q;
     const bool any = j > 0;
+    if (a.part_o) {
+      // split over keys: unnormalised O (relative to m_run, times G) and (m_run, l_run)
+      const size_t prow = ((size_t)blockIdx.z * a.n_q + (row_ok ? gi : 0)) * a.H + h;
+      float* po = a.part_o + prow * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        if (any) {
+          tmem_ld32(t_o + 32 * c, o);
+          tmem_wait_ld();
+        }
+        if (row_ok) {
+          float4* d4 = reinterpret_cast<float4*>(po + 32 * c);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            float4 v;
+            v.x = (any && l_run > 0.f) ? __uint_as_float(o[4 * k]) * vnorm : 0.f;
+            v.y = (any && l_run > 0.f) ? __uint_as_float(o[4 * k + 1]) * vnorm : 0.f;
+            v.z = (any && l_run > 0.f) ? __uint_as_float(o[4 * k + 2]) * vnorm : 0.f;
+            v.w = (any && l_run > 0.f) ? __uint_as_float(o[4 * k + 3]) * vnorm : 0.f;
+            if (!ok) v.x = v.y = v.z = v.w = __uint_as_float(0x7FC00000u);
+            d4[k] = v;
+          }
+        }
+      }
+      if (row_ok) {
+        float2* pml = reinterpret_cast<float2*>(a.part_ml) +
+                      ((size_t)blockIdx.z * a.H + h) * a.n_q + gi;
+        *pml = ok ? make_float2(m_run, l_run)
+                  : make_float2(__uint_as_float(0x7FC00000u), __uint_as_float(0x7FC00000u));
+      }
+    } else {
     uint16_t* dst = a.out + ((size_t)(row_ok ? gi : 0) * a.H + h) * D;
-    const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+    const float inv_l = (l_run > 0.f) ? (1.f / l_run) * vnorm : 0.f;
 #pragma unroll 1
     for (int c = 0; c < D / 32; ++c) {
       uint32_t o[32];
@@ -614,6 +688,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) v = __uint_as_float(0x7FC00000u);
       a.lse[(size_t)h * a.n_q + gi] = v;
     }
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -623,10 +698,57 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Merge the split partials of one (query row, head) per warp: M = max m_s over splits
+// with l_s > 0, w_s = 2^(m_s - M), out = sum w_s O_s / sum w_s l_s, lse = (M + log2 L) ln 2.
+__global__ void __launch_bounds__(256) split_combine_kernel(const AttnArgs a, int n_splits) {
+  const int wid = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (wid >= a.n_q * a.H) return;                 // whole warp leaves together
+  const int gi = wid / a.H, h = wid % a.H;
+  const float2* pml = reinterpret_cast<const float2*>(a.part_ml);
+  float M = -INFINITY;
+  bool bad = false;                               // a split that gave up: NaN out
+  for (int z = 0; z < n_splits; ++z) {
+    const float2 ml = pml[((size_t)z * a.H + h) * a.n_q + gi];
+    bad |= isnan(ml.y);
+    if (ml.y > 0.f) M = fmaxf(M, ml.x);
+  }
+  float L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int z = 0; z < n_splits; ++z) {
+    const float2 ml = pml[((size_t)z * a.H + h) * a.n_q + gi];
+    if (!(ml.y > 0.f)) continue;
+    const float w = ex2(ml.x - M);
+    L += w * ml.y;
+    const float4 o = reinterpret_cast<const float4*>(
+        a.part_o + (((size_t)z * a.n_q + gi) * a.H + h) * D)[lane];
+    acc.x += w * o.x;
+    acc.y += w * o.y;
+    acc.z += w * o.z;
+    acc.w += w * o.w;
+  }
+  float inv = L > 0.f ? 1.f / L : 0.f;
+  if (bad) inv = __uint_as_float(0x7FC00000u);
+  uint2 pk;
+  pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+  pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+  reinterpret_cast<uint2*>(a.out + ((size_t)gi * a.H + h) * D)[lane] = pk;
+  if (lane == 0 && a.lse)
+    a.lse[(size_t)h * a.n_q + gi] = bad ? __uint_as_float(0x7FC00000u)
+                                    : L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f
+                                              : -INFINITY;
+}
+
 }  // namespace
 
+int launch_split_combine(const AttnArgs& a, int D_, int n_splits, cudaStream_t s) {
+  if (D_ != D) return KV_EUNSUPPORTED;
+  const int warps = a.n_q * a.H;
+  split_combine_kernel<<<(warps + 7) / 8, 256, 0, s>>>(a, n_splits);
+  return cudaPeekAtLastError() == cudaSuccess ? KV_OK : KV_ECUDA;
+}
+
 int launch_attention_sm100_d128(const AttnArgs& a, const void* tmap_k_sw128,
-                                const void* tmap_v_sw128, cudaStream_t s) {
+                                const void* tmap_v_sw128, cudaStream_t s, int n_splits) {
   static bool configured = false;
   if (!configured) {
     if (cudaFuncSetAttribute(chunk_attn_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -637,7 +759,7 @@ int launch_attention_sm100_d128(const AttnArgs& a, const void* tmap_k_sw128,
   CUtensorMap mk, mv;
   memcpy(&mk, tmap_k_sw128, sizeof(mk));
   memcpy(&mv, tmap_v_sw128, sizeof(mv));
-  dim3 grid((a.n_q + BM - 1) / BM, a.H);
+  dim3 grid((a.n_q + BM - 1) / BM, a.H, n_splits);
   chunk_attn_sm100_kernel<<<grid, kThreads, Layout::bytes, s>>>(mk, mv, a);
   return cudaPeekAtLastError() == cudaSuccess ? KV_OK : KV_ECUDA;
 }

@@ -46,6 +46,10 @@ struct AttnArgs {
   float score_scale_log2;   // softmax_scale * log2(e)
   float bias_log2;          // history_bias * log2(e)
   unsigned int* timeouts;   // device counter of waits that gave up
+  // split over keys (gridDim.z splits): when part_o is set, each split writes its
+  // unnormalised O [split][n_q][H][D] and (m, l) [split][H][n_q] (log2 units) there
+  float* part_o;
+  float* part_ml;
 };
 
 // Device address of the library's wait-timeout counter on the current device.
@@ -58,6 +62,8 @@ int launch_rotate(const RotateArgs& a, int D, cudaStream_t s);
 int launch_attention(const AttnArgs& a, int D, const void* tmap_k, const void* tmap_v,
                      const void* tmap_k_sw128, const void* tmap_v_sw128, cudaStream_t s);
 int launch_attention_sm100_d128(const AttnArgs& a, const void* tmap_k_sw128,
-                                const void* tmap_v_sw128, cudaStream_t s);
+                                const void* tmap_v_sw128, cudaStream_t s, int n_splits = 1);
+// Merge split partials into out (bf16) and lse.
+int launch_split_combine(const AttnArgs& a, int D, int n_splits, cudaStream_t s);
 
 }  // namespace kvring

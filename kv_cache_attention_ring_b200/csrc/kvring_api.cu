@@ -246,9 +246,14 @@ int kv_ring_delta_rotate(kv_ring_t* kv, int64_t delta, void* stream) {
   return KV_OK;
 }
 
-int chunk_attention(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
-                    int n_current, const kv_block_mask_t* mask, const kv_cache_bias_t* bias,
-                    float softmax_scale, void* out, float* lse, uint32_t flags, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared validation and argument set-up of the chunk-attention entry points.
+int attention_args(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0, int n_current,
+                   const kv_block_mask_t* mask, const kv_cache_bias_t* bias,
+                   float softmax_scale, void* out, float* lse, uint32_t flags, AttnArgs* a) {
   int rc = check_ring(kv);
   if (rc) return rc;
   if (flags != 0) return KV_EINVAL;
@@ -269,31 +274,82 @@ int chunk_attention(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
   if (n_current > nv) return KV_ERANGE;
   if (!in_table(kv, q_pos0, q_pos0 + n_q - 1)) return KV_ERANGE;
   if ((int64_t)n_q * kv->n_heads > ((int64_t)1 << 31)) return KV_ERANGE;
-  AttnArgs a;
-  a.q = static_cast<const uint16_t*>(q);
-  a.out = static_cast<uint16_t*>(out);
-  a.lse = lse;
-  a.k_scale = kv->k_scale;
-  a.v_scale = kv->v_scale;
-  a.rope_q0 = kv->rope_table + (size_t)(q_pos0 - kv->rope_pos_min) * kv->head_dim;
-  a.n_q = n_q;
-  a.H = kv->n_heads;
-  a.C = kv->capacity;
-  a.n_current = n_current;
-  a.newest_slot = mod_c(kv->write_slot + kv->pending - 1, kv->capacity);
-  a.n_valid = nv;
-  a.q_first = m.q_first_len;
-  a.q_block = m.q_block_len;
-  a.k_first = m.k_first_len;
-  a.k_block = m.k_block_len;
+  a->q = static_cast<const uint16_t*>(q);
+  a->out = static_cast<uint16_t*>(out);
+  a->lse = lse;
+  a->k_scale = kv->k_scale;
+  a->v_scale = kv->v_scale;
+  a->rope_q0 = kv->rope_table + (size_t)(q_pos0 - kv->rope_pos_min) * kv->head_dim;
+  a->n_q = n_q;
+  a->H = kv->n_heads;
+  a->C = kv->capacity;
+  a->n_current = n_current;
+  a->newest_slot = mod_c(kv->write_slot + kv->pending - 1, kv->capacity);
+  a->n_valid = nv;
+  a->q_first = m.q_first_len;
+  a->q_block = m.q_block_len;
+  a->k_first = m.k_first_len;
+  a->k_block = m.k_block_len;
   const float log2e = 1.4426950408889634f;
-  a.score_scale_log2 = softmax_scale * log2e;
-  a.bias_log2 = b * log2e;
-  a.timeouts = timeout_counter();
-  if (!a.timeouts) return KV_ECUDA;
+  a->score_scale_log2 = softmax_scale * log2e;
+  a->bias_log2 = b * log2e;
+  a->timeouts = nullptr;
+  a->part_o = nullptr;
+  a->part_ml = nullptr;
+  return KV_OK;
+}
+
+// The device-side wait-timeout counter (the one CUDA query of the set-up; host validation
+// comes first so that argument errors are reported without a device).
+int attach_timeouts(AttnArgs* a) {
+  a->timeouts = timeout_counter();
+  return a->timeouts ? KV_OK : KV_ECUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int chunk_attention(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
+                    int n_current, const kv_block_mask_t* mask, const kv_cache_bias_t* bias,
+                    float softmax_scale, void* out, float* lse, uint32_t flags, void* stream) {
+  AttnArgs a;
+  int rc = attention_args(kv, q, n_q, q_pos0, n_current, mask, bias, softmax_scale, out, lse,
+                          flags, &a);
+  if (rc || n_q == 0) return rc;
+  if ((rc = attach_timeouts(&a))) return rc;
   return launch_attention(a, kv->head_dim, kv->opaque + kOpaqueTmapK,
                           kv->opaque + kOpaqueTmapV, kv->opaque + kOpaqueTmapKsw,
                           kv->opaque + kOpaqueTmapVsw, static_cast<cudaStream_t>(stream));
+}
+
+size_t chunk_attention_workspace_size(int n_q, int n_heads, int head_dim, int n_splits) {
+  if (n_q < 0 || n_heads < 1 || head_dim < 1 || n_splits < 1) return 0;
+  return (size_t)n_splits * (size_t)n_q * (size_t)n_heads * ((size_t)head_dim * 4 + 8);
+}
+
+int chunk_attention_split(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
+                          int n_current, const kv_block_mask_t* mask,
+                          const kv_cache_bias_t* bias, float softmax_scale, void* out,
+                          float* lse, int n_splits, void* workspace, size_t workspace_bytes,
+                          uint32_t flags, void* stream) {
+  AttnArgs a;
+  int rc = attention_args(kv, q, n_q, q_pos0, n_current, mask, bias, softmax_scale, out, lse,
+                          flags, &a);
+  if (rc || n_q == 0) return rc;
+  if (kv->head_dim != 128) return KV_EUNSUPPORTED;
+  if (n_splits < 1 || n_splits > 64) return KV_EINVAL;
+  const size_t need = chunk_attention_workspace_size(n_q, kv->n_heads, kv->head_dim, n_splits);
+  if (!workspace || !aligned16(workspace)) return KV_EINVAL;
+  if (workspace_bytes < need) return KV_ERANGE;
+  if ((rc = attach_timeouts(&a))) return rc;
+  a.part_o = static_cast<float*>(workspace);
+  a.part_ml = a.part_o + (size_t)n_splits * n_q * kv->n_heads * kv->head_dim;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  rc = launch_attention_sm100_d128(a, kv->opaque + kOpaqueTmapKsw, kv->opaque + kOpaqueTmapVsw,
+                                   s, n_splits);
+  if (rc) return rc;
+  return launch_split_combine(a, kv->head_dim, n_splits, s);
 }
 
 int kv_wait_timeout_count(uint32_t* host_count) {

@@ -144,3 +144,22 @@ def test_attention_validation_before_launch(L):
     m = kv.kv_block_mask_t(0, 1, 1, 1)
     assert L.chunk_attention(r, 16, 8, 0, 8, ctypes.byref(m), None, 0.125, 16, None, 0,
                              None) == kv.KV_EINVAL
+
+
+def test_split_workspace_size_and_validation(L):
+    assert kv.chunk_attention_workspace_size(25, 32, 128, 8) == 8 * 25 * 32 * (4 * 128 + 8)
+    assert kv.chunk_attention_workspace_size(25, 32, 128, 0) == 0
+    s = _fake_ring(D=128)
+    s.live = 64
+    r = ctypes.byref(s)
+    args = (r, 16, 8, 0, 8, None, None, 0.125, 16, None)
+    need = kv.chunk_attention_workspace_size(8, 2, 128, 4)
+    assert L.chunk_attention_split(*args, 0, 16, need, 0, None) == kv.KV_EINVAL     # splits
+    assert L.chunk_attention_split(*args, 65, 16, need, 0, None) == kv.KV_EINVAL
+    assert L.chunk_attention_split(*args, 4, None, need, 0, None) == kv.KV_EINVAL   # workspace
+    assert L.chunk_attention_split(*args, 4, 17, need, 0, None) == kv.KV_EINVAL     # misaligned
+    assert L.chunk_attention_split(*args, 4, 16, need - 1, 0, None) == kv.KV_ERANGE
+    s64 = _fake_ring(D=64)
+    s64.live = 64
+    assert L.chunk_attention_split(ctypes.byref(s64), 16, 8, 0, 8, None, None, 0.125, 16, None,
+                                   4, 16, need, 0, None) in (kv.KV_EUNSUPPORTED, kv.KV_ECUDA)
