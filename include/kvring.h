@@ -204,6 +204,36 @@ KV_API int chunk_attention_split(const kv_ring_t* kv, const void* q, int n_q, in
                                  float* lse, int n_splits, void* workspace,
                                  size_t workspace_bytes, uint32_t flags, void* stream);
 
+/* Size of the library's own scratch for chunk_attention_split_noalloc: 16 MiB per
+ * device.  8 splits of 25 queries x 32 heads x 128 take 3.3 MB; 4 splits of 1,024
+ * queries x 8 heads x 128 (17.0 MB) do not fit. */
+#define KV_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* chunk_attention_split without a caller workspace, for callers that cannot allocate
+ * device memory at call time: a real-time loop whose memory was reserved up front (the
+ * rings and the model own the whole HBM), code whose allocator must not be entered
+ * while a step runs (cudaMalloc and cudaFree can synchronise the device and so stall
+ * every other stream), or a plain C caller with no allocator at all.  The pages have no
+ * counterpart; this is a convenience of this library.
+ * The partials go to a static device buffer of KV_NOALLOC_SCRATCH_BYTES in the library
+ * (one per device, 256-byte aligned).  The first call on a device looks up that
+ * buffer's address (with that device current) and keeps it; make that first call
+ * before any stream capture.  The call allocates nothing: no cudaMalloc, cudaFree or
+ * allocating library routine.  Nothing in the scratch has to start at zero (every
+ * partial is written before the merge reads it).  There is one scratch per device, so
+ * calls that overlap in time on one device (other streams, other threads) race on it
+ * and give wrong results: order them on one stream.
+ * Arguments and result as chunk_attention_split.  Errors: those of
+ * chunk_attention_split, and KV_ERANGE when chunk_attention_workspace_size(n_q, H, D,
+ * n_splits) exceeds KV_NOALLOC_SCRATCH_BYTES (checked on the host before any CUDA
+ * call); KV_ECUDA when the address lookup fails. */
+KV_API int chunk_attention_split_noalloc(const kv_ring_t* kv, const void* q, int n_q,
+                                         int64_t q_pos0, int n_current,
+                                         const kv_block_mask_t* mask,
+                                         const kv_cache_bias_t* bias, float softmax_scale,
+                                         void* out, float* lse, int n_splits, uint32_t flags,
+                                         void* stream);
+
 /* Static description of a status code.  Never NULL. */
 KV_API const char* kv_status_string(int status);
 

@@ -7,7 +7,8 @@ missing or the device is not sm_100, calls raise.
 
 Entry points (same names as the C ABI): ``kv_rope_table_build``, ``KvRing`` (fills a
 ``kv_ring_t`` and calls ``kv_ring_init``), ``kv_ring_write``, ``kv_ring_commit``,
-``kv_ring_delta_rotate``, ``chunk_attention``, ``kv_status_string``,
+``kv_ring_delta_rotate``, ``chunk_attention``, ``chunk_attention_workspace_size``,
+``chunk_attention_split``, ``chunk_attention_split_noalloc``, ``kv_status_string``,
 ``kv_wait_timeout_count``.
 """
 from __future__ import annotations
@@ -27,7 +28,9 @@ KV_COMMIT = 1
 
 EXPORTS = ("kv_rope_table_build", "kv_ring_init", "kv_ring_write", "kv_ring_commit",
            "kv_ring_delta_rotate", "chunk_attention", "chunk_attention_workspace_size",
-           "chunk_attention_split", "kv_status_string", "kv_wait_timeout_count")
+           "chunk_attention_split", "chunk_attention_split_noalloc", "kv_status_string",
+           "kv_wait_timeout_count")
+KV_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class KvError(RuntimeError):
@@ -83,6 +86,8 @@ def lib() -> ctypes.CDLL:
         L.chunk_attention_workspace_size.restype = ctypes.c_size_t
         L.chunk_attention_split.argtypes = [P, P, I, I64, I, P, P, ctypes.c_float, P, P, I, P,
                                             ctypes.c_size_t, ctypes.c_uint32, P]
+        L.chunk_attention_split_noalloc.argtypes = [P, P, I, I64, I, P, P, ctypes.c_float, P,
+                                                    P, I, ctypes.c_uint32, P]
         _lib = L
     return _lib
 
@@ -234,6 +239,28 @@ def chunk_attention_split(ring: KvRing, q, q_pos0: int, n_current: int, n_splits
                                        None if lse is None else _ptr(lse), int(n_splits),
                                        _ptr(workspace), nbytes, 0, _stream(stream)),
            "chunk_attention_split")
+    return out, lse
+
+
+def chunk_attention_split_noalloc(ring: KvRing, q, q_pos0: int, n_current: int, n_splits: int,
+                                  out, lse=None, mask=None, cache_bias: float = 0.0,
+                                  softmax_scale: float | None = None, stream=None):
+    """chunk_attention_split with the library's static per-device scratch instead of a
+    workspace; `out` (and `lse`, if wanted) are caller-allocated, so the call allocates
+    nothing.  Calls that overlap in time on one device race on the scratch."""
+    import torch
+    assert q.is_cuda and q.dtype == torch.bfloat16 and q.is_contiguous()
+    n_q = int(q.shape[0])
+    assert q.shape == (n_q, ring.H, ring.D) and out.shape == q.shape
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(ring.D)
+    m = None if mask is None else kv_block_mask_t(*(int(x) for x in mask))
+    b = kv_cache_bias_t(float(cache_bias))
+    _check(lib().chunk_attention_split_noalloc(
+        ring.ref, _ptr(q), n_q, int(q_pos0), int(n_current),
+        None if m is None else ctypes.byref(m), ctypes.byref(b), float(softmax_scale),
+        _ptr(out), None if lse is None else _ptr(lse), int(n_splits), 0, _stream(stream)),
+        "chunk_attention_split_noalloc")
     return out, lse
 
 

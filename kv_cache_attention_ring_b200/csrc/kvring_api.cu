@@ -10,6 +10,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "../../include/kvring.h"
 #include "internal.h"
 
@@ -20,6 +22,27 @@ unsigned int* timeout_counter() {
   void* p = nullptr;
   if (cudaGetSymbolAddress(&p, g_wait_timeouts) != cudaSuccess) return nullptr;
   return static_cast<unsigned int*>(p);
+}
+
+// Partials of chunk_attention_split_noalloc: part of the module image, so every device
+// that loads the library has its own copy and no call allocates.
+__device__ __align__(256) unsigned char g_noalloc_scratch[KV_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the current device's scratch, looked up once per device.
+void* noalloc_scratch() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = p;
+  }
+  return g_noalloc_ptr[dev];
 }
 }
 
@@ -344,6 +367,30 @@ int chunk_attention_split(const kv_ring_t* kv, const void* q, int n_q, int64_t q
   if (workspace_bytes < need) return KV_ERANGE;
   if ((rc = attach_timeouts(&a))) return rc;
   a.part_o = static_cast<float*>(workspace);
+  a.part_ml = a.part_o + (size_t)n_splits * n_q * kv->n_heads * kv->head_dim;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  rc = launch_attention_sm100_d128(a, kv->opaque + kOpaqueTmapKsw, kv->opaque + kOpaqueTmapVsw,
+                                   s, n_splits);
+  if (rc) return rc;
+  return launch_split_combine(a, kv->head_dim, n_splits, s);
+}
+
+int chunk_attention_split_noalloc(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
+                                  int n_current, const kv_block_mask_t* mask,
+                                  const kv_cache_bias_t* bias, float softmax_scale, void* out,
+                                  float* lse, int n_splits, uint32_t flags, void* stream) {
+  AttnArgs a;
+  int rc = attention_args(kv, q, n_q, q_pos0, n_current, mask, bias, softmax_scale, out, lse,
+                          flags, &a);
+  if (rc || n_q == 0) return rc;
+  if (kv->head_dim != 128) return KV_EUNSUPPORTED;
+  if (n_splits < 1 || n_splits > 64) return KV_EINVAL;
+  const size_t need = chunk_attention_workspace_size(n_q, kv->n_heads, kv->head_dim, n_splits);
+  if (need > KV_NOALLOC_SCRATCH_BYTES) return KV_ERANGE;
+  if ((rc = attach_timeouts(&a))) return rc;
+  void* scratch = noalloc_scratch();
+  if (!scratch) return KV_ECUDA;
+  a.part_o = static_cast<float*>(scratch);
   a.part_ml = a.part_o + (size_t)n_splits * n_q * kv->n_heads * kv->head_dim;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   rc = launch_attention_sm100_d128(a, kv->opaque + kOpaqueTmapKsw, kv->opaque + kOpaqueTmapVsw,

@@ -163,3 +163,21 @@ def test_split_workspace_size_and_validation(L):
     s64.live = 64
     assert L.chunk_attention_split(ctypes.byref(s64), 16, 8, 0, 8, None, None, 0.125, 16, None,
                                    4, 16, need, 0, None) in (kv.KV_EUNSUPPORTED, kv.KV_ECUDA)
+
+
+def test_noalloc_rejects_oversize_before_any_cuda_call(L):
+    s = _fake_ring(C=4096, D=128)
+    s.live = 2048
+    r = ctypes.byref(s)
+    assert kv.KV_NOALLOC_SCRATCH_BYTES == 16 << 20
+    # 1,024 queries x 2 heads x 128 x 9 splits = 9.6 MB fits; 17 splits (18.1 MB) do not
+    assert kv.chunk_attention_workspace_size(1024, 2, 128, 17) > kv.KV_NOALLOC_SCRATCH_BYTES
+    assert L.chunk_attention_split_noalloc(r, 16, 1024, 0, 8, None, None, 0.125, 16, None,
+                                           17, 0, None) == kv.KV_ERANGE
+    assert L.chunk_attention_split_noalloc(r, 16, 1024, 0, 8, None, None, 0.125, 16, None,
+                                           0, 0, None) == kv.KV_EINVAL
+    assert L.chunk_attention_split_noalloc(r, 16, 0, 0, 8, None, None, 0.125, 16, None,
+                                           4, 0, None) == kv.KV_OK          # nothing to do
+    # within the limit the call reaches the device (none here)
+    assert L.chunk_attention_split_noalloc(r, 16, 1024, 0, 8, None, None, 0.125, 16, None,
+                                           9, 0, None) == kv.KV_ECUDA
