@@ -267,7 +267,7 @@ def rotate_timing(torch, kv, inputs, dev, reps: int = 20) -> dict:
 def e2e_timing(torch, kv, step: RunwayStep, steps: int, stream) -> dict:
     """Same step through the public API from pinned host buffers: every call copies its
     q, k, v host->device and its output device->host inside the timed region."""
-    n_sets = 8
+    n_sets = min(8, step.n_rings)
     host = []
     for s in range(n_sets):
         host.append([[step.q[s][p].cpu().pin_memory(), step.k[s][p].cpu().pin_memory(),
