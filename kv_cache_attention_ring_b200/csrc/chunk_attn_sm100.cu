@@ -77,7 +77,7 @@ struct Layout {
   static constexpr uint32_t vh = vcode + NV * BN * D;           // NB x f16 2 panels, sw128
   static constexpr uint32_t info = vh + NB * 2 * kVPanel;      // NI x Info
   static constexpr uint32_t bars = info + NI * sizeof(Info);    // mbarriers
-  static constexpr int kNumBars = 2 * NK + 2 * NV + 2 * NB + 2 * NI + 4 + 4 + 2 + 1;
+  static constexpr int kNumBars = 2 * NK + 2 * NV + 2 * NB + 2 * NI + 4 + 4 + 1;
   static constexpr uint32_t misc = bars + 8 * kNumBars;         // tmem addr, abort flag, G
   static constexpr uint32_t bytes = misc + 16 + 1024;           // + alignment slack
 };
@@ -95,13 +95,13 @@ struct Bars {
   __device__ uint64_t* vhempty(int s) { return b + 2 * NK + 2 * NV + NB + s; }
   __device__ uint64_t* ifull(int s) { return b + 2 * NK + 2 * NV + 2 * NB + s; }
   __device__ uint64_t* iempty(int s) { return b + 2 * NK + 2 * NV + 2 * NB + NI + s; }
-  // buffer `buf` of tile g holds S (sfull) / holds P (pfull); the P.V of tile g has
-  // completed (pvdone); all MMAs are done (ofinal).  P-ready is per buffer because the
-  // softmax may finish tile j+1 before the MMA issuer has consumed tile j's signal.
+  // buffer `buf` of tile g holds S (sfull) / holds P (pfull); all MMAs are done (ofinal).
+  // P-ready is per buffer because the softmax may finish tile j+1 before the MMA issuer
+  // has consumed tile j's signal.  The P.V of key tile j (both query tiles) has completed
+  // when V buffer j % NB is released (vhempty).
   __device__ uint64_t* sfull(int g, int buf) { return b + 2 * (NK + NV + NB + NI) + 2 * g + buf; }
   __device__ uint64_t* pfull(int g, int buf) { return b + 2 * (NK + NV + NB + NI) + 4 + 2 * g + buf; }
-  __device__ uint64_t* pvdone(int g) { return b + 2 * (NK + NV + NB + NI) + 8 + g; }
-  __device__ uint64_t* ofinal() { return b + 2 * (NK + NV + NB + NI) + 10; }
+  __device__ uint64_t* ofinal() { return b + 2 * (NK + NV + NB + NI) + 8; }
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -251,7 +251,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bars.sfull(g, 1), 1);
       mbar_init(bars.pfull(g, 0), 128);
       mbar_init(bars.pfull(g, 1), 128);
-      mbar_init(bars.pvdone(g), 1);
     }
     mbar_init(bars.ofinal(), 1);
     *abort_flag = 0;
@@ -323,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (mbar_try_wait(bar, parity)) return true;       // fast path: already complete
     if (*abort_flag) return false;
     if (mbar_wait(bar, parity, a.timeouts)) return true;
     *abort_flag = 1;
@@ -352,62 +352,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sQhi = smem_u32(sm + Layout::qhi), sQlo = smem_u32(sm + Layout::qlo);
       const uint32_t sK = smem_u32(sm + Layout::kbuf), sV = smem_u32(sm + Layout::vh);
       // S_g = Q_g K^T into buffer buf of tile g (hi and lo halves of Q accumulate)
+      // descriptors are built once; a step of s bytes adds s >> 4 to the start field
+      const uint64_t dQhi = smem_desc_sw128(sQhi, 16, 1024), dQlo = smem_desc_sw128(sQlo, 16, 1024);
+      const uint64_t dK = smem_desc_sw128(sK, 16, 1024), dV = smem_desc_sw128(sV, kVPanel, 1024);
       auto issue_s = [&](int gg, int buf, int sk) {
         const uint32_t d = tmem + 128 * gg + 64 * buf;
-        const uint32_t kb = sK + sk * BN * D;
+        const uint64_t qh = dQhi + ((gg * 128 * D) >> 4), ql = dQlo + ((gg * 128 * D) >> 4);
+        const uint64_t kd = dK + ((sk * BN * D) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk)
-          tc_mma_f8_ss(d, smem_desc_sw128(sQhi + gg * 128 * D + kk * 32, 16, 1024),
-                       smem_desc_sw128(kb + kk * 32, 16, 1024), idS, kk > 0);
+          tc_mma_f8_ss(d, qh + 2 * kk, kd + 2 * kk, idS, kk > 0);
 #pragma unroll
-        for (int kk = 0; kk < D / 32; ++kk)
-          tc_mma_f8_ss(d, smem_desc_sw128(sQlo + gg * 128 * D + kk * 32, 16, 1024),
-                       smem_desc_sw128(kb + kk * 32, 16, 1024), idS, 1);
+        for (int kk = 0; kk < D / 32; ++kk) tc_mma_f8_ss(d, ql + 2 * kk, kd + 2 * kk, idS, 1);
       };
       // O_g (+)= P_g V with P_g read from tensor memory (buffer buf)
       auto issue_pv = [&](int gg, int buf, int vbi, uint32_t acc) {
         const uint32_t d = tmem + 256 + 128 * gg;
         const uint32_t p = tmem + 128 * gg + 64 * buf;
-        const uint32_t vb = sV + vbi * 2 * kVPanel;
+        const uint64_t vd = dV + ((vbi * 2 * kVPanel) >> 4);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          tc_mma_f16_ts(d, p + 8 * kk, smem_desc_sw128(vb + kk * 2048, kVPanel, 1024), idO,
-                        acc | (kk > 0));
+          tc_mma_f16_ts(d, p + 8 * kk, vd + 128 * kk, idO, acc | (kk > 0));
+      };
+      // S_g(jj) into buffer jj & 1; tile 1 of the CTA starts two S groups after tile 0, so
+      // the two softmax groups drift apart and take turns on the exp unit.
+      auto s_group = [&](int gg, int jj) -> bool {
+        const int sk = jj % NK;
+        if (gg == 0) {
+          if (!wait(bars.kfull(sk), (jj / NK) & 1)) return false;
+          tc_fence_after();
+        }
+        issue_s(gg, jj & 1, sk);
+        tc_commit(bars.sfull(gg, jj & 1));
+        if (gg == 1) tc_commit(bars.kempty(sk));       // both tiles have read K(jj)
+        return true;
       };
       int j = 0;
       bool ok = true;
-      if (n_mine > 0) {
-        ok = wait(bars.kfull(0), 0);
-        if (ok) {
-          tc_fence_after();
-          issue_s(0, 0, 0);
-          tc_commit(bars.sfull(0, 0));
-          issue_s(1, 0, 0);
-          tc_commit(bars.sfull(1, 0));
-          tc_commit(bars.kempty(0));
-        }
-      }
+      for (int gg = 0; gg < 2 && ok; ++gg)
+        for (int jj = 0; jj < 2 && jj < n_mine && ok; ++jj) ok = s_group(gg, jj);
+      // per key tile j and query tile g: P.V(j) as soon as P_g(j) is ready, then S_g(j + 2)
+      // into the buffer P_g(j) occupied (tensor-core operations run in issue order)
       for (; ok && j < n_mine; ++j) {
-        if (j + 1 < n_mine) {                          // S of the next tile, one ahead
-          const int jn = j + 1, sk = jn % NK;
-          if (!(ok = wait(bars.kfull(sk), (jn / NK) & 1))) break;
-          tc_fence_after();
-          issue_s(0, jn & 1, sk);
-          tc_commit(bars.sfull(0, jn & 1));
-          issue_s(1, jn & 1, sk);
-          tc_commit(bars.sfull(1, jn & 1));
-          tc_commit(bars.kempty(sk));
-        }
         if (!(ok = wait(bars.vhfull(j % NB), (j / NB) & 1))) break;
-        if (!(ok = wait(bars.pfull(0, j & 1), (j >> 1) & 1))) break;
-        tc_fence_after();
-        issue_pv(0, j & 1, j % NB, j > 0);
-        tc_commit(bars.pvdone(0));
-        if (!(ok = wait(bars.pfull(1, j & 1), (j >> 1) & 1))) break;
-        tc_fence_after();
-        issue_pv(1, j & 1, j % NB, j > 0);
-        tc_commit(bars.pvdone(1));
-        tc_commit(bars.vhempty(j % NB));
+        for (int gg = 0; gg < 2; ++gg) {
+          if (!(ok = wait(bars.pfull(gg, j & 1), (j >> 1) & 1))) break;
+          tc_fence_after();
+          issue_pv(gg, j & 1, j % NB, j > 0);
+          if (gg == 1) tc_commit(bars.vhempty(j % NB));
+          if (j + 2 < n_mine && !(ok = s_group(gg, j + 2))) break;
+        }
       }
       if (j > 0) tc_commit(bars.ofinal());
       else mbar_arrive(bars.ofinal());
@@ -526,9 +520,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float4* k4 = reinterpret_cast<const float4*>(in.kscl);
       float m0 = -INFINITY, m1 = -INFINITY;
       if (!special) {
+        // key scales in two batches of 8 shared-memory loads, so their latency overlaps
+        float4 kq[8];
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
-          const float4 ks = k4[q];
+          if ((q & 7) == 0) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) kq[i] = k4[q + i];
+          }
+          const float4 ks = kq[q & 7];
           float u0, u1, u2, u3;
           f2_unpack(f2_mul(f2_pack(__uint_as_float(sr[4 * q]), __uint_as_float(sr[4 * q + 1])),
                            f2_pack(ks.x, ks.y)), u0, u1);
@@ -604,7 +604,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       l_run = l_run * alpha + ((s0 + s1) + (s2 + s3));
       // rescale O_g once the previous P.V of this tile has landed (rare; warp-collective)
       if (__any_sync(0xffffffffu, scale_o)) {
-        ok = wait(bars.pvdone(g), (j - 1) & 1);
+        // P.V(j - 1) of both tiles has completed once V buffer (j - 1) is released
+        ok = wait(bars.vhempty((j - 1) % NB), ((j - 1) / NB) & 1);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
 #pragma unroll 1

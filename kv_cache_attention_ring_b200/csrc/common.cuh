@@ -345,6 +345,56 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
+// Maximum that propagates NaN (any NaN input gives NaN).
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+__device__ __forceinline__ float max3_nan(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Row quantisation rule shared by the ring write and the delta rotation, for the 16
+// values this lane owns of a row spread over G lanes (one 16-byte store of codes):
+// scale = fl32(amax / 448), codes = e4m3(fl32(y * fl32(448 / amax))); amax = 0 or
+// 448/amax not finite -> scale 0 and zero codes; a NaN or infinite value anywhere in
+// the row -> NaN scale and 0x7F codes.  The row maximum propagates NaN, so one test of
+// it replaces a finiteness test per element.  Every lane of the group returns the same
+// *scale_out.
+template <int G>
+__device__ __forceinline__ uint4 quant_row16(const float (&y)[16], float* scale_out) {
+  float amax = max3_nan(fabsf(y[0]), fabsf(y[1]), fabsf(y[2]));
+#pragma unroll
+  for (int i = 3; i < 15; i += 2) amax = max3_nan(amax, fabsf(y[i]), fabsf(y[i + 1]));
+  amax = max_nan(amax, fabsf(y[15]));
+#pragma unroll
+  for (int off = G / 2; off > 0; off >>= 1)
+    amax = max_nan(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  if (!(amax <= 3.402823466e38f)) {                 // NaN or infinity in the row
+    *scale_out = __uint_as_float(0x7FC00000u);
+    return make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+  }
+  const float inv = (amax > 0.f) ? div_rn(448.f, amax) : 0.f;
+  if (!(amax > 0.f) || !isfinite(inv)) {
+    *scale_out = 0.f;
+    return make_uint4(0u, 0u, 0u, 0u);
+  }
+  *scale_out = div_rn(amax, 448.f);
+  const uint64_t inv2 = f2_pack(inv, inv);
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float a0, a1, b0, b1;
+    f2_unpack(f2_mul(f2_pack(y[4 * i], y[4 * i + 1]), inv2), a0, a1);
+    f2_unpack(f2_mul(f2_pack(y[4 * i + 2], y[4 * i + 3]), inv2), b0, b1);
+    w[i] = e4m3x2(a0, a1) | (e4m3x2(b0, b1) << 16);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // Shared-memory matrix descriptor (sm_100 format): start>>4 in [0,14), LBO>>4 in [16,30),
 // SBO>>4 in [32,46), fixed version 1 in [46,48), swizzle mode in [61,64) (2 = 128-byte).
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes,

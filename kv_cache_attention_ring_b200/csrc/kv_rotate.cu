@@ -16,93 +16,80 @@ namespace kvring {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kRows = 8;        // rows per lane group: all their loads are in flight at once
 
-template <int D>
-__global__ void __launch_bounds__(kThreads) kv_rotate_kernel(const RotateArgs a) {
-  constexpr int G = D / 16;
-  __shared__ float4 s_cs[D / 4];
-  if (threadIdx.x < D / 4)
-    s_cs[threadIdx.x] = make_float4(a.cs[4 * threadIdx.x], a.cs[4 * threadIdx.x + 1],
-                                    a.cs[4 * threadIdx.x + 2], a.cs[4 * threadIdx.x + 3]);
-  __syncthreads();
-
-  const int lane_in_row = threadIdx.x % G;
-  const int64_t row = (int64_t)blockIdx.x * (kThreads / G) + threadIdx.x / G;
-  const int64_t rows = a.count * a.H;
-  const bool active = row < rows;
-  const int64_t r = active ? row : rows - 1;
-  const int h = (int)(r / a.count);
-  const int64_t i = r % a.count;
-  int64_t slot = a.first_slot + i;
-  if (slot >= a.C) slot -= a.C;
-  const int e0 = lane_in_row * 16;
-  const size_t at = ((size_t)h * a.C + slot);
-
-  const uint4 raw = *reinterpret_cast<const uint4*>(a.kc + at * D + e0);
-  const float sc = a.ks[at];
+// Rotate and requantise one row's 16 codes (this lane's share); returns the new codes and,
+// through *scale_out, the row's new scale (the same in every lane of the group).
+template <int G>
+__device__ __forceinline__ uint4 rotate16(uint4 raw, float sc, const float4* cs4,
+                                          float* scale_out) {
   const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-  float x[16], y[16];
+  const uint64_t sc2 = f2_pack(sc, sc);
+  float y[16];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const float2 lo = f16x2_to_float2(e4m3x2_to_f16x2((uint16_t)(w[j] & 0xFFFFu)));
     const float2 hi = f16x2_to_float2(e4m3x2_to_f16x2((uint16_t)(w[j] >> 16)));
-    x[4 * j] = mul_rn(lo.x, sc);
-    x[4 * j + 1] = mul_rn(lo.y, sc);
-    x[4 * j + 2] = mul_rn(hi.x, sc);
-    x[4 * j + 3] = mul_rn(hi.y, sc);
-  }
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float4 cs = s_cs[e0 / 4 + j];
-    float x0 = x[4 * j], x1 = x[4 * j + 1];
+    const float4 cs = cs4[j];
+    float x0, x1, x2, x3;
+    f2_unpack(f2_mul(f2_pack(lo.x, lo.y), sc2), x0, x1);
+    f2_unpack(f2_mul(f2_pack(hi.x, hi.y), sc2), x2, x3);
     y[4 * j] = sub_rn(mul_rn(x0, cs.x), mul_rn(x1, cs.y));
     y[4 * j + 1] = add_rn(mul_rn(x0, cs.y), mul_rn(x1, cs.x));
-    x0 = x[4 * j + 2];
-    x1 = x[4 * j + 3];
+    x0 = x2;
+    x1 = x3;
     y[4 * j + 2] = sub_rn(mul_rn(x0, cs.z), mul_rn(x1, cs.w));
     y[4 * j + 3] = add_rn(mul_rn(x0, cs.w), mul_rn(x1, cs.z));
   }
+  return quant_row16<G>(y, scale_out);      // the write's row rule
+}
 
-  // requantise (same row rule as the write)
-  float amax = 0.f;
-  uint32_t bad = 0;
+// Grid (slot blocks, heads).  A block covers kRows passes of kThreads / G consecutive
+// valid slots of head blockIdx.y; lane group g of pass k owns valid slot
+// blockIdx.x * (kRows * kThreads / G) + k * (kThreads / G) + g (counted from the oldest).
+// Every lane first issues the loads of all its rows, then rotates and stores them.
+template <int D>
+__global__ void __launch_bounds__(kThreads) kv_rotate_kernel(const RotateArgs a) {
+  constexpr int G = D / 16;
+  constexpr int kPass = kThreads / G;
+  __shared__ float4 s_cs[D / 4];
+  if (threadIdx.x < D / 4)
+    s_cs[threadIdx.x] = make_float4(a.cs[4 * threadIdx.x], a.cs[4 * threadIdx.x + 1],
+                                    a.cs[4 * threadIdx.x + 2], a.cs[4 * threadIdx.x + 3]);
+
+  const int lane_in_row = threadIdx.x % G;
+  const int e0 = lane_in_row * 16;
+  const int h = blockIdx.y;
+  const int count = (int)a.count;
+  const int i0 = blockIdx.x * (kRows * kPass) + threadIdx.x / G;
+  uint8_t* const kc_h = a.kc + (size_t)h * a.C * D + e0;
+  float* const ks_h = a.ks + (size_t)h * a.C;
+  auto slot_of = [&](int k) {
+    const int i = min(i0 + k * kPass, count - 1);     // all lanes stay for the shuffles
+    int sl = (int)a.first_slot + i;
+    return sl >= a.C ? sl - a.C : sl;
+  };
+  uint4 raw[kRows];
+  float sc[kRows];
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    amax = fmaxf(amax, fabsf(y[k]));
-    bad |= (uint32_t)!isfinite(y[k]);
+  for (int k = 0; k < kRows; ++k) {
+    const int sl = slot_of(k);
+    raw[k] = *reinterpret_cast<const uint4*>(kc_h + (size_t)sl * D);
+    sc[k] = ks_h[sl];
   }
+  __syncthreads();   // s_cs ready; every lane has read its rows before any store below
+  const float4* cs4 = s_cs + e0 / 4;
 #pragma unroll
-  for (int off = G / 2; off > 0; off >>= 1) {
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    bad |= __shfl_xor_sync(0xffffffffu, bad, off);
-  }
-  uint4 q;
-  float scale;
-  const float inv = (amax > 0.f) ? div_rn(448.f, amax) : 0.f;
-  if (bad) {
-    scale = __uint_as_float(0x7FC00000u);
-    q = make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
-  } else if (!(amax > 0.f) || !isfinite(inv)) {
-    scale = 0.f;
-    q = make_uint4(0u, 0u, 0u, 0u);
-  } else {
-    scale = div_rn(amax, 448.f);
-    uint32_t o[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t lo = e4m3x2(mul_rn(y[4 * j], inv), mul_rn(y[4 * j + 1], inv));
-      const uint32_t hi = e4m3x2(mul_rn(y[4 * j + 2], inv), mul_rn(y[4 * j + 3], inv));
-      o[j] = lo | (hi << 16);
-    }
-    q = make_uint4(o[0], o[1], o[2], o[3]);
-  }
-  // every lane of the row has read its codes before any lane overwrites the row's scale
-  __syncwarp();
-  if (active) {
-    *reinterpret_cast<uint4*>(a.kc + at * D + e0) = q;
-    if (lane_in_row == 0) {
-      a.ks[at] = scale;
-      if (h == 0) a.slot_pos[slot] += a.delta;
+  for (int k = 0; k < kRows; ++k) {
+    float scale;
+    const uint4 q = rotate16<G>(raw[k], sc[k], cs4, &scale);
+    if (i0 + k * kPass < count) {
+      const int sl = slot_of(k);
+      *reinterpret_cast<uint4*>(kc_h + (size_t)sl * D) = q;
+      if (lane_in_row == 0) {
+        ks_h[sl] = scale;
+        if (h == 0) a.slot_pos[sl] += a.delta;
+      }
     }
   }
 }
@@ -110,10 +97,10 @@ __global__ void __launch_bounds__(kThreads) kv_rotate_kernel(const RotateArgs a)
 template <int D>
 int launch_rotate_d(const RotateArgs& a, cudaStream_t s) {
   constexpr int G = D / 16;
-  const int64_t rows = a.count * a.H;
-  if (rows == 0) return KV_OK;
-  const int64_t blocks = (rows + (kThreads / G) - 1) / (kThreads / G);
-  kv_rotate_kernel<D><<<(unsigned)blocks, kThreads, 0, s>>>(a);
+  if (a.count == 0 || a.H == 0) return KV_OK;
+  const int64_t per_block = (int64_t)kRows * (kThreads / G);
+  const dim3 grid((unsigned)((a.count + per_block - 1) / per_block), (unsigned)a.H);
+  kv_rotate_kernel<D><<<grid, kThreads, 0, s>>>(a);
   return cudaPeekAtLastError() == cudaSuccess ? KV_OK : KV_ECUDA;
 }
 

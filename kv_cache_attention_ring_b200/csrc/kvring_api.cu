@@ -171,6 +171,7 @@ int kv_ring_init(kv_ring_t* kv) {
     return KV_EINVAL;
   if (kv->rope_pos_max < kv->rope_pos_min || !(kv->rope_base > 0.0)) return KV_EINVAL;
   if ((int64_t)kv->capacity * kv->n_heads > (int64_t)1 << 31) return KV_ERANGE;
+  if (kv->n_heads > 65535) return KV_ERANGE;          // heads index grid dimension y
   int dev = 0, major = 0, minor = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return KV_ECUDA;
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
