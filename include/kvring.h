@@ -94,7 +94,7 @@ extern "C" {
  *   write_slot + pending - 1 (mod capacity). */
 typedef struct kv_ring {
   int32_t capacity;          /* C: number of slots, >= 1 */
-  int32_t n_heads;           /* H */
+  int32_t n_heads;           /* H, 1..65535 */
   int32_t head_dim;          /* D: 64 or 128 */
   int32_t initialized;       /* set by kv_ring_init; do not write */
   int64_t write_slot;        /* physical slot of the first pending/next token, [0, C) */
