@@ -16,7 +16,7 @@ namespace kvring {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kRows = 8;        // rows per lane group: all their loads are in flight at once
+constexpr int kRows = 4;        // rows per lane group: all their loads are in flight at once
 
 // Rotate and requantise one row's 16 codes (this lane's share); returns the new codes and,
 // through *scale_out, the row's new scale (the same in every lane of the group).
@@ -49,7 +49,7 @@ __device__ __forceinline__ uint4 rotate16(uint4 raw, float sc, const float4* cs4
 // blockIdx.x * (kRows * kThreads / G) + k * (kThreads / G) + g (counted from the oldest).
 // Every lane first issues the loads of all its rows, then rotates and stores them.
 template <int D>
-__global__ void __launch_bounds__(kThreads) kv_rotate_kernel(const RotateArgs a) {
+__global__ void __launch_bounds__(kThreads, 4) kv_rotate_kernel(const RotateArgs a) {
   constexpr int G = D / 16;
   constexpr int kPass = kThreads / G;
   __shared__ float4 s_cs[D / 4];

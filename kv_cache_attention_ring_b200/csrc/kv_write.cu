@@ -5,9 +5,10 @@
 //
 // HBM-bound streaming kernel.  A row is one (token, head) pair; G = D/16 threads share a
 // row and each owns 16 consecutive elements (8 rotation pairs): 16-byte vector loads of
-// the inputs and of the (cos, sin) table, one 16-byte store of 16 codes each for K and V.  The row's amax
-// and non-finite flag are reduced with shuffles inside the G-lane group.  Algorithmic
-// traffic per row: 2*D*sizeof(in) read + 2*D codes + 2 scales (+ slot position) written.
+// the inputs and of the (cos, sin) table, one 16-byte store of 16 codes each for K and V.
+// The row's maximum magnitude (NaN-propagating) is reduced with shuffles inside the
+// G-lane group.  Algorithmic traffic per row: 2*D*sizeof(in) read + 2*D codes + 2 scales
+// (+ slot position) written.
 #include "common.cuh"
 #include "internal.h"
 #include "../../include/kvring.h"
@@ -17,7 +18,7 @@ namespace kvring {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kRows = 2;        // rows per lane group: all their loads are in flight at once
+constexpr int kRows = 1;        // rows per lane group (more in flight cost occupancy here)
 
 template <typename T>
 struct In;
