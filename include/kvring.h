@@ -76,6 +76,10 @@ extern "C" {
 
 /* ------------------------------------------------------------------ flags */
 #define KV_COMMIT 1u          /* kv_ring_write: commit the chunk after writing it */
+#define KV_QK_FP8 1u          /* chunk_attention*: "mode B" -- the rotated bf16 query row is
+                                 also quantised to e4m3 by the write's row rule (one fp32
+                                 scale per row) and Q.K^T runs as one e4m3 MMA set instead
+                                 of the exact hi + lo pair; head_dim 128 only */
 
 /* Per-stream ring-head state.  Plain data: the caller fills the shape, the device
  * pointers, the RoPE table fields and next_pos, then calls kv_ring_init.  Copying the
@@ -177,8 +181,10 @@ KV_API int kv_ring_delta_rotate(kv_ring_t* kv, int64_t delta, void* stream);
  * chunk (masked by `mask`, no bias), the rest are history (bias added, always visible).
  * out: device bf16 [n_q][H][D]; lse: device fp32 [H][n_q] natural-log sum of exp, or
  * NULL.  A row with no visible key gets out = 0 and lse = -inf.  softmax_scale > 0.
- * flags must be 0.  Errors: KV_EINVAL, KV_ERANGE (n_current > valid slots, a query
- * position outside the table), KV_ESTATE, KV_ECUDA. */
+ * flags: 0 (the query stays bf16: exact, "mode A") or KV_QK_FP8 (mode B; its result
+ * matches the definition evaluated on the quantised-then-dequantised query).  Errors:
+ * KV_EINVAL (also an unknown flag), KV_ERANGE (n_current > valid slots, a query position
+ * outside the table), KV_EUNSUPPORTED (KV_QK_FP8 at head_dim 64), KV_ESTATE, KV_ECUDA. */
 KV_API int chunk_attention(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
                     int n_current, const kv_block_mask_t* mask, const kv_cache_bias_t* bias,
                     float softmax_scale, void* out, float* lse, uint32_t flags, void* stream);

@@ -25,6 +25,7 @@ LIB_PATH = os.path.join(_HERE, "libkvring.so")
 KV_OK, KV_EINVAL, KV_ERANGE, KV_EUNSUPPORTED, KV_ECUDA, KV_ESTATE = 0, -1, -2, -3, -4, -5
 KV_DTYPE_BF16, KV_DTYPE_FP32 = 1, 2
 KV_COMMIT = 1
+KV_QK_FP8 = 1
 
 EXPORTS = ("kv_rope_table_build", "kv_ring_init", "kv_ring_write", "kv_ring_commit",
            "kv_ring_delta_rotate", "chunk_attention", "chunk_attention_workspace_size",
@@ -186,7 +187,7 @@ def kv_ring_delta_rotate(ring: KvRing, delta: int, stream=None) -> None:
 
 def chunk_attention(ring: KvRing, q, q_pos0: int, n_current: int, mask=None,
                     cache_bias: float = 0.0, softmax_scale: float | None = None, out=None,
-                    lse=None, want_lse: bool = True, stream=None):
+                    lse=None, want_lse: bool = True, stream=None, mode_b: bool = False):
     """q: bf16 [n_q][H][D] on the GPU.  mask: (q_first, q_block, k_first, k_block) or None.
     Returns (out bf16 [n_q][H][D], lse fp32 [H][n_q] or None)."""
     import torch
@@ -204,7 +205,8 @@ def chunk_attention(ring: KvRing, q, q_pos0: int, n_current: int, mask=None,
     _check(lib().chunk_attention(ring.ref, _ptr(q), n_q, int(q_pos0), int(n_current),
                                  None if m is None else ctypes.byref(m), ctypes.byref(b),
                                  float(softmax_scale), _ptr(out),
-                                 None if lse is None else _ptr(lse), 0, _stream(stream)),
+                                 None if lse is None else _ptr(lse),
+                                 KV_QK_FP8 if mode_b else 0, _stream(stream)),
            "chunk_attention")
     return out, lse
 
@@ -217,7 +219,7 @@ def chunk_attention_workspace_size(n_q: int, n_heads: int, head_dim: int, n_spli
 def chunk_attention_split(ring: KvRing, q, q_pos0: int, n_current: int, n_splits: int,
                           workspace, mask=None, cache_bias: float = 0.0,
                           softmax_scale: float | None = None, out=None, lse=None,
-                          want_lse: bool = True, stream=None):
+                          want_lse: bool = True, stream=None, mode_b: bool = False):
     """chunk_attention with the keys split over n_splits groups; `workspace` is a device
     tensor of at least chunk_attention_workspace_size(...) bytes."""
     import torch
@@ -237,7 +239,8 @@ def chunk_attention_split(ring: KvRing, q, q_pos0: int, n_current: int, n_splits
                                        None if m is None else ctypes.byref(m), ctypes.byref(b),
                                        float(softmax_scale), _ptr(out),
                                        None if lse is None else _ptr(lse), int(n_splits),
-                                       _ptr(workspace), nbytes, 0, _stream(stream)),
+                                       _ptr(workspace), nbytes, KV_QK_FP8 if mode_b else 0,
+                                       _stream(stream)),
            "chunk_attention_split")
     return out, lse
 

@@ -218,6 +218,54 @@ __device__ __forceinline__ void q_split(const AttnArgs& a, int gi, int h, int k,
   }
 }
 
+// Mode B: quantise bf16(RoPE(q_gi)) to e4m3 by the write's row rule (scale = amax/448,
+// codes = e4m3(y * (448/amax)); zero rows -> scale 0; a non-finite element -> NaN scale)
+// into the swizzled K-major operand row; returns the row's scale.  Rows beyond n_q get
+// zero codes and scale 0.
+__device__ __forceinline__ float q_quant_b(const AttnArgs& a, int gi, int h, uint8_t* qc, int row) {
+  if (gi >= a.n_q) {
+#pragma unroll
+    for (int c = 0; c < D / 16; ++c)
+      *reinterpret_cast<uint4*>(qc + row * 128 + ((c ^ (row & 7)) << 4)) = make_uint4(0, 0, 0, 0);
+    return 0.f;
+  }
+  float amax = 0.f;
+#pragma unroll 4
+  for (int c = 0; c < D / 8; ++c) {
+    float y[8];
+    q_rot8(a, gi, h, c, y);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) amax = max_nan(amax, fabsf(y[e]));
+  }
+  float inv = 0.f, scale = 0.f;
+  bool zero = false;
+  if (!(amax <= 3.402823466e38f)) {
+    scale = __uint_as_float(0x7FC00000u);
+  } else {
+    inv = amax > 0.f ? div_rn(448.f, amax) : 0.f;
+    zero = !(amax > 0.f) || !isfinite(inv);
+    scale = zero ? 0.f : div_rn(amax, 448.f);
+  }
+  const bool bad = isnan(scale);
+#pragma unroll 2
+  for (int c = 0; c < D / 16; ++c) {
+    float y0[8], y1[8];
+    q_rot8(a, gi, h, 2 * c, y0);
+    q_rot8(a, gi, h, 2 * c + 1, y1);
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float* y = j < 2 ? y0 + 4 * j : y1 + 4 * (j - 2);
+      const uint32_t lo = e4m3x2(mul_rn(y[0], inv), mul_rn(y[1], inv));
+      const uint32_t hi = e4m3x2(mul_rn(y[2], inv), mul_rn(y[3], inv));
+      w[j] = bad ? 0x7F7F7F7Fu : zero ? 0u : (lo | (hi << 16));
+    }
+    *reinterpret_cast<uint4*>(qc + row * 128 + ((c ^ (row & 7)) << 4)) =
+        make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  return scale;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_attn_sm100_kernel(const __grid_constant__ CUtensorMap tmk,
                             const __grid_constant__ CUtensorMap tmv, const AttnArgs a) {
@@ -268,10 +316,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int gi = q0 + 128 * g + row_in_tile;
   float rowmul = 1.f;
   if (warp >= kWarpSoft) {
-    int k = q_exponent(a, gi, h);
-    k = (k == INT_MIN) ? 0 : max(-126, min(127, k));
-    q_split(a, gi, h, k, sm + Layout::qhi, sm + Layout::qlo, 128 * g + row_in_tile);
-    rowmul = ldexpf(1.f, k);
+    if (a.mode_b) {
+      rowmul = q_quant_b(a, gi, h, sm + Layout::qhi, 128 * g + row_in_tile);
+    } else {
+      int k = q_exponent(a, gi, h);
+      k = (k == INT_MIN) ? 0 : max(-126, min(127, k));
+      q_split(a, gi, h, k, sm + Layout::qhi, sm + Layout::qlo, 128 * g + row_in_tile);
+      rowmul = ldexpf(1.f, k);
+    }
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -351,19 +403,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idO = idesc_f16_f32(128, D, 0, 1);
       const uint32_t sQhi = smem_u32(sm + Layout::qhi), sQlo = smem_u32(sm + Layout::qlo);
       const uint32_t sK = smem_u32(sm + Layout::kbuf), sV = smem_u32(sm + Layout::vh);
+      const bool mode_b = a.mode_b != 0;
       // S_g = Q_g K^T into buffer buf of tile g (hi and lo halves of Q accumulate)
       // descriptors are built once; a step of s bytes adds s >> 4 to the start field
       const uint64_t dQhi = smem_desc_sw128(sQhi, 16, 1024), dQlo = smem_desc_sw128(sQlo, 16, 1024);
       const uint64_t dK = smem_desc_sw128(sK, 16, 1024), dV = smem_desc_sw128(sV, kVPanel, 1024);
+      // query halves: hi and lo (exact split), or the one e4m3 operand (mode B)
+      const int n_halves = mode_b ? 1 : 2;
       auto issue_s = [&](int gg, int buf, int sk) {
         const uint32_t d = tmem + 128 * gg + 64 * buf;
-        const uint64_t qh = dQhi + ((gg * 128 * D) >> 4), ql = dQlo + ((gg * 128 * D) >> 4);
         const uint64_t kd = dK + ((sk * BN * D) >> 4);
+        for (int hf = 0; hf < n_halves; ++hf) {
+          const uint64_t qd = (hf == 0 ? dQhi : dQlo) + ((gg * 128 * D) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < D / 32; ++kk)
-          tc_mma_f8_ss(d, qh + 2 * kk, kd + 2 * kk, idS, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < D / 32; ++kk) tc_mma_f8_ss(d, ql + 2 * kk, kd + 2 * kk, idS, 1);
+          for (int kk = 0; kk < D / 32; ++kk)
+            tc_mma_f8_ss(d, qd + 2 * kk, kd + 2 * kk, idS, (hf | kk) != 0);
+        }
       };
       // O_g (+)= P_g V with P_g read from tensor memory (buffer buf)
       auto issue_pv = [&](int gg, int buf, int vbi, uint32_t acc) {

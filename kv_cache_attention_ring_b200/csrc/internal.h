@@ -46,6 +46,7 @@ struct AttnArgs {
   float score_scale_log2;   // softmax_scale * log2(e)
   float bias_log2;          // history_bias * log2(e)
   unsigned int* timeouts;   // device counter of waits that gave up
+  int mode_b;               // query quantised to e4m3 per row (one MMA set for Q.K^T)
   // split over keys (gridDim.z splits): when part_o is set, each split writes its
   // unnormalised O [split][n_q][H][D] and (m, l) [split][H][n_q] (log2 units) there
   float* part_o;

@@ -280,8 +280,9 @@ int attention_args(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0, 
                    float softmax_scale, void* out, float* lse, uint32_t flags, AttnArgs* a) {
   int rc = check_ring(kv);
   if (rc) return rc;
-  if (flags != 0) return KV_EINVAL;
+  if (flags & ~KV_QK_FP8) return KV_EINVAL;
   if (n_q < 0 || n_current < 0) return KV_EINVAL;
+  if ((flags & KV_QK_FP8) && kv->head_dim != 128) return KV_EUNSUPPORTED;
   if (n_q == 0) return KV_OK;
   if (!q || !out || !aligned16(q) || !aligned16(out)) return KV_EINVAL;
   if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return KV_EINVAL;
@@ -320,6 +321,7 @@ int attention_args(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0, 
   a->timeouts = nullptr;
   a->part_o = nullptr;
   a->part_ml = nullptr;
+  a->mode_b = (flags & KV_QK_FP8) ? 1 : 0;
   return KV_OK;
 }
 

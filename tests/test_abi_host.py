@@ -131,7 +131,8 @@ def test_attention_validation_before_launch(L):
     ok_args = (r, 16, 8, 0, 8, None, None, 0.125, 16, None)
     assert L.chunk_attention(*ok_args[:1], 16, 0, 0, 0, None, None, 0.125, 16, None, 0,
                              None) == kv.KV_OK                            # n_q = 0: no launch
-    assert L.chunk_attention(*ok_args, 1, None) == kv.KV_EINVAL           # flags
+    assert L.chunk_attention(*ok_args, 2, None) == kv.KV_EINVAL           # unknown flag
+    assert L.chunk_attention(*ok_args, kv.KV_QK_FP8, None) == kv.KV_EUNSUPPORTED  # mode B, D 64
     assert L.chunk_attention(r, 16, 8, 0, 65, None, None, 0.125, 16, None, 0,
                              None) == kv.KV_ERANGE                        # n_current > valid
     assert L.chunk_attention(r, 16, 8, 4090, 8, None, None, 0.125, 16, None, 0,
