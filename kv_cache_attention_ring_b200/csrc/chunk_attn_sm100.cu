@@ -570,86 +570,129 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(t_s + 32, hi);
       }
       tmem_wait_ld();
-      // pass 1, in place: t = S * kscl (* r + bias later) for fast tiles, masked t for the
-      // others; row maximum of the tile
-      const float4* k4 = reinterpret_cast<const float4*>(in.kscl);
-      float m0 = -INFINITY, m1 = -INFINITY;
-      if (!special) {
-        // key scales in two batches of 8 shared-memory loads, so their latency overlaps
-        float4 kq[8];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          if ((q & 7) == 0) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) kq[i] = k4[q + i];
-          }
-          const float4 ks = kq[q & 7];
-          float u0, u1, u2, u3;
-          f2_unpack(f2_mul(f2_pack(__uint_as_float(sr[4 * q]), __uint_as_float(sr[4 * q + 1])),
-                           f2_pack(ks.x, ks.y)), u0, u1);
-          f2_unpack(f2_mul(f2_pack(__uint_as_float(sr[4 * q + 2]), __uint_as_float(sr[4 * q + 3])),
-                           f2_pack(ks.z, ks.w)), u2, u3);
-          sr[4 * q] = __float_as_uint(u0);
-          sr[4 * q + 1] = __float_as_uint(u1);
-          sr[4 * q + 2] = __float_as_uint(u2);
-          sr[4 * q + 3] = __float_as_uint(u3);
-          m0 = max3f(m0, u0, u1);
-          m1 = max3f(m1, u2, u3);
-        }
-      } else {
-        const float4* b4 = reinterpret_cast<const float4*>(in.kb);
-        const int4* t4 = reinterpret_cast<const int4*>(in.ktok);
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const float4 ks = k4[q], kb = b4[q];
-          const int4 tk = t4[q];
-          float u0, u1, u2, u3;
-          f2_unpack(f2_fma(f2_mul(f2_pack(__uint_as_float(sr[4 * q]), __uint_as_float(sr[4 * q + 1])),
-                                  f2_pack(ks.x, ks.y)), r2, f2_pack(kb.x, kb.y)), u0, u1);
-          f2_unpack(f2_fma(f2_mul(f2_pack(__uint_as_float(sr[4 * q + 2]), __uint_as_float(sr[4 * q + 3])),
-                                  f2_pack(ks.z, ks.w)), r2, f2_pack(kb.z, kb.w)), u2, u3);
-          u0 = tk.x < lim ? u0 : -INFINITY;
-          u1 = tk.y < lim ? u1 : -INFINITY;
-          u2 = tk.z < lim ? u2 : -INFINITY;
-          u3 = tk.w < lim ? u3 : -INFINITY;
-          sr[4 * q] = __float_as_uint(u0);
-          sr[4 * q + 1] = __float_as_uint(u1);
-          sr[4 * q + 2] = __float_as_uint(u2);
-          sr[4 * q + 3] = __float_as_uint(u3);
-          m0 = max3f(m0, u0, u1);
-          m1 = max3f(m1, u2, u3);
-        }
-      }
-      const float mloc = special ? fmaxf(m0, m1) : fmaf(fmaxf(m0, m1), rowmul, a.bias_log2);
-      // lazy reference maximum: move m only when the tile maximum exceeds it by more than
-      // 2^8 (rows of a tile may differ; everything below is per row)
+      const float4* k4s = reinterpret_cast<const float4*>(in.kscl);
       const float m_old = m_run;
-      const bool move = mloc > m_old + kRescaleLog2 || (m_old == -INFINITY && mloc > -INFINITY);
-      if (move) m_run = mloc;
-      const float mref = (m_run == -INFINITY) ? 0.f : m_run;
-      // pass 2: p = 2^(t - m); P = f16(p) over the S columns of tensor memory
-      const float off = special ? -mref : a.bias_log2 - mref;
-      const uint64_t mul2 = special ? f2_pack(1.f, 1.f) : r2;
-      const uint64_t off2 = f2_pack(off, off);
+      bool move = false, single = false;
       uint64_t sum01 = f2_pack(0.f, 0.f), sum23 = sum01;
+      if (!special && __all_sync(0xffffffffu, m_run != -INFINITY)) {
+        // single pass against the current reference maximum: p = 2^(S kscl r + bias - m),
+        // the tile maximum tracked on the way; kept unless a row's tile maximum exceeds m
+        // by more than 2^8 (then the two passes below recompute the tile from S)
+        const float off = a.bias_log2 - m_run;
+        const uint64_t off2 = f2_pack(off, off);
+        float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t pk[16];
+        for (int c = 0; c < 2; ++c) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int q8 = 0; q8 < 8; ++q8) {
-          const int q = 8 * c + q8;
-          float t0, t1, t2, t3;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[4 * q]), __uint_as_float(sr[4 * q + 1])), mul2,
-                           off2), t0, t1);
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[4 * q + 2]), __uint_as_float(sr[4 * q + 3])), mul2,
-                           off2), t2, t3);
-          const float p0 = ex2(t0), p1 = ex2(t1), p2 = ex2(t2), p3 = ex2(t3);   // 2^-inf = 0
-          sum01 = f2_add(sum01, f2_pack(p0, p1));
-          sum23 = f2_add(sum23, f2_pack(p2, p3));
-          pk[2 * q8] = pack_f16x2(p0, p1);
-          pk[2 * q8 + 1] = pack_f16x2(p2, p3);
+          for (int q8 = 0; q8 < 8; ++q8) {
+            const int q = 8 * c + q8;
+            const float4 ks = k4s[q];
+            const uint64_t u01 = f2_mul(f2_pack(__uint_as_float(sr[4 * q]), __uint_as_float(sr[4 * q + 1])),
+                                        f2_pack(ks.x, ks.y));
+            const uint64_t u23 = f2_mul(f2_pack(__uint_as_float(sr[4 * q + 2]), __uint_as_float(sr[4 * q + 3])),
+                                        f2_pack(ks.z, ks.w));
+            float u0, u1, u2, u3, t0, t1, t2, t3;
+            f2_unpack(u01, u0, u1);
+            f2_unpack(u23, u2, u3);
+            m0 = max3f(m0, u0, u1);
+            m1 = max3f(m1, u2, u3);
+            f2_unpack(f2_fma(u01, r2, off2), t0, t1);
+            f2_unpack(f2_fma(u23, r2, off2), t2, t3);
+            const float p0 = ex2(t0), p1 = ex2(t1), p2 = ex2(t2), p3 = ex2(t3);
+            sum01 = f2_add(sum01, f2_pack(p0, p1));
+            sum23 = f2_add(sum23, f2_pack(p2, p3));
+            pk[2 * q8] = pack_f16x2(p0, p1);
+            pk[2 * q8 + 1] = pack_f16x2(p2, p3);
+          }
+          // P over S columns already read into registers; a recomputation overwrites it
+          tmem_st16(t_s + 16 * c, pk);
         }
-        tmem_st16(t_s + 16 * c, pk);
+        const float mloc = fmaf(fmaxf(m0, m1), rowmul, a.bias_log2);
+        single = !__any_sync(0xffffffffu, mloc > m_run + kRescaleLog2);
+      }
+      if (!single) {
+        // pass 1, in place: t = S * kscl (* r + bias later) for fast tiles, masked t for the
+        // others; row maximum of the tile
+        const float4* k4 = reinterpret_cast<const float4*>(in.kscl);
+        float m0 = -INFINITY, m1 = -INFINITY;
+        if (!special) {
+          // key scales in two batches of 8 shared-memory loads, so their latency overlaps
+          float4 kq[8];
+  #pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            if ((q & 7) == 0) {
+  #pragma unroll
+              for (int i = 0; i < 8; ++i) kq[i] = k4[q + i];
+            }
+            const float4 ks = kq[q & 7];
+            float u0, u1, u2, u3;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(sr[4 * q]), __uint_as_float(sr[4 * q + 1])),
+                             f2_pack(ks.x, ks.y)), u0, u1);
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(sr[4 * q + 2]), __uint_as_float(sr[4 * q + 3])),
+                             f2_pack(ks.z, ks.w)), u2, u3);
+            sr[4 * q] = __float_as_uint(u0);
+            sr[4 * q + 1] = __float_as_uint(u1);
+            sr[4 * q + 2] = __float_as_uint(u2);
+            sr[4 * q + 3] = __float_as_uint(u3);
+            m0 = max3f(m0, u0, u1);
+            m1 = max3f(m1, u2, u3);
+          }
+        } else {
+          const float4* b4 = reinterpret_cast<const float4*>(in.kb);
+          const int4* t4 = reinterpret_cast<const int4*>(in.ktok);
+  #pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const float4 ks = k4[q], kb = b4[q];
+            const int4 tk = t4[q];
+            float u0, u1, u2, u3;
+            f2_unpack(f2_fma(f2_mul(f2_pack(__uint_as_float(sr[4 * q]), __uint_as_float(sr[4 * q + 1])),
+                                    f2_pack(ks.x, ks.y)), r2, f2_pack(kb.x, kb.y)), u0, u1);
+            f2_unpack(f2_fma(f2_mul(f2_pack(__uint_as_float(sr[4 * q + 2]), __uint_as_float(sr[4 * q + 3])),
+                                    f2_pack(ks.z, ks.w)), r2, f2_pack(kb.z, kb.w)), u2, u3);
+            u0 = tk.x < lim ? u0 : -INFINITY;
+            u1 = tk.y < lim ? u1 : -INFINITY;
+            u2 = tk.z < lim ? u2 : -INFINITY;
+            u3 = tk.w < lim ? u3 : -INFINITY;
+            sr[4 * q] = __float_as_uint(u0);
+            sr[4 * q + 1] = __float_as_uint(u1);
+            sr[4 * q + 2] = __float_as_uint(u2);
+            sr[4 * q + 3] = __float_as_uint(u3);
+            m0 = max3f(m0, u0, u1);
+            m1 = max3f(m1, u2, u3);
+          }
+        }
+        const float mloc = special ? fmaxf(m0, m1) : fmaf(fmaxf(m0, m1), rowmul, a.bias_log2);
+        // lazy reference maximum: move m only when the tile maximum exceeds it by more than
+        // 2^8 (rows of a tile may differ; everything below is per row)
+        move = mloc > m_old + kRescaleLog2 || (m_old == -INFINITY && mloc > -INFINITY);
+        if (move) m_run = mloc;
+        const float mref = (m_run == -INFINITY) ? 0.f : m_run;
+        // pass 2: p = 2^(t - m); P = f16(p) over the S columns of tensor memory
+        const float off = special ? -mref : a.bias_log2 - mref;
+        const uint64_t mul2 = special ? f2_pack(1.f, 1.f) : r2;
+        const uint64_t off2 = f2_pack(off, off);
+        sum01 = f2_pack(0.f, 0.f);
+        sum23 = sum01;
+  #pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t pk[16];
+  #pragma unroll
+          for (int q8 = 0; q8 < 8; ++q8) {
+            const int q = 8 * c + q8;
+            float t0, t1, t2, t3;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[4 * q]), __uint_as_float(sr[4 * q + 1])), mul2,
+                             off2), t0, t1);
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[4 * q + 2]), __uint_as_float(sr[4 * q + 3])), mul2,
+                             off2), t2, t3);
+            const float p0 = ex2(t0), p1 = ex2(t1), p2 = ex2(t2), p3 = ex2(t3);   // 2^-inf = 0
+            sum01 = f2_add(sum01, f2_pack(p0, p1));
+            sum23 = f2_add(sum23, f2_pack(p2, p3));
+            pk[2 * q8] = pack_f16x2(p0, p1);
+            pk[2 * q8 + 1] = pack_f16x2(p2, p3);
+          }
+          tmem_st16(t_s + 16 * c, pk);
+        }
       }
       float s0, s1, s2, s3;
       f2_unpack(sum01, s0, s1);
