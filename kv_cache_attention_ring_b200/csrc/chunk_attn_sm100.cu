@@ -21,17 +21,24 @@
 //    f16(e4m3(vc) * vs / G) in shared memory (|V'| <= 448, one f16 rounding, 2^-11
 //    relative); P = f16(p) (p <= 1) is written to tensor memory over the S columns it
 //    came from and read from there as the A operand; the epilogue multiplies O by G.
+//  * Mode B (KV_QK_FP8): the rotated bf16 row is instead quantised to e4m3 by the write's
+//    row rule, and the row scale takes the place of r; S' is one set of D/32 MMAs.
 //  * Tensor memory (512 columns): tile g owns two S/P buffers of 64 columns,
-//    [128g, 128g+64) and [128g+64, 128g+128), and O_g = [256+128g, 384+128g).  The MMA
-//    issuer runs one key tile ahead: S_g(j+1) is computed into the other buffer while
-//    the softmax of tile g works on S_g(j); issue order S0(j+1) S1(j+1) PV0(j) PV1(j).
+//    [128g, 128g+64) and [128g+64, 128g+128), and O_g = [256+128g, 384+128g).  Per key
+//    tile j and query tile g the MMA issuer runs P.V_g(j) as soon as P_g(j) is in tensor
+//    memory, then S_g(j+2) into the buffer P_g(j) occupied (tensor-core operations of one
+//    thread run in issue order), so the softmax finds S_g(j+1) ready after S_g(j).
 //  * Warps: 0 TMA producer, 1 MMA issuer, 2-3 V converters + per-key info, 4-7 softmax
 //    of tile 0, 8-11 softmax of tile 1 (thread = query row = TMEM lane).
-//  * Softmax in log2 units with paired fp32 instructions (f32x2): the 64-column S row
-//    sits in registers; pass 1 scales it in place and finds the maximum, pass 2 takes
-//    2^(t - m).  The reference maximum m moves lazily (only when the tile maximum
-//    exceeds it by more than 8, a factor 256); O is then rescaled in tensor memory after
-//    the previous P.V has completed.  out = O / l is exact regardless of m.
+//  * Softmax in log2 units with paired fp32 instructions (f32x2) on the 64-column S row
+//    held in registers.  The reference maximum m moves lazily (only when the tile
+//    maximum exceeds it by more than 8, a factor 256); O is then rescaled in tensor
+//    memory after the previous P.V has completed.  out = O / l is exact regardless of m.
+//    A history-only tile with m already set takes one pass (scale, 2^(t - m), P, tile
+//    maximum on the way); the first tile, tiles with current or invalid keys, and tiles
+//    whose maximum exceeds m by more than 8 take two (maximum first, then 2^(t - m)).
+//  * Split over keys (gridDim.z > 1): each CTA takes a contiguous share of the valid
+//    tiles and writes fp32 partials (O G, m, l); split_combine_kernel merges them.
 //  * Keys are visited in physical slot order; the ring wrap costs nothing (attention
 //    does not depend on key order once bias and mask are per key).
 // Every mbarrier wait is bounded (about a second); on a timeout the CTA abandons the
