@@ -181,3 +181,31 @@ class BruteRing:
             out[live, h] = (P @ V[h]) / l
             lse[h, live] = (m[live] + np.log(l))[:, 0]
         return out, lse
+
+
+class BruteAnchoredRing(BruteRing):
+    """A persistent anchor beside the sliding window ("Why Live Video Generation Still
+    Struggles With Timing", Transcript: recent history plus the first chunk kept as an
+    anchor).  The first ``A`` committed tokens stay for good; the window holds the last
+    ``C`` tokens after them, the pending chunk included.  Keys are ordered anchor first,
+    so the current chunk is still the newest ``n_current`` of them; a reset re-rotates
+    every cached key, the anchor's too."""
+
+    def __init__(self, A: int, C: int, H: int, D: int, base: float = 10000.0,
+                 next_pos: int = 0):
+        super().__init__(C, H, D, base, next_pos)
+        self.A = A
+
+    def window(self) -> list[dict]:
+        return self.tokens[: self.A] + (self.tokens[self.A:] + self.pending)[-self.C:]
+
+    def fifo_arrays(self):
+        """The FIFO part scattered into ring arrays (slot = (global index - A) mod C)."""
+        C, H, D = self.C, self.H, self.D
+        kc = np.zeros((H, C, D), np.uint8)
+        ks = np.zeros((H, C), F32)
+        sp = np.zeros(C, np.int32)
+        for tok in self.window()[min(self.A, len(self.tokens)):]:
+            s = (tok["g"] - self.A) % C
+            kc[:, s], ks[:, s], sp[s] = tok["kc"], tok["ks"], tok["pos"]
+        return kc, ks, sp

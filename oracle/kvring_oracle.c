@@ -14,7 +14,7 @@
  *    attention bias during transitions (read here as an additive logit on history slots).
  *  - "Why Live Video Generation Still Struggles With Timing": attention is bidirectional
  *    inside the current chunk and backward-only across chunks; a sliding window of
- *    recent history.
+ *    recent history, with the first chunk kept beside it as a persistent anchor.
  *  - "Stream LTX", section "Training": block structure (1 s blocks of video + audio
  *    latents) and a causal mask on every attention path.
  *
@@ -262,16 +262,25 @@ static int64_t block_id(int64_t t, int64_t first, int64_t len) {
 }
 
 /* Attention of query rows rows[0..n_rows) (all n_q rows if rows is NULL) over the valid
- * slots.  q is [n_q][H][D] binary32 (the exact values of the caller's inputs).
- * out: [n_rows][H][D] binary64; lse: [H][n_rows] binary64 (natural log), may be NULL.
- * flags bit 0 (mode B): the rotated bf16 query is also quantised to e4m3 per row by
- * the write rule and dequantised before the dot products. */
-ORC_API void orc_chunk_attention(const orc_ring* r, const float* q, int n_q, int64_t q_pos0,
-                                 int n_current, int q_first, int q_block, int k_first,
-                                 int k_block, float cache_bias, float softmax_scale, int flags,
-                                 const int32_t* rows, int n_rows, double* out, double* lse) {
-  const int C = r->C, H = r->H, D = r->D;
-  const int64_t nv = valid_slots(r);
+ * slots of rings[0..n_rings).  rings[0] is the stream's main ring: its newest n_current
+ * slots are the current chunk (block mask, no bias) and the rest is history.  Every valid
+ * slot of rings[1..] is history too: always visible, cache_bias added.  That is how a
+ * persistent anchor ("Why Live Video Generation Still Struggles With Timing", Transcript:
+ * the first chunk kept beside a sliding window of recent history) joins the attention.
+ * All rings share H, D and the RoPE base.  q is [n_q][H][D] binary32 (the exact values of
+ * the caller's inputs).  out: [n_rows][H][D] binary64; lse: [H][n_rows] binary64 (natural
+ * log), may be NULL.  flags bit 0 (mode B): the rotated bf16 query is also quantised to
+ * e4m3 per row by the write rule and dequantised before the dot products. */
+ORC_API void orc_chunk_attention_multi(const orc_ring* const* rings, int n_rings,
+                                       const float* q, int n_q, int64_t q_pos0, int n_current,
+                                       int q_first, int q_block, int k_first, int k_block,
+                                       float cache_bias, float softmax_scale, int flags,
+                                       const int32_t* rows, int n_rows, double* out,
+                                       double* lse) {
+  const orc_ring* r0 = rings[0];
+  const int H = r0->H, D = r0->D;
+  int64_t nv = 0;
+  for (int g = 0; g < n_rings; ++g) nv += valid_slots(rings[g]);
   if (!rows) n_rows = n_q;
 #pragma omp parallel for collapse(2) schedule(dynamic, 1)
   for (int ri = 0; ri < n_rows; ++ri) {
@@ -279,7 +288,7 @@ ORC_API void orc_chunk_attention(const orc_ring* r, const float* q, int n_q, int
       const int i = rows ? rows[ri] : ri;
       float c[256], s[256], y[512];
       double qt[512];
-      orc_rope_cs(q_pos0 + i, D, r->base, c, s);
+      orc_rope_cs(q_pos0 + i, D, r0->base, c, s);
       orc_rope_apply(q + ((size_t)i * H + h) * D, D, c, s, y);
       for (int d = 0; d < D; ++d) y[d] = orc_bf16_round(y[d]);
       if (flags & 1) {
@@ -293,33 +302,41 @@ ORC_API void orc_chunk_attention(const orc_ring* r, const float* q, int n_q, int
       const int64_t qb = block_id(i, q_first, q_block);
       double* sc = (double*)malloc(sizeof(double) * (size_t)(nv > 0 ? nv : 1));
       int64_t* sl = (int64_t*)malloc(sizeof(int64_t) * (size_t)(nv > 0 ? nv : 1));
+      int* sg = (int*)malloc(sizeof(int) * (size_t)(nv > 0 ? nv : 1));
       int64_t nvis = 0;
       double m = -INFINITY;
-      for (int64_t age = 0; age < nv; ++age) {
-        int history = age >= n_current;
-        if (!history) {
-          int64_t t = n_current - 1 - age;            /* token index inside the chunk */
-          if (block_id(t, k_first, k_block) > qb) continue;
+      for (int g = 0; g < n_rings; ++g) {
+        const orc_ring* r = rings[g];
+        const int C = r->C;
+        const int64_t nv_g = valid_slots(r);
+        for (int64_t age = 0; age < nv_g; ++age) {
+          int history = g > 0 || age >= n_current;
+          if (!history) {
+            int64_t t = n_current - 1 - age;          /* token index inside the chunk */
+            if (block_id(t, k_first, k_block) > qb) continue;
+          }
+          int64_t slot = orc_slot_of_age(r, age);
+          const uint8_t* kr = r->kc + ((size_t)h * C + slot) * D;
+          double ksc = (double)r->ks[(size_t)h * C + slot], dot = 0.0;
+          for (int d = 0; d < D; ++d) dot += qt[d] * (orc_e4m3_decode(kr[d]) * ksc);
+          double sv = (double)softmax_scale * dot + (history ? (double)cache_bias : 0.0);
+          sc[nvis] = sv;
+          sl[nvis] = slot;
+          sg[nvis] = g;
+          ++nvis;
+          if (sv > m) m = sv;
         }
-        int64_t slot = orc_slot_of_age(r, age);
-        const uint8_t* kr = r->kc + ((size_t)h * C + slot) * D;
-        double ksc = (double)r->ks[(size_t)h * C + slot], dot = 0.0;
-        for (int d = 0; d < D; ++d) dot += qt[d] * (orc_e4m3_decode(kr[d]) * ksc);
-        double sv = (double)softmax_scale * dot + (history ? (double)cache_bias : 0.0);
-        sc[nvis] = sv;
-        sl[nvis] = slot;
-        ++nvis;
-        if (sv > m) m = sv;
       }
       if (m == -INFINITY) nvis = 0;  /* every visible score is -inf: nothing attended */
       double* o = out + ((size_t)ri * H + h) * D;
       for (int d = 0; d < D; ++d) o[d] = 0.0;
       double l = 0.0;
       for (int64_t j = 0; j < nvis; ++j) {
+        const orc_ring* r = rings[sg[j]];
         double p = exp(sc[j] - m);
         l += p;
-        const uint8_t* vr = r->vc + ((size_t)h * C + sl[j]) * D;
-        double vsc = (double)r->vs[(size_t)h * C + sl[j]];
+        const uint8_t* vr = r->vc + ((size_t)h * r->C + sl[j]) * D;
+        double vsc = (double)r->vs[(size_t)h * r->C + sl[j]];
         for (int d = 0; d < D; ++d) o[d] += p * (orc_e4m3_decode(vr[d]) * vsc);
       }
       if (nvis > 0) {
@@ -328,8 +345,19 @@ ORC_API void orc_chunk_attention(const orc_ring* r, const float* q, int n_q, int
       if (lse) lse[(size_t)h * n_rows + ri] = nvis > 0 ? m + log(l) : -INFINITY;
       free(sc);
       free(sl);
+      free(sg);
     }
   }
+}
+
+/* The one-ring case: the stream's ring alone. */
+ORC_API void orc_chunk_attention(const orc_ring* r, const float* q, int n_q, int64_t q_pos0,
+                                 int n_current, int q_first, int q_block, int k_first,
+                                 int k_block, float cache_bias, float softmax_scale, int flags,
+                                 const int32_t* rows, int n_rows, double* out, double* lse) {
+  const orc_ring* rings[1] = {r};
+  orc_chunk_attention_multi(rings, 1, q, n_q, q_pos0, n_current, q_first, q_block, k_first,
+                            k_block, cache_bias, softmax_scale, flags, rows, n_rows, out, lse);
 }
 
 /* ---------------------------------------------------------------- array helpers for tests */

@@ -63,6 +63,10 @@ def lib() -> ctypes.CDLL:
             P, P, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_float, ctypes.c_int, P,
             ctypes.c_int, P, P]
+        L.orc_chunk_attention_multi.argtypes = [
+            P, ctypes.c_int, P, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_float,
+            ctypes.c_int, P, ctypes.c_int, P, P]
         L.orc_e4m3_encode_n.argtypes = [P, ctypes.c_int64, P]
         L.orc_e4m3_decode_n.argtypes = [P, ctypes.c_int64, P]
         L.orc_bf16_round_n.argtypes = [P, ctypes.c_int64, P]
@@ -205,21 +209,51 @@ class OracleRing:
         """Returns (out [rows][H][D] f64, lse [H][rows] f64).
 
         mask = (q_first_len, q_block_len, k_first_len, k_block_len)."""
-        q = _f32(q)
-        n_q = q.shape[0]
-        assert q.shape == (n_q, self.H, self.D)
-        if softmax_scale is None:
-            softmax_scale = float(np.float32(1.0 / np.sqrt(self.D)))
-        if rows is None:
-            rows_arr, n_rows, rp = None, n_q, None
-        else:
-            rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
-            assert rows_arr.min() >= 0 and rows_arr.max() < n_q
-            n_rows, rp = rows_arr.size, _p(rows_arr)
-        out = np.zeros((n_rows, self.H, self.D), np.float64)
-        lse = np.zeros((self.H, n_rows), np.float64)
+        q, n_q, softmax_scale, rows_arr, n_rows, rp, out, lse = _attn_io(
+            self, q, softmax_scale, rows)
         qf, qb, kf, kb = (int(x) for x in mask)
         lib().orc_chunk_attention(self._ptr(), _p(q), n_q, int(q_pos0), int(n_current), qf, qb,
                                   kf, kb, float(cache_bias), float(softmax_scale),
                                   int(bool(mode_b)), rp, n_rows, _p(out), _p(lse))
         return out, lse
+
+
+def _attn_io(ring: "OracleRing", q, softmax_scale, rows):
+    """Shared marshalling of the attention calls: query array, scale, row list, outputs."""
+    q = _f32(q)
+    n_q = q.shape[0]
+    assert q.shape == (n_q, ring.H, ring.D)
+    if softmax_scale is None:
+        softmax_scale = float(np.float32(1.0 / np.sqrt(ring.D)))
+    if rows is None:
+        rows_arr, n_rows, rp = None, n_q, None
+    else:
+        rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+        assert rows_arr.min() >= 0 and rows_arr.max() < n_q
+        n_rows, rp = rows_arr.size, _p(rows_arr)
+    out = np.zeros((n_rows, ring.H, ring.D), np.float64)
+    lse = np.zeros((ring.H, n_rows), np.float64)
+    return q, n_q, softmax_scale, rows_arr, n_rows, rp, out, lse
+
+
+def attention_multi(main: OracleRing, history_rings, q, q_pos0: int, n_current: int,
+                    mask=(1 << 30, 1 << 30, 1 << 30, 1 << 30), cache_bias: float = 0.0,
+                    softmax_scale: float | None = None, rows=None, mode_b: bool = False):
+    """Attention over the valid slots of ``main`` and of every ring in ``history_rings``.
+
+    ``main`` holds the current chunk (its newest ``n_current`` slots); every slot of the
+    other rings is history (always visible, ``cache_bias`` added), e.g. a persistent
+    anchor chunk kept beside the sliding window.  Same return values as
+    ``OracleRing.attention``."""
+    rings = [main, *history_rings]
+    for r in rings:
+        assert (r.H, r.D, r._s.base) == (main.H, main.D, main._s.base)
+    q, n_q, softmax_scale, rows_arr, n_rows, rp, out, lse = _attn_io(
+        main, q, softmax_scale, rows)
+    ptrs = (ctypes.c_void_p * len(rings))(*[ctypes.addressof(r._s) for r in rings])
+    qf, qb, kf, kb = (int(x) for x in mask)
+    lib().orc_chunk_attention_multi(ctypes.cast(ptrs, ctypes.c_void_p), len(rings), _p(q), n_q,
+                                    int(q_pos0), int(n_current), qf, qb, kf, kb,
+                                    float(cache_bias), float(softmax_scale), int(bool(mode_b)),
+                                    rp, n_rows, _p(out), _p(lse))
+    return out, lse

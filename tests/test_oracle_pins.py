@@ -308,3 +308,79 @@ def test_minus_inf_bias_without_current_keys_attends_nothing(orc):
     b = brute.BruteRing(o.C, o.H, o.D)
     bo, bl = b.attention(q, 0, 0, (1, 1, 1, 1), -np.inf, 0.125)
     assert (bo == 0).all() and np.isneginf(bl).all()
+
+
+# ---------------------------------------------------------------- persistent anchor
+
+def _lse_merge(parts):
+    """Merge (out [n][H][D], lse [H][n]) results over disjoint key sets: the softmax over
+    the union, written in closed form from the parts."""
+    lses = np.stack([l for _, l in parts])                        # [P][H][n]
+    top = lses.max(0)
+    safe = np.where(np.isfinite(top), top, 0.0)
+    w = np.exp(lses - safe)                                       # [P][H][n]
+    tot = w.sum(0)
+    out = sum(wp.T[:, :, None] * o for wp, (o, _) in zip(w, parts))
+    with np.errstate(invalid="ignore", divide="ignore"):
+        out = np.where(tot.T[:, :, None] > 0, out / tot.T[:, :, None], 0.0)
+        lse = np.where(tot > 0, safe + np.log(tot), -np.inf)
+    return out, lse
+
+
+def test_anchor_beside_window_matches_brute_tiny(orc):
+    """First chunk kept as a persistent anchor ring, later chunks in a 128-slot window ring
+    that wraps twice; a reset re-rotates both.  The oracle's multi-ring attention equals the
+    brute model's dense attention over anchor + window, the rings equal the brute arrays bit
+    for bit, and the anchor is never evicted."""
+    A, W, H, D, n = 32, 128, 2, 64, 32
+    rng = np.random.default_rng(17)
+    anchor = orc.OracleRing(A, H, D)
+    win = orc.OracleRing(W, H, D, next_pos=A)
+    b = brute.BruteAnchoredRing(A, W, H, D)
+    sm = float(np.float32(1 / np.sqrt(D)))
+    worst, worst_merge = 0.0, 0.0
+    for ch in range(10):
+        main, hist = (anchor, [win]) if ch == 0 else (win, [anchor])
+        q = rng.standard_normal((n, H, D)).astype(np.float32)
+        for p in range(2):
+            k = rng.standard_normal((n, H, D)).astype(np.float32)
+            v = rng.standard_normal((n, H, D)).astype(np.float32)
+            main.write(k, v)
+            b.write(k, v)
+            for bias in (0.0, -2.0):
+                for mask in ((32, 32, 32, 32), (8, 8, 8, 8)):
+                    oo, ol = orc.attention_multi(main, hist, q, main.next_pos, n, mask, bias)
+                    bo, bl = b.attention(q, b.next_pos, n, mask, bias, sm)
+                    worst = max(worst, np.abs(oo - bo).max(), np.abs(ol - bl).max())
+                    # the union of disjoint key sets: the closed-form merge of the parts
+                    parts = [orc.attention_multi(main, [], q, main.next_pos, n, mask, bias)]
+                    parts += [orc.attention_multi(r, [], q, main.next_pos, 0, mask, bias)
+                              for r in hist]
+                    mo, ml = _lse_merge(parts)
+                    worst_merge = max(worst_merge, np.abs(mo - oo).max(),
+                                      np.abs(ml - ol).max())
+        main.commit()
+        b.commit()
+        if ch == 6:
+            for r in (anchor, win):
+                r.delta_rotate(-96)
+            b.delta_rotate(-96)
+        # the anchor holds the first chunk for good; the window the last W tokens after it
+        kc, ks, sp = b.fifo_arrays()
+        assert (win.kc == kc).all() and (win.ks.view(np.uint32) == ks.view(np.uint32)).all()
+        assert (win.slot_pos == sp).all()
+        assert b.next_pos == win.next_pos
+        for s, tok in enumerate(b.window()[:A]):
+            assert (anchor.kc[:, s] == tok["kc"]).all() and anchor.slot_pos[s] == tok["pos"]
+            assert (anchor.ks[:, s].view(np.uint32) == tok["ks"].view(np.uint32)).all()
+    assert (anchor.slot_pos == np.arange(A) - 96).all()      # first chunk, shifted once
+    assert worst < 1e-12 and worst_merge < 1e-12
+
+
+def test_empty_anchor_is_the_plain_ring(orc):
+    o, q, _ = _ring_with_history(orc)
+    empty = orc.OracleRing(16, o.H, o.D)
+    n = q.shape[0]
+    a = o.attention(q, o.next_pos, n, (4, 4, 4, 4), -0.5)
+    m = orc.attention_multi(o, [empty], q, o.next_pos, n, (4, 4, 4, 4), -0.5)
+    assert np.array_equal(a[0], m[0]) and np.array_equal(a[1], m[1])
