@@ -1,9 +1,12 @@
 """The benchmark's arithmetic, checked on the CPU: unmasked-pair counts against a brute
-count of the mask, FLOP and byte figures against their closed forms, and the traffic
-record's source-hash rule."""
+count of the mask, FLOP and byte figures against their closed forms, the traffic
+record's source-hash rule, and the reference arm's output line."""
 import hashlib
 import importlib.util
+import json
 import os
+import subprocess
+import sys
 
 import numpy as np
 
@@ -53,3 +56,32 @@ def test_committed_traffic_record_matches_the_attention_source():
     src = os.path.join(ROOT, "kv_cache_attention_ring_b200", "csrc", "chunk_attn_sm100.cu")
     t = b.traffic_for(src)
     assert t is not None and 60e6 < t < 100e6              # about the 76.6 MB algorithmic
+
+
+def _run_bench(env_extra, *args):
+    env = dict(os.environ, OMP_NUM_THREADS="4", **env_extra)
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args],
+                          capture_output=True, text=True, env=env, timeout=600)
+
+
+def test_reference_arm_prints_one_contract_line():
+    """The reference arm (the oracle on the host cores) prints exactly one JSON line with
+    the contract's keys, on rank 0; other ranks exit 0 without output or work."""
+    r = _run_bench({}, "--impl", "reference", "--steps", "1", "--warmup", "0")
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["unit"] == "us/call" and d["higher_is_better"] is False
+    assert d["value"] > 0 and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    assert d["config"]["workload"].startswith("runway_chunk_step")
+    r1 = _run_bench({"RANK": "1", "WORLD_SIZE": "2"}, "--impl", "reference", "--steps", "1",
+                    "--warmup", "0")
+    assert r1.returncode == 0 and r1.stdout.strip() == ""
