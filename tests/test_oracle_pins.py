@@ -384,3 +384,14 @@ def test_empty_anchor_is_the_plain_ring(orc):
     a = o.attention(q, o.next_pos, n, (4, 4, 4, 4), -0.5)
     m = orc.attention_multi(o, [empty], q, o.next_pos, n, (4, 4, 4, 4), -0.5)
     assert np.array_equal(a[0], m[0]) and np.array_equal(a[1], m[1])
+
+
+def test_gathered_rows_equal_the_full_rows(orc):
+    """The sampled-row form the full-size parity tests use: attention of a gathered subset
+    of query rows equals those rows of the full result exactly (rows are independent)."""
+    o, q, _ = _ring_with_history(orc, n=16)
+    n = q.shape[0]
+    full, lse = o.attention(q, o.next_pos, n, (3, 5, 3, 5), -1.5)
+    rows = [15, 0, 7, 7, 3]
+    part, lp = o.attention(q, o.next_pos, n, (3, 5, 3, 5), -1.5, rows=rows)
+    assert np.array_equal(part, full[rows]) and np.array_equal(lp, lse[:, rows])
