@@ -210,6 +210,36 @@ KV_API int chunk_attention_split(const kv_ring_t* kv, const void* q, int n_q, in
                                  float* lse, int n_splits, void* workspace,
                                  size_t workspace_bytes, uint32_t flags, void* stream);
 
+/* Most rings one chunk_attention_multi call reads. */
+#define KV_MAX_RINGS 8
+
+/* Chunk attention over the stream's ring plus history-only rings, such as the first chunk
+ * kept as a persistent anchor beside the sliding window ("Why Live Video Generation Still
+ * Struggles With Timing", Transcript).  rings[0] is the stream's ring: its newest n_current
+ * valid slots are the current chunk, exactly as in chunk_attention.  Every valid slot of
+ * rings[1 .. n_rings) is history: always visible, cache_bias added.  The result is softmax
+ * attention over the union of all rings' valid slots, with chunk_attention's contract for
+ * out, lse, mask, softmax_scale and flags.
+ * Each ring's keys are split over n_splits groups as in chunk_attention_split.  All
+ * partials go to one workspace of at least chunk_attention_workspace_size(n_q, H, 128,
+ * n_rings * n_splits) bytes (device, 16-byte aligned, caller-owned, uninitialised is
+ * fine), and one merge writes out and lse.
+ * rings: host array of n_rings (1..KV_MAX_RINGS) initialised rings with equal n_heads,
+ * head_dim (128) and rope_base.  Each ring's RoPE table must cover q_pos0 .. q_pos0 + n_q - 1;
+ * the queries are rotated once per ring from that ring's table, so the tables must hold the
+ * same angles (kv_rope_table_build with that base).  n_rings * n_splits <= 64.
+ * Errors, all before anything is enqueued: KV_EINVAL (rings null or n_rings out of range,
+ * a null entry, n_splits out of range, rings that differ in heads, head_dim or base, the
+ * errors of chunk_attention_split), KV_EUNSUPPORTED (head_dim 64), KV_ERANGE (workspace too
+ * small, n_current above rings[0]'s valid slots, a query position outside a table),
+ * KV_ESTATE (a ring not initialised), KV_ECUDA. */
+KV_API int chunk_attention_multi(const kv_ring_t* const* rings, int n_rings, const void* q,
+                                 int n_q, int64_t q_pos0, int n_current,
+                                 const kv_block_mask_t* mask, const kv_cache_bias_t* bias,
+                                 float softmax_scale, void* out, float* lse, int n_splits,
+                                 void* workspace, size_t workspace_bytes, uint32_t flags,
+                                 void* stream);
+
 /* Size of the library's own scratch for chunk_attention_split_noalloc: 16 MiB per
  * device.  8 splits of 25 queries x 32 heads x 128 take 3.3 MB; 4 splits of 1,024
  * queries x 8 heads x 128 (17.0 MB) do not fit. */

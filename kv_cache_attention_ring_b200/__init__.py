@@ -29,9 +29,10 @@ KV_QK_FP8 = 1
 
 EXPORTS = ("kv_rope_table_build", "kv_ring_init", "kv_ring_write", "kv_ring_commit",
            "kv_ring_delta_rotate", "chunk_attention", "chunk_attention_workspace_size",
-           "chunk_attention_split", "chunk_attention_split_noalloc", "kv_status_string",
-           "kv_wait_timeout_count")
+           "chunk_attention_split", "chunk_attention_split_noalloc", "chunk_attention_multi",
+           "kv_status_string", "kv_wait_timeout_count")
 KV_NOALLOC_SCRATCH_BYTES = 16 << 20
+KV_MAX_RINGS = 8
 
 
 class KvError(RuntimeError):
@@ -89,6 +90,8 @@ def lib() -> ctypes.CDLL:
                                             ctypes.c_size_t, ctypes.c_uint32, P]
         L.chunk_attention_split_noalloc.argtypes = [P, P, I, I64, I, P, P, ctypes.c_float, P,
                                                     P, I, ctypes.c_uint32, P]
+        L.chunk_attention_multi.argtypes = [P, I, P, I, I64, I, P, P, ctypes.c_float, P, P, I,
+                                            P, ctypes.c_size_t, ctypes.c_uint32, P]
         _lib = L
     return _lib
 
@@ -242,6 +245,40 @@ def chunk_attention_split(ring: KvRing, q, q_pos0: int, n_current: int, n_splits
                                        _ptr(workspace), nbytes, KV_QK_FP8 if mode_b else 0,
                                        _stream(stream)),
            "chunk_attention_split")
+    return out, lse
+
+
+def chunk_attention_multi(rings, q, q_pos0: int, n_current: int, n_splits: int, workspace,
+                          mask=None, cache_bias: float = 0.0, softmax_scale: float | None = None,
+                          out=None, lse=None, want_lse: bool = True, stream=None,
+                          mode_b: bool = False):
+    """chunk_attention over rings[0], the stream's ring that holds the current chunk, and
+    the history-only rings[1:] (a persistent anchor, for instance).  `workspace` is a
+    device tensor of at least chunk_attention_workspace_size(n_q, H, D, len(rings) *
+    n_splits) bytes."""
+    import torch
+    rings = list(rings)
+    r0 = rings[0]
+    assert q.is_cuda and q.dtype == torch.bfloat16 and q.is_contiguous()
+    n_q = int(q.shape[0])
+    assert q.shape == (n_q, r0.H, r0.D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((r0.H, n_q), dtype=torch.float32, device=q.device)
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(r0.D)
+    m = None if mask is None else kv_block_mask_t(*(int(x) for x in mask))
+    b = kv_cache_bias_t(float(cache_bias))
+    arr = (ctypes.c_void_p * len(rings))(*[ctypes.addressof(r.s) for r in rings])
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().chunk_attention_multi(arr, len(rings), _ptr(q), n_q, int(q_pos0),
+                                       int(n_current), None if m is None else ctypes.byref(m),
+                                       ctypes.byref(b), float(softmax_scale), _ptr(out),
+                                       None if lse is None else _ptr(lse), int(n_splits),
+                                       _ptr(workspace), nbytes, KV_QK_FP8 if mode_b else 0,
+                                       _stream(stream)),
+           "chunk_attention_multi")
     return out, lse
 
 

@@ -402,6 +402,50 @@ int chunk_attention_split_noalloc(const kv_ring_t* kv, const void* q, int n_q, i
   return launch_split_combine(a, kv->head_dim, n_splits, s);
 }
 
+int chunk_attention_multi(const kv_ring_t* const* rings, int n_rings, const void* q, int n_q,
+                          int64_t q_pos0, int n_current, const kv_block_mask_t* mask,
+                          const kv_cache_bias_t* bias, float softmax_scale, void* out,
+                          float* lse, int n_splits, void* workspace, size_t workspace_bytes,
+                          uint32_t flags, void* stream) {
+  if (!rings || n_rings < 1 || n_rings > KV_MAX_RINGS) return KV_EINVAL;
+  AttnArgs a[KV_MAX_RINGS];
+  for (int r = 0; r < n_rings; ++r) {
+    if (!rings[r]) return KV_EINVAL;
+    // every ring after the first holds history only
+    int rc = attention_args(rings[r], q, n_q, q_pos0, r == 0 ? n_current : 0, mask, bias,
+                            softmax_scale, out, lse, flags, &a[r]);
+    if (rc) return rc;
+    if (rings[r]->n_heads != rings[0]->n_heads || rings[r]->head_dim != rings[0]->head_dim ||
+        rings[r]->rope_base != rings[0]->rope_base)
+      return KV_EINVAL;
+  }
+  if (n_q == 0) return KV_OK;
+  if (rings[0]->head_dim != 128) return KV_EUNSUPPORTED;
+  if (n_splits < 1 || n_splits > 64 || n_rings * n_splits > 64) return KV_EINVAL;
+  const int H = rings[0]->n_heads, D = rings[0]->head_dim, S = n_rings * n_splits;
+  const size_t need = chunk_attention_workspace_size(n_q, H, D, S);
+  if (!workspace || !aligned16(workspace)) return KV_EINVAL;
+  if (workspace_bytes < need) return KV_ERANGE;
+  // partials of all rings in one workspace: O as [S][n_q][H][D], then (m, l) as
+  // [S][H][n_q]; ring r owns splits [r * n_splits, (r + 1) * n_splits)
+  float* const part_o = static_cast<float*>(workspace);
+  float* const part_ml = part_o + (size_t)S * n_q * H * D;
+  if (int rc = attach_timeouts(&a[0])) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (int r = 0; r < n_rings; ++r) {
+    a[r].timeouts = a[0].timeouts;
+    a[r].part_o = part_o + (size_t)r * n_splits * n_q * H * D;
+    a[r].part_ml = part_ml + (size_t)r * n_splits * n_q * H * 2;
+    const int rc = launch_attention_sm100_d128(a[r], rings[r]->opaque + kOpaqueTmapKsw,
+                                               rings[r]->opaque + kOpaqueTmapVsw, s, n_splits);
+    if (rc) return rc;
+  }
+  AttnArgs m = a[0];
+  m.part_o = part_o;
+  m.part_ml = part_ml;
+  return launch_split_combine(m, D, S, s);
+}
+
 int kv_wait_timeout_count(uint32_t* host_count) {
   if (!host_count) return KV_EINVAL;
   unsigned int v = 0;

@@ -182,3 +182,41 @@ def test_noalloc_rejects_oversize_before_any_cuda_call(L):
     # within the limit the call reaches the device (none here)
     assert L.chunk_attention_split_noalloc(r, 16, 1024, 0, 8, None, None, 0.125, 16, None,
                                            9, 0, None) == kv.KV_ECUDA
+
+
+def test_multi_ring_validation_before_launch(L):
+    """chunk_attention_multi refuses bad ring lists, splits and workspaces on the host.
+    Every call here is invalid, so none reaches a launch (the rings are fakes)."""
+    main, anchor = _fake_ring(D=128), _fake_ring(C=64, D=128)
+    main.live, anchor.live = 64, 32
+    arr = lambda *rs: (ctypes.c_void_p * len(rs))(*[ctypes.addressof(r) for r in rs])
+    need = kv.chunk_attention_workspace_size(8, 2, 128, 2 * 4)
+
+    def call(rings, n_rings, n_current=8, n_splits=4, ws=16, nbytes=need, flags=0):
+        return L.chunk_attention_multi(rings, n_rings, 16, 8, 0, n_current, None, None, 0.125,
+                                       16, None, n_splits, ws, nbytes, flags, None)
+
+    two = arr(main, anchor)
+    assert call(None, 2) == kv.KV_EINVAL
+    assert call(two, 0) == kv.KV_EINVAL
+    assert call(arr(*([main] * 9)), 9) == kv.KV_EINVAL                  # > KV_MAX_RINGS
+    assert call((ctypes.c_void_p * 2)(ctypes.addressof(main), None), 2) == kv.KV_EINVAL
+    assert call(two, 2, n_splits=0) == kv.KV_EINVAL
+    assert call(two, 2, n_splits=33) == kv.KV_EINVAL                    # 2 x 33 > 64 splits
+    assert call(two, 2, ws=None) == kv.KV_EINVAL
+    assert call(two, 2, ws=17) == kv.KV_EINVAL                          # misaligned
+    assert call(two, 2, nbytes=need - 1) == kv.KV_ERANGE                # sized for 8 splits
+    assert call(two, 2, n_current=65) == kv.KV_ERANGE                   # main ring: 64 valid
+    assert call(two, 2, flags=2) == kv.KV_EINVAL
+    wide = _fake_ring(C=64, H=4, D=128)
+    assert call(arr(main, wide), 2) == kv.KV_EINVAL                     # heads differ
+    other_base = _fake_ring(C=64, D=128)
+    other_base.rope_base = 500000.0
+    assert call(arr(main, other_base), 2) == kv.KV_EINVAL
+    short_table = _fake_ring(C=64, D=128, pmax=4)
+    assert call(arr(main, short_table), 2) == kv.KV_ERANGE              # q positions 0..7
+    assert call(arr(main, kv.kv_ring_t()), 2) == kv.KV_ESTATE
+    m64, a64 = _fake_ring(D=64), _fake_ring(C=64, D=64)
+    m64.live = 64
+    assert call(arr(m64, a64), 2) == kv.KV_EUNSUPPORTED
+    assert kv.KV_MAX_RINGS == 8
