@@ -44,15 +44,30 @@ def bf16(x32: np.ndarray) -> np.ndarray:
     return t.to(torch.bfloat16).to(torch.float32).numpy()
 
 
-def angles(p: int, D: int, base: float):
-    c = np.array([math.cos(p * (base ** (-(2.0 * i) / D))) for i in range(D // 2)], F32)
-    s = np.array([math.sin(p * (base ** (-(2.0 * i) / D))) for i in range(D // 2)], F32)
+def angles(p: int, D: int, base: float, rope3d=None):
+    """(cos, sin) per pair of token position p.  rope3d = (pairs_t, pairs_h, pairs_w,
+    grid_h, grid_w): pair i belongs to the time, height or width run; its coordinate is
+    the token's frame, row or column in a raster-ordered grid_h x grid_w frame, and its
+    frequency counts within its own run."""
+    if rope3d is None:
+        coord = [p] * (D // 2)
+        freq = [base ** (-(2.0 * i) / D) for i in range(D // 2)]
+    else:
+        pt, ph, pw, gh, gw = rope3d
+        frame, rest = divmod(p, gh * gw)          # floor division, rest >= 0
+        row, col = divmod(rest, gw)
+        coord, freq = [], []
+        for n, cval in ((pt, frame), (ph, row), (pw, col)):
+            coord += [cval] * n
+            freq += [base ** (-(2.0 * k) / (2 * n)) for k in range(n)]
+    c = np.array([math.cos(coord[i] * freq[i]) for i in range(D // 2)], F32)
+    s = np.array([math.sin(coord[i] * freq[i]) for i in range(D // 2)], F32)
     return c, s
 
 
-def rope32(x: np.ndarray, p: int, base: float) -> np.ndarray:
+def rope32(x: np.ndarray, p: int, base: float, rope3d=None) -> np.ndarray:
     """x: [..., D] float32, one position for all leading rows."""
-    c, s = angles(p, x.shape[-1], base)
+    c, s = angles(p, x.shape[-1], base, rope3d)
     x0, x1 = x[..., 0::2].astype(F32), x[..., 1::2].astype(F32)
     y = np.empty(x.shape, F32)
     y[..., 0::2] = x0 * c - x1 * s
@@ -87,8 +102,10 @@ def quant(y: np.ndarray):
 class BruteRing:
     """The ring as a linear list of token records."""
 
-    def __init__(self, C: int, H: int, D: int, base: float = 10000.0, next_pos: int = 0):
+    def __init__(self, C: int, H: int, D: int, base: float = 10000.0, next_pos: int = 0,
+                 rope3d=None):
         self.C, self.H, self.D, self.base = C, H, D, base
+        self.rope3d = rope3d
         self.tokens: list[dict] = []   # committed tokens, oldest first
         self.pending: list[dict] = []
         self.next_pos = next_pos
@@ -99,7 +116,7 @@ class BruteRing:
         self.pending = []
         for t in range(k.shape[0]):
             pos = self.next_pos + t
-            kc, ks = quant(rope32(k[t], pos, self.base))
+            kc, ks = quant(rope32(k[t], pos, self.base, self.rope3d))
             vc, vs = quant(v[t])
             self.pending.append(dict(g=g0 + t, pos=pos, kc=kc, ks=ks, vc=vc, vs=vs))
         if commit:
@@ -119,10 +136,12 @@ class BruteRing:
                 self.next_pos)
 
     def delta_rotate(self, delta: int):
+        if self.rope3d is not None and delta % (self.rope3d[3] * self.rope3d[4]) != 0:
+            raise ValueError("3-D resets move whole frames")
         for tok in self.window():
             # binary32 product: both factors are binary32, numpy rounds once
             x = (e4m3_values(tok["kc"]).astype(F32) * tok["ks"][:, None]).astype(F32)
-            tok["kc"], tok["ks"] = quant(rope32(x, delta, self.base))
+            tok["kc"], tok["ks"] = quant(rope32(x, delta, self.base, self.rope3d))
             tok["pos"] += delta
         self.next_pos += delta
 
@@ -168,7 +187,8 @@ class BruteRing:
         K = np.stack([e4m3_values(t["kc"]) * t["ks"][:, None].astype(np.float64) for t in win], 1)
         V = np.stack([e4m3_values(t["vc"]) * t["vs"][:, None].astype(np.float64) for t in win], 1)
         for h in range(H):
-            Q = np.stack([bf16(rope32(q[i, h], q_pos0 + i, self.base)) for i in range(n_q)])
+            Q = np.stack([bf16(rope32(q[i, h], q_pos0 + i, self.base, self.rope3d))
+                          for i in range(n_q)])
             if mode_b:
                 qc, qs = quant(Q)
                 Q = e4m3_values(qc) * qs[:, None].astype(np.float64)

@@ -177,6 +177,9 @@ ORC_API void orc_quant_row(const float* y, int D, uint8_t* code, float* scale) {
 typedef struct {
   int32_t C, H, D, _pad;
   double base;
+  /* 3-D RoPE (all zero: 1-D): pairs of the t, h, w runs of the head dimension and the
+   * frame grid (tokens per frame = grid_h * grid_w, raster order) */
+  int32_t pairs_t, pairs_h, pairs_w, grid_h, grid_w, _pad2;
   int64_t write_slot, live, pending, next_pos;
   uint8_t* kc;      /* [H][C][D] */
   uint8_t* vc;      /* [H][C][D] */
@@ -184,6 +187,37 @@ typedef struct {
   float* vs;        /* [H][C] */
   int32_t* slot_pos; /* [C] */
 } orc_ring;
+
+/* Angles of token position p under the ring's RoPE rule, rounded to binary32.
+ *  1-D (pairs all zero): pair i turns by p * base^(-2i/D) (orc_rope_cs).
+ *  3-D: the video-DiT form of RoPE, read from "Why Live Video Generation Still Struggles
+ *  With Timing", Transcript (positions of long streams calibrated and reset along time):
+ *  the D/2 pairs form three consecutive runs for time, height and width (pairs_t,
+ *  pairs_h, pairs_w of them); token position p is frame f = floor(p / (gh*gw)), row
+ *  y = floor(p / gw) mod gh and column x = p mod gw of a raster-ordered frame grid
+ *  gh x gw; pair k of a run of n pairs turns by (its coordinate) * base^(-2k/(2n)).
+ *  With pairs (D/2, 0, 0) and a 1 x 1 grid this is the 1-D rule, bit for bit. */
+ORC_API void orc_rope_cs_ring(const orc_ring* r, int64_t p, float* c, float* s) {
+  if (r->pairs_t == 0 && r->pairs_h == 0 && r->pairs_w == 0) {
+    orc_rope_cs(p, r->D, r->base, c, s);
+    return;
+  }
+  const int64_t gh = r->grid_h, gw = r->grid_w, hw = gh * gw;
+  int64_t f = p / hw;
+  if (p % hw != 0 && p < 0) f -= 1;                        /* floor division */
+  const int64_t rem = p - f * hw;                          /* 0 <= rem < hw */
+  const int64_t coord[3] = {f, rem / gw, rem % gw};
+  const int n[3] = {r->pairs_t, r->pairs_h, r->pairs_w};
+  int at = 0;
+  for (int a = 0; a < 3; ++a) {
+    for (int k = 0; k < n[a]; ++k, ++at) {
+      double theta = pow(r->base, -(2.0 * (double)k) / (double)(2 * n[a]));
+      double angle = (double)coord[a] * theta;
+      c[at] = (float)cos(angle);
+      s[at] = (float)sin(angle);
+    }
+  }
+}
 
 static int64_t mod_c(int64_t a, int64_t C) {
   int64_t r = a % C;
@@ -217,7 +251,7 @@ ORC_API void orc_ring_write(orc_ring* r, const float* k, const float* v, int n, 
     float c[256], s[256], y[512];
     int64_t slot = mod_c(r->write_slot + t, C);
     int64_t pos = r->next_pos + t;
-    orc_rope_cs(pos, D, r->base, c, s);
+    orc_rope_cs_ring(r, pos, c, s);
     r->slot_pos[slot] = (int32_t)pos;
     for (int h = 0; h < H; ++h) {
       const float* kr = k + ((size_t)t * H + h) * D;
@@ -233,11 +267,17 @@ ORC_API void orc_ring_write(orc_ring* r, const float* k, const float* v, int n, 
 }
 
 /* Position reset: re-rotate every valid cached key by delta (dequantise, rotate,
- * requantise); V is untouched; slot positions and next_pos shift by delta. */
-ORC_API void orc_ring_delta_rotate(orc_ring* r, int64_t delta) {
+ * requantise); V is untouched; slot positions and next_pos shift by delta.  Under 3-D
+ * RoPE a reset moves time only: delta must be a whole number of frames (a multiple of
+ * grid_h * grid_w), whose angles are zero on the h and w runs; otherwise nothing changes
+ * and -1 is returned. */
+ORC_API int orc_ring_delta_rotate(orc_ring* r, int64_t delta) {
   const int C = r->C, H = r->H, D = r->D;
   float c[256], s[256];
-  orc_rope_cs(delta, D, r->base, c, s);
+  if ((r->pairs_t | r->pairs_h | r->pairs_w) != 0 &&
+      delta % ((int64_t)r->grid_h * r->grid_w) != 0)
+    return -1;
+  orc_rope_cs_ring(r, delta, c, s);
   int64_t nv = valid_slots(r);
 #pragma omp parallel for schedule(static)
   for (int64_t age = 0; age < nv; ++age) {
@@ -253,6 +293,7 @@ ORC_API void orc_ring_delta_rotate(orc_ring* r, int64_t delta) {
     }
   }
   r->next_pos += delta;
+  return 0;
 }
 
 /* ---------------------------------------------------------------- chunk attention */
@@ -288,7 +329,7 @@ ORC_API void orc_chunk_attention_multi(const orc_ring* const* rings, int n_rings
       const int i = rows ? rows[ri] : ri;
       float c[256], s[256], y[512];
       double qt[512];
-      orc_rope_cs(q_pos0 + i, D, r0->base, c, s);
+      orc_rope_cs_ring(r0, q_pos0 + i, c, s);
       orc_rope_apply(q + ((size_t)i * H + h) * D, D, c, s, y);
       for (int d = 0; d < D; ++d) y[d] = orc_bf16_round(y[d]);
       if (flags & 1) {

@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         L.orc_ring_commit.argtypes = [P]
         L.orc_ring_write.argtypes = [P, P, P, ctypes.c_int, ctypes.c_int]
         L.orc_ring_delta_rotate.argtypes = [P, ctypes.c_int64]
+        L.orc_ring_delta_rotate.restype = ctypes.c_int
+        L.orc_rope_cs_ring.argtypes = [P, ctypes.c_int64, P, P]
         L.orc_chunk_attention.argtypes = [
             P, P, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_float, ctypes.c_int, P,
@@ -145,6 +147,9 @@ def quant_rows(y) -> tuple[np.ndarray, np.ndarray]:
 class _RingStruct(ctypes.Structure):
     _fields_ = [("C", ctypes.c_int32), ("H", ctypes.c_int32), ("D", ctypes.c_int32),
                 ("_pad", ctypes.c_int32), ("base", ctypes.c_double),
+                ("pairs_t", ctypes.c_int32), ("pairs_h", ctypes.c_int32),
+                ("pairs_w", ctypes.c_int32), ("grid_h", ctypes.c_int32),
+                ("grid_w", ctypes.c_int32), ("_pad2", ctypes.c_int32),
                 ("write_slot", ctypes.c_int64), ("live", ctypes.c_int64),
                 ("pending", ctypes.c_int64), ("next_pos", ctypes.c_int64),
                 ("kc", ctypes.c_void_p), ("vc", ctypes.c_void_p), ("ks", ctypes.c_void_p),
@@ -152,10 +157,13 @@ class _RingStruct(ctypes.Structure):
 
 
 class OracleRing:
-    """Host-side oracle ring: codes [H][C][D] u8, scales [H][C] f32, slot_pos [C] i32."""
+    """Host-side oracle ring: codes [H][C][D] u8, scales [H][C] f32, slot_pos [C] i32.
+
+    rope3d = (pairs_t, pairs_h, pairs_w, grid_h, grid_w) selects 3-D RoPE (see
+    ``orc_rope_cs_ring`` in the C file); None is 1-D RoPE."""
 
     def __init__(self, capacity: int, n_heads: int, head_dim: int, base: float = 10000.0,
-                 next_pos: int = 0):
+                 next_pos: int = 0, rope3d=None):
         assert head_dim % 2 == 0 and head_dim <= 512
         self.C, self.H, self.D = capacity, n_heads, head_dim
         self.kc = np.zeros((n_heads, capacity, head_dim), np.uint8)
@@ -163,7 +171,11 @@ class OracleRing:
         self.ks = np.zeros((n_heads, capacity), np.float32)
         self.vs = np.zeros((n_heads, capacity), np.float32)
         self.slot_pos = np.zeros(capacity, np.int32)
-        self._s = _RingStruct(capacity, n_heads, head_dim, 0, float(base), 0, 0, 0,
+        r3 = (0, 0, 0, 0, 0) if rope3d is None else tuple(int(x) for x in rope3d)
+        if rope3d is not None:
+            assert sum(r3[:3]) == head_dim // 2 and min(r3) >= 0 and r3[3] >= 1 and r3[4] >= 1
+        self.rope3d = rope3d
+        self._s = _RingStruct(capacity, n_heads, head_dim, 0, float(base), *r3, 0, 0, 0, 0,
                               int(next_pos), self.kc.ctypes.data, self.vc.ctypes.data,
                               self.ks.ctypes.data, self.vs.ctypes.data,
                               self.slot_pos.ctypes.data)
@@ -201,7 +213,17 @@ class OracleRing:
         lib().orc_ring_commit(self._ptr())
 
     def delta_rotate(self, delta: int) -> None:
-        lib().orc_ring_delta_rotate(self._ptr(), int(delta))
+        rc = lib().orc_ring_delta_rotate(self._ptr(), int(delta))
+        if rc != 0:
+            raise ValueError(f"3-D RoPE resets move whole frames: {delta} is not a multiple "
+                             f"of the frame size")
+
+    def rope_cs(self, p: int):
+        """(cos, sin) of token position p under this ring's RoPE rule, binary32."""
+        c = np.empty(self.D // 2, np.float32)
+        s = np.empty(self.D // 2, np.float32)
+        lib().orc_rope_cs_ring(self._ptr(), int(p), _p(c), _p(s))
+        return c, s
 
     def attention(self, q, q_pos0: int, n_current: int, mask=(1 << 30, 1 << 30, 1 << 30, 1 << 30),
                   cache_bias: float = 0.0, softmax_scale: float | None = None, rows=None,

@@ -159,12 +159,13 @@ def test_quant_degenerate_rows(orc):
 
 # ---------------------------------------------------------------- ring == linear buffer
 
-def _tiny_stream(orc, check_every_pass=True, mode_b=False):
+def _tiny_stream(orc, check_every_pass=True, mode_b=False, rope3d=None):
     """The tiny workload: 12 chunks of 32 into 256 slots, 4 passes per chunk (3 pending
     rewrites and a commit), reset by -128 after chunk 8; attention on every last pass."""
     C, H, D, n = 256, 2, 64, 32
     rng = np.random.default_rng(1)
-    o, b = orc.OracleRing(C, H, D), brute.BruteRing(C, H, D)
+    o = orc.OracleRing(C, H, D, rope3d=rope3d)
+    b = brute.BruteRing(C, H, D, rope3d=rope3d)
     sm = float(np.float32(1 / np.sqrt(D)))
     worst = 0.0
     for ch in range(12):
