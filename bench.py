@@ -176,11 +176,10 @@ class RunwayStep:
             return (torch.randn((n, H, D), generator=g, device=dev) * sc).to(torch.bfloat16)
 
         self.rings = []
-        pre_k, pre_v = rnd(), rnd()
         for r in range(rings):
             ring = kv.KvRing(C, H, D, 0, 64 * n, device=dev, rope_table=self.table)
-            for _ in range(math.ceil(C / n)):          # fill: steady state, ring full
-                kv.kv_ring_write(ring, pre_k, pre_v, commit=True)
+            for _ in range(math.ceil(C / n)):          # fill: steady state, ring full, every
+                kv.kv_ring_write(ring, rnd(), rnd(), commit=True)   # chunk drawn afresh
             self.rings.append(ring)
         self.q = [[rnd() for _ in range(PASSES)] for _ in range(rings)]
         self.k = [[rnd() for _ in range(PASSES)] for _ in range(rings)]
@@ -232,6 +231,166 @@ def timed(torch, fn, reps: int, stream) -> float:
     return a.elapsed_time(b) / reps
 
 
+def per_call_percentiles(torch, step: "RunwayStep", stream) -> dict:
+    """Per-call device time (write + attention) of one eager pass over the step's 240
+    calls: an event between consecutive calls (the host runs ahead of the device, so the
+    gaps are device time)."""
+    kv, n = step.kv, step.w.n
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(step.n_rings * PASSES + 1)]
+    states = [tuple(r.state()) for r in step.rings]
+    torch.cuda.synchronize()
+    evs[0].record(stream)
+    i = 0
+    for p in range(PASSES):
+        for r, ring in enumerate(step.rings):
+            kv.kv_ring_write(ring, step.k[r][p], step.v[r][p], commit=(p == PASSES - 1))
+            kv.chunk_attention(ring, step.q[r][p], step._q_pos(ring, p, ("write",)), n,
+                               step.mask, 0.0, out=step.out[r], want_lse=False)
+            i += 1
+            evs[i].record(stream)
+    torch.cuda.synchronize()
+    for r, st in zip(step.rings, states):
+        r.s.write_slot, r.s.live, r.s.pending, r.s.next_pos = st
+    us = np.array([evs[k].elapsed_time(evs[k + 1]) * 1e3 for k in range(i)])
+    return {"p50_us": float(np.percentile(us, 50)), "p99_us": float(np.percentile(us, 99)),
+            "max_us": float(us.max()), "calls": int(i)}
+
+
+def fp8_gemm_peak(torch, reps: int = 10) -> dict:
+    """Dense e4m3 GEMM throughput on this GPU (torch._scaled_mm, 8192^3, bf16 out, best of
+    `reps`): the measured FP8 denominator beside the nominal bf16 x 2."""
+    try:
+        n = 8192
+        a = torch.randn((n, n), device="cuda").to(torch.float8_e4m3fn)
+        b = torch.randn((n, n), device="cuda").to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device="cuda")
+        for _ in range(3):
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        best = float("inf")
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        del a, b
+        return {"tflops": 2.0 * n ** 3 / (best * 1e-3) / 1e12, "shape": "8192^3 e4m3, bf16 out",
+                "how": "torch._scaled_mm, best of %d" % reps}
+    except Exception as e:                      # no FP8 GEMM in this torch build
+        return {"tflops": None, "error": str(e)[:200]}
+
+
+def attn_pairs(n_q: int, n_hist: int, q_first: int, q_block: int, k_first: int, k_block: int,
+               n_cur: int) -> int:
+    """Unmasked (query, key) pairs per head: every history slot plus the visible current
+    keys under the block mask (block id t < first ? 0 : 1 + (t - first) // len)."""
+    def bid(t, first, blen):
+        return np.where(t < first, 0, 1 + (t - first) // blen)
+    qb = bid(np.arange(n_q), q_first, q_block)
+    kb = bid(np.arange(n_cur), k_first, k_block)
+    kb_sorted = np.sort(kb)
+    visible = np.searchsorted(kb_sorted, qb, side="right")
+    return int(n_q * n_hist + visible.sum())
+
+
+def _filled_ring(torch, kv, inputs, w, dev, n_chunks, first_n=None, span=None):
+    span = 2 * w.C if span is None else span
+    ring = kv.KvRing(w.C, w.H, w.D, -span // 4, span, device=dev)
+    for ch in range(n_chunks):
+        n = first_n if (ch == 0 and first_n) else w.n
+        q, k, v = inputs.chunk_qkv_torch(w, ch, device=dev)
+        kv.kv_ring_write(ring, k[:n].contiguous(), v[:n].contiguous(), commit=True)
+    return ring
+
+
+def config_timings(torch, kv, inputs, dev, stream, peaks, reps: int = 10) -> dict:
+    """The other workloads, each timed on its own ring (every ring is larger than L2):
+    Wan-style chunk (bias sweep), joint audio+video paths, long-stream chunk."""
+    out = {}
+    bf16_sus = peaks["bf16_sus"]
+    # Wan-style: 4 committed chunks + the pending one, 4 passes with bias -3..0
+    w = inputs.WAN
+    ring = _filled_ring(torch, kv, inputs, w, dev, 4)
+    q, k, v = inputs.chunk_qkv_torch(w, 4, device=dev)
+    kv.kv_ring_write(ring, k, v)
+    o = torch.empty_like(q)
+    def wan():
+        for b in w.biases:
+            kv.chunk_attention(ring, q, ring.next_pos, w.n, w.mask, b, out=o, want_lse=False)
+    wan()
+    ms = timed(torch, wan, reps, stream) / len(w.biases)
+    flop = 4 * w.D * w.H * attn_pairs(w.n, w.C - w.n, *w.mask, w.n)
+    out["wan_4680x23400"] = {"us_per_call": ms * 1e3, "gflop_per_call": flop / 1e9,
+                             "tflops": flop / (ms * 1e-3) / 1e12,
+                             "frac_bf16_sustained": flop / (ms * 1e-3) / 1e12 / bf16_sus,
+                             "biases": list(w.biases)}
+    del ring, q, k, v, o
+    # joint audio+video: 20 prior blocks in each ring plus the pending block
+    wv, wa = inputs.AV_VIDEO, inputs.AV_AUDIO
+    # both rings cover the video positions: cross-modal queries keep their own positions
+    rv = _filled_ring(torch, kv, inputs, wv, dev, 20, wv.extra["first_n"], span=2 * wv.C)
+    ra = _filled_ring(torch, kv, inputs, wa, dev, 20, wa.extra["first_n"], span=2 * wv.C)
+    qv, kvv, vv = inputs.chunk_qkv_torch(wv, 20, device=dev)
+    qa, kva, va = inputs.chunk_qkv_torch(wa, 20, device=dev)
+    kv.kv_ring_write(rv, kvv, vv)
+    kv.kv_ring_write(ra, kva, va)
+    ov, oa = torch.empty_like(qv), torch.empty_like(qa)
+    splits = 16
+    ws = torch.empty(kv.chunk_attention_workspace_size(wa.n, wa.H, wa.D, splits),
+                     dtype=torch.uint8, device=dev)
+    def vv_():
+        kv.chunk_attention(rv, qv, rv.next_pos, wv.n, None, 0.0, out=ov, want_lse=False)
+    def av_():
+        kv.chunk_attention_split(rv, qa, ra.next_pos, wv.n, splits, ws, cache_bias=0.0,
+                                 out=oa, want_lse=False)
+    def va_():
+        kv.chunk_attention(ra, qv, rv.next_pos, wa.n, None, 0.0, out=ov, want_lse=False)
+    def aa_():
+        kv.chunk_attention(ra, qa, ra.next_pos, wa.n, None, 0.0, out=oa, want_lse=False)
+    for f in (vv_, av_, va_, aa_):
+        f()
+    t_vv = timed(torch, vv_, reps, stream)
+    t_av = timed(torch, av_, reps, stream)
+    t_va = timed(torch, va_, reps, stream)
+    t_aa = timed(torch, aa_, reps, stream)
+    f_vv = 4 * wv.D * wv.H * wv.n * wv.C
+    av_bytes = wv.C * wv.H * (2 * wv.D + 8)          # K, V codes and scales of the video ring
+    out["av_v2v_1152x24192"] = {"us_per_call": t_vv * 1e3, "gflop_per_call": f_vv / 1e9,
+                                "tflops": f_vv / (t_vv * 1e-3) / 1e12,
+                                "frac_bf16_sustained": f_vv / (t_vv * 1e-3) / 1e12 / bf16_sus}
+    out["av_a2v_25x24192_split16"] = {"us_per_call": t_av * 1e3, "bytes_per_call": av_bytes,
+                                      "gbs": av_bytes / (t_av * 1e-3) / 1e9,
+                                      "frac_hbm": av_bytes / (t_av * 1e-3) / 1e9 / peaks["hbm"]}
+    out["av_v2a_1152x525"] = {"us_per_call": t_va * 1e3}
+    out["av_a2a_25x525"] = {"us_per_call": t_aa * 1e3}
+    del rv, ra, ws
+    # long stream: a full 32,768-slot ring of Student-t keys/values, a 1,024-token chunk
+    w = inputs.STRESS
+    ring = _filled_ring(torch, kv, inputs, w, dev, w.C // w.n)
+    q, k, v = inputs.chunk_qkv_torch(w, w.C // w.n, device=dev)
+    def wr():
+        kv.kv_ring_write(ring, k, v)
+    wr()
+    o = torch.empty_like(q)
+    def at():
+        kv.chunk_attention(ring, q, ring.next_pos, w.n, None, -4.0, out=o, want_lse=False)
+    at()
+    t_w = timed(torch, wr, reps, stream)
+    t_a = timed(torch, at, reps, stream)
+    f_a = 4 * w.D * w.H * w.n * w.C
+    wb = write_bytes(w.n, w.H, w.D)
+    out["stress_1024x32768"] = {"attn_us": t_a * 1e3, "attn_gflop": f_a / 1e9,
+                                "attn_tflops": f_a / (t_a * 1e-3) / 1e12,
+                                "attn_frac_bf16_sustained": f_a / (t_a * 1e-3) / 1e12 / bf16_sus,
+                                "write_us": t_w * 1e3, "write_gbs": wb / (t_w * 1e-3) / 1e9,
+                                "write_frac_hbm": wb / (t_w * 1e-3) / 1e9 / peaks["hbm"],
+                                "inputs": "K, V Student-t(4); Q N(0,1); bias -4"}
+    del ring
+    torch.cuda.synchronize()
+    return out
+
+
 def max_over_ranks(torch, dist, x: float) -> float:
     if dist is None:
         return x
@@ -267,33 +426,59 @@ def rotate_timing(torch, kv, inputs, dev, reps: int = 20) -> dict:
 
 def e2e_timing(torch, kv, step: RunwayStep, steps: int, stream) -> dict:
     """Same step through the public API from pinned host buffers: every call copies its
-    q, k, v host->device and its output device->host inside the timed region."""
+    q, k, v host->device and its output device->host inside the timed region.  The copies
+    overlap the kernels: a copy-in stream brings call i+1's inputs while call i computes,
+    and a copy-out stream returns call i's output while call i+1 computes (device inputs
+    and outputs double-buffered, ordered by events)."""
     n_sets = min(8, step.n_rings)
     host = []
     for s in range(n_sets):
         host.append([[step.q[s][p].cpu().pin_memory(), step.k[s][p].cpu().pin_memory(),
                       step.v[s][p].cpu().pin_memory()] for p in range(PASSES)])
-    dq = torch.empty_like(step.q[0][0])
-    dk = torch.empty_like(step.k[0][0])
-    dv = torch.empty_like(step.v[0][0])
     outs = [torch.empty(step.out[0].shape, dtype=torch.bfloat16).pin_memory() for _ in range(n_sets)]
+    dev_in = [[torch.empty_like(step.q[0][0]) for _ in range(3)] for _ in range(2)]
+    dev_out = [torch.empty_like(step.out[0]) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]      # inputs of buffer b have landed
+    ev_used = [torch.cuda.Event() for _ in range(2)]    # kernels are done with buffer b
+    ev_out = [torch.cuda.Event() for _ in range(2)]     # output of buffer b is on the host
     n = step.w.n
+    calls = [(p, r) for p in range(PASSES) for r in range(step.n_rings)]
+
+    def issue_in(i):
+        p, r = calls[i]
+        b = i % 2
+        s_in.wait_event(ev_used[b])                     # call i-2 has finished with b
+        with torch.cuda.stream(s_in):
+            for d, h in zip(dev_in[b], host[r % n_sets][p]):
+                d.copy_(h, non_blocking=True)
+        ev_in[b].record(s_in)
 
     def one_step():
-        for p in range(PASSES):
-            for r, ring in enumerate(step.rings):
-                hq, hk, hv = host[r % n_sets][p]
-                dq.copy_(hq, non_blocking=True)
-                dk.copy_(hk, non_blocking=True)
-                dv.copy_(hv, non_blocking=True)
-                last = p == PASSES - 1
-                kv.kv_ring_write(ring, dk, dv, commit=last)
-                kv.chunk_attention(ring, dq, ring.next_pos - (n if last else 0), n, step.mask,
-                                   0.0, out=step.out[r], want_lse=False)
-                outs[r % n_sets].copy_(step.out[r], non_blocking=True)
+        s_in.wait_stream(stream)                        # nothing starts before the timer
+        issue_in(0)
+        for i, (p, r) in enumerate(calls):
+            b = i % 2
+            if i + 1 < len(calls):
+                issue_in(i + 1)
+            ring = step.rings[r]
+            stream.wait_event(ev_in[b])
+            stream.wait_event(ev_out[b])                # call i-2's output has left dev_out[b]
+            dq, dk, dv = dev_in[b]
+            last = p == PASSES - 1
+            kv.kv_ring_write(ring, dk, dv, commit=last, stream=stream)
+            kv.chunk_attention(ring, dq, ring.next_pos - (n if last else 0), n, step.mask,
+                               0.0, out=dev_out[b], want_lse=False, stream=stream)
+            ev_used[b].record(stream)
+            s_out.wait_event(ev_used[b])
+            with torch.cuda.stream(s_out):
+                outs[r % n_sets].copy_(dev_out[b], non_blocking=True)
+            ev_out[b].record(s_out)
+        stream.wait_stream(s_out)                       # the timer ends after the last copy
 
     one_step()
     ms = timed(torch, one_step, steps, stream)
+    dq = dev_in[0][0]
     h2d = step.n_rings * PASSES * 3 * dq.numel() * dq.element_size()
     d2h = step.n_rings * PASSES * step.out[0].numel() * 2
     return {"ms_per_step": ms, "h2d": h2d, "d2h": d2h}
@@ -337,10 +522,14 @@ class CpuBaseline:
         t_attn = time.perf_counter() - t0
         per_call_s = t_write + t_attn * w.n / self.rows
         cores = int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
+        full = self.rows == w.n
+        what = ("one full call: 757-token x 40-head write + attention of all 757 query rows x "
+                "40 heads over 5,788 slots, timed whole" if full else
+                f"one full 757-token x 40-head write + attention of {self.rows} seeded query "
+                f"rows x 40 heads over 5,788 slots; attention time scaled x{w.n}/{self.rows} "
+                f"(rows are independent, so the work scales exactly)")
         return {"value": per_call_s * 1e6, "unit": UNIT, "cores": cores, "kind": "oracle",
-                "sample": f"one full 757-token x 40-head write + attention of {self.rows} "
-                          f"seeded query rows x 40 heads over 5,788 slots, attention scaled "
-                          f"x{w.n}/{self.rows}",
+                "sample": what, "scaled_estimate": not full,
                 "write_s": t_write, "attn_s": t_attn}
 
 
@@ -376,6 +565,10 @@ def run_reference(args, rank: int, world: int):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_block({"reference": "fp64 C oracle (OpenMP), bounded sample per "
                                                  "step, scaled to a full call"}),
+            "estimate": "value and ms_per_step are scaled estimates: each step times one "
+                        "full write and a seeded row sample of the attention, and scales the "
+                        "attention by 757/rows; ms_per_step multiplies by the 240 calls of "
+                        "a step, which no step actually ran",
             "cpu_baseline": cb,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -447,9 +640,13 @@ def main():
     if args.no_extras:
         rot = {"us_per_launch": float("nan"), "bytes_per_launch": 0}
         e2e = {"ms_per_step": float("nan"), "h2d": 0, "d2h": 0}
+        per_call, fp8, configs = None, None, None
     else:
         rot = rotate_timing(torch, kv, inputs, dev)
         e2e = e2e_timing(torch, kv, step, args.e2e_steps, stream)
+        per_call = per_call_percentiles(torch, step, stream)
+        fp8 = fp8_gemm_peak(torch)
+        configs = config_timings(torch, kv, inputs, dev, stream, peaks)
     rot_us = max_over_ranks(torch, dist, rot["us_per_launch"])
     e2e_ms = max_over_ranks(torch, dist, e2e["ms_per_step"])
     timeouts = kv.kv_wait_timeout_count()
@@ -479,7 +676,11 @@ def main():
                       "frac_bf16_sustained": attn_tflops / peaks["bf16_sus"],
                       "frac_fp8_dense": attn_tflops / fp8_peak,
                       "fp8_peak_tflops": fp8_peak,
-                      "fp8_peak_note": f"{peaks['src']} bf16 burst x 2 (nominal ratio)"},
+                      "fp8_peak_note": f"{peaks['src']} bf16 burst x 2 (nominal ratio)",
+                      "fp8_gemm_measured": fp8,
+                      "frac_fp8_measured": (attn_tflops / fp8["tflops"]
+                                            if fp8 and fp8.get("tflops") else None),
+                      "per_call_write_plus_attention": per_call},
         "attention_mode_b": {
             "us_per_call": ms_attn_b * 1e3, "tflops": flop / (ms_attn_b * 1e-3) / 1e12,
             "frac_bf16_sustained": flop / (ms_attn_b * 1e-3) / 1e12 / peaks["bf16_sus"],
@@ -500,13 +701,14 @@ def main():
                                   f"P.V is f16 (same rate), so the bf16 peak bounds 4*D flops/pair"},
         "e2e": {"value": e2e_ms * 1e3 / (R * PASSES) / world, "unit": UNIT,
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+        "configs": configs,
         "gpu_launches": 2 * R * PASSES * args.steps,
         "clocks": clk,
         "wait_timeouts": timeouts,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.no_extras:
         cpu = CpuBaseline()
-        cpu.calibrate(target_s=12.0)
+        cpu.calibrate(target_s=30.0)                 # a whole call on a 16-core host
         line["cpu_baseline"] = cpu.sample()
     if dist is not None:
         dist.barrier()

@@ -17,9 +17,14 @@
  *
  * Conventions shared by every entry point
  *  - Ownership: the caller allocates and owns every device buffer and the CUDA stream.
- *    The library allocates no device memory, keeps no global state and never
- *    synchronises the stream.  Kernels are enqueued on `stream` (a cudaStream_t; NULL is
- *    the legacy default stream) and read/write only the buffers named in the call.
+ *    The library allocates no device memory at run time and never synchronises the
+ *    stream.  Kernels are enqueued on `stream` (a cudaStream_t; NULL is the legacy default
+ *    stream) and read/write only the buffers named in the call, plus the library's own
+ *    module-level device state: a wait-timeout counter (kv_wait_timeout_count) and the
+ *    scratch of chunk_attention_split_noalloc, one of each per device, present from module
+ *    load.  The host keeps, per device, the addresses of those two symbols (looked up on
+ *    first use, then cached) and whether each kernel's shared-memory limit has been
+ *    raised; these tables are guarded by mutexes.
  *  - Errors: every function returns KV_OK (0) or a negative KV_E* code.  Argument, shape,
  *    state and range errors are detected on the host before anything is enqueued, and
  *    leave the ring state unchanged.  A launch failure returns KV_ECUDA (the CUDA error
@@ -114,6 +119,13 @@ typedef struct kv_ring {
   int64_t rope_pos_min;      /* first position held by rope_table */
   int64_t rope_pos_max;      /* last position held by rope_table */
   double rope_base;          /* base used to build the table (for the delta rotation) */
+  /* 3-D RoPE (all three pair counts 0 = 1-D RoPE): pairs of the time, height and width
+   * runs of the head dimension (their sum is head_dim/2) and the frame grid
+   * (rope_grid_h x rope_grid_w tokens per frame, raster order).  The table must then be
+   * built by kv_rope3d_table_build with the same values. */
+  int32_t rope_pairs_t, rope_pairs_h, rope_pairs_w;
+  int32_t rope_grid_h, rope_grid_w;
+  int32_t rope_reserved;     /* 0 */
   uint64_t opaque[96];       /* library-owned: encoded TMA descriptors of the caches */
 } kv_ring_t;
 
@@ -145,9 +157,27 @@ typedef struct kv_cache_bias {
 KV_API int kv_rope_table_build(float* host_out, int64_t pos_min, int64_t pos_max, int head_dim,
                         double base);
 
+/* 3-D RoPE table: the same layout and binary32 rounding as kv_rope_table_build, for the
+ * video form of RoPE ("Why Live Video Generation Still Struggles With Timing",
+ * Transcript: positions of long streams are calibrated and reset along time; the run
+ * split and frame grid are the usual video-DiT layout).  Token position p is frame
+ * f = floor(p / (grid_h * grid_w)), row y = floor(p / grid_w) mod grid_h and column
+ * x = p mod grid_w; pairs [0, pairs_t) turn by f * theta, the next pairs_h by y * theta,
+ * the last pairs_w by x * theta, where the k-th pair of a run of n pairs has
+ * theta = base^(-2k / (2n)) (pow in binary64, angle in binary64, cos/sin rounded to
+ * binary32).  With pairs (D/2, 0, 0) and a 1 x 1 grid the table is kv_rope_table_build's.
+ * The kernels read the table by position, so the write, the query rotation and the
+ * attention are unchanged.  Errors: KV_EINVAL (null, pairs negative or not summing to
+ * D/2, grid < 1, pos_max < pos_min, base <= 0). */
+KV_API int kv_rope3d_table_build(float* host_out, int64_t pos_min, int64_t pos_max, int head_dim,
+                                 double base, int pairs_t, int pairs_h, int pairs_w,
+                                 int grid_h, int grid_w);
+
 /* Validate a filled kv_ring_t, check the current device is sm_100, encode the TMA
  * descriptors of the caches into kv->opaque, and reset write_slot, live and pending to 0
  * (next_pos is kept).  Must be called again after any device pointer changes.
+ * 3-D RoPE fields: all pair counts 0 (1-D), or non-negative counts summing to head_dim/2
+ * with rope_grid_h, rope_grid_w >= 1 and rope_grid_h * rope_grid_w <= 2^24.
  * Errors: KV_EINVAL, KV_EUNSUPPORTED, KV_ECUDA. */
 KV_API int kv_ring_init(kv_ring_t* kv);
 
@@ -169,10 +199,13 @@ KV_API int kv_ring_commit(kv_ring_t* kv);
 
 /* Position reset ("Runway Characters", abstract: a delta rotation when positions reset):
  * every valid cached key row is dequantised (code * scale, binary32), rotated by the
- * angles of `delta` (computed on the host by the RoPE rule with kv->rope_base) and
+ * angles of `delta` (computed on the host by the ring's RoPE rule with kv->rope_base) and
  * requantised by the rule above; slot_pos of valid slots and next_pos shift by delta.
- * V is untouched.  Errors: KV_EINVAL, KV_ERANGE (shifted positions leave int32),
- * KV_ESTATE, KV_ECUDA. */
+ * V is untouched.  Under 3-D RoPE a reset moves time only: delta must be a whole number
+ * of frames (a multiple of rope_grid_h * rope_grid_w), whose angles are zero on the
+ * height and width runs (those pairs pass through the rotation unchanged and are
+ * requantised with the row).  Errors: KV_EINVAL (also a 3-D delta that is not a whole
+ * number of frames), KV_ERANGE (shifted positions leave int32), KV_ESTATE, KV_ECUDA. */
 KV_API int kv_ring_delta_rotate(kv_ring_t* kv, int64_t delta, void* stream);
 
 /* Chunk attention ("Runway Characters", abstract: each call reads the whole cache, only
@@ -188,6 +221,26 @@ KV_API int kv_ring_delta_rotate(kv_ring_t* kv, int64_t delta, void* stream);
 KV_API int chunk_attention(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
                     int n_current, const kv_block_mask_t* mask, const kv_cache_bias_t* bias,
                     float softmax_scale, void* out, float* lse, uint32_t flags, void* stream);
+
+/* Chunk attention for a gathered subset of the chunk's query rows ("Why Live Video
+ * Generation Still Struggles With Timing", Transcript, the LiveEdit passage: a mask cache
+ * finds the edited regions and self-attention is recomputed only there).  q, n_q, q_pos0,
+ * n_current, mask, bias, softmax_scale, out, lse and flags mean what they mean for
+ * chunk_attention, for the whole chunk of n_q queries.  rows: device int32 [n_rows],
+ * 4-byte aligned, the chunk indices of the queries to compute, in any order, duplicates
+ * allowed.  For each listed index i in [0, n_q), out[i] and lse[:, i] receive exactly
+ * the values chunk_attention writes there (query rotated at q_pos0 + i, block id of i);
+ * every other row of out and lse is left as it was (the static regions keep their
+ * previous outputs).  A listed index outside [0, n_q) is skipped: nothing is computed or
+ * written for it (the indices live on the device, so the host cannot reject them).
+ * n_rows = 0 enqueues nothing.  head_dim 128 only.  Errors: those of chunk_attention,
+ * KV_EINVAL (rows null or misaligned, n_rows < 0), KV_ERANGE (n_rows * n_heads > 2^31),
+ * KV_EUNSUPPORTED (head_dim 64). */
+KV_API int chunk_attention_rows(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
+                                int n_current, const int32_t* rows, int n_rows,
+                                const kv_block_mask_t* mask, const kv_cache_bias_t* bias,
+                                float softmax_scale, void* out, float* lse, uint32_t flags,
+                                void* stream);
 
 /* Bytes of workspace chunk_attention_split needs: n_splits * n_q * n_heads * (4*head_dim + 8).
  * 0 for invalid arguments. */

@@ -8,8 +8,8 @@ missing or the device is not sm_100, calls raise.
 Entry points (same names as the C ABI): ``kv_rope_table_build``, ``KvRing`` (fills a
 ``kv_ring_t`` and calls ``kv_ring_init``), ``kv_ring_write``, ``kv_ring_commit``,
 ``kv_ring_delta_rotate``, ``chunk_attention``, ``chunk_attention_workspace_size``,
-``chunk_attention_split``, ``chunk_attention_split_noalloc``, ``kv_status_string``,
-``kv_wait_timeout_count``.
+``chunk_attention_split``, ``chunk_attention_split_noalloc``, ``chunk_attention_multi``,
+``chunk_attention_rows``, ``kv_status_string``, ``kv_wait_timeout_count``.
 """
 from __future__ import annotations
 
@@ -27,10 +27,10 @@ KV_DTYPE_BF16, KV_DTYPE_FP32 = 1, 2
 KV_COMMIT = 1
 KV_QK_FP8 = 1
 
-EXPORTS = ("kv_rope_table_build", "kv_ring_init", "kv_ring_write", "kv_ring_commit",
+EXPORTS = ("kv_rope_table_build", "kv_rope3d_table_build", "kv_ring_init", "kv_ring_write", "kv_ring_commit",
            "kv_ring_delta_rotate", "chunk_attention", "chunk_attention_workspace_size",
            "chunk_attention_split", "chunk_attention_split_noalloc", "chunk_attention_multi",
-           "kv_status_string", "kv_wait_timeout_count")
+           "chunk_attention_rows", "kv_status_string", "kv_wait_timeout_count")
 KV_NOALLOC_SCRATCH_BYTES = 16 << 20
 KV_MAX_RINGS = 8
 
@@ -50,7 +50,11 @@ class kv_ring_t(ctypes.Structure):
                 ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
                 ("slot_pos", ctypes.c_void_p), ("rope_table", ctypes.c_void_p),
                 ("rope_pos_min", ctypes.c_int64), ("rope_pos_max", ctypes.c_int64),
-                ("rope_base", ctypes.c_double), ("opaque", ctypes.c_uint64 * 96)]
+                ("rope_base", ctypes.c_double),
+                ("rope_pairs_t", ctypes.c_int32), ("rope_pairs_h", ctypes.c_int32),
+                ("rope_pairs_w", ctypes.c_int32), ("rope_grid_h", ctypes.c_int32),
+                ("rope_grid_w", ctypes.c_int32), ("rope_reserved", ctypes.c_int32),
+                ("opaque", ctypes.c_uint64 * 96)]
 
 
 class kv_block_mask_t(ctypes.Structure):
@@ -75,12 +79,15 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         P, I, I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
         L.kv_rope_table_build.argtypes = [P, I64, I64, I, ctypes.c_double]
+        L.kv_rope3d_table_build.argtypes = [P, I64, I64, I, ctypes.c_double, I, I, I, I, I]
         L.kv_ring_init.argtypes = [P]
         L.kv_ring_write.argtypes = [P, P, P, I, I, ctypes.c_uint32, P]
         L.kv_ring_commit.argtypes = [P]
         L.kv_ring_delta_rotate.argtypes = [P, I64, P]
         L.chunk_attention.argtypes = [P, P, I, I64, I, P, P, ctypes.c_float, P, P,
                                       ctypes.c_uint32, P]
+        L.chunk_attention_rows.argtypes = [P, P, I, I64, I, P, I, P, P, ctypes.c_float, P, P,
+                                           ctypes.c_uint32, P]
         L.kv_status_string.argtypes = [I]
         L.kv_status_string.restype = ctypes.c_char_p
         L.kv_wait_timeout_count.argtypes = [P]
@@ -125,11 +132,27 @@ def kv_rope_table_build(pos_min: int, pos_max: int, head_dim: int,
     return out
 
 
+def kv_rope3d_table_build(pos_min: int, pos_max: int, head_dim: int, rope3d,
+                          base: float = 10000.0) -> np.ndarray:
+    """Host 3-D RoPE table [(pos_max-pos_min+1)][head_dim/2][2] float32; rope3d =
+    (pairs_t, pairs_h, pairs_w, grid_h, grid_w)."""
+    out = np.empty((pos_max - pos_min + 1, head_dim // 2, 2), np.float32)
+    _check(lib().kv_rope3d_table_build(ctypes.c_void_p(out.ctypes.data), int(pos_min),
+                                       int(pos_max), int(head_dim), float(base),
+                                       *(int(x) for x in rope3d)),
+           "kv_rope3d_table_build")
+    return out
+
+
 class KvRing:
-    """A ring with its caller-owned device buffers (torch tensors) and its kv_ring_t."""
+    """A ring with its caller-owned device buffers (torch tensors) and its kv_ring_t.
+
+    rope3d = (pairs_t, pairs_h, pairs_w, grid_h, grid_w) selects 3-D RoPE (the table is
+    then built with kv_rope3d_table_build); None is 1-D RoPE."""
 
     def __init__(self, capacity: int, n_heads: int, head_dim: int, pos_min: int, pos_max: int,
-                 base: float = 10000.0, next_pos: int = 0, device=None, rope_table=None):
+                 base: float = 10000.0, next_pos: int = 0, device=None, rope_table=None,
+                 rope3d=None):
         import torch
         dev = torch.device("cuda") if device is None else torch.device(device)
         C, H, D = int(capacity), int(n_heads), int(head_dim)
@@ -140,7 +163,9 @@ class KvRing:
         self.v_scale = torch.zeros((H, C), dtype=torch.float32, device=dev)
         self.slot_pos = torch.zeros((C,), dtype=torch.int32, device=dev)
         if rope_table is None:
-            rope_table = torch.from_numpy(kv_rope_table_build(pos_min, pos_max, D, base)).to(dev)
+            host = (kv_rope_table_build(pos_min, pos_max, D, base) if rope3d is None else
+                    kv_rope3d_table_build(pos_min, pos_max, D, rope3d, base))
+            rope_table = torch.from_numpy(host).to(dev)
         self.rope_table = rope_table
         s = kv_ring_t()
         s.capacity, s.n_heads, s.head_dim = C, H, D
@@ -150,6 +175,9 @@ class KvRing:
         s.slot_pos = self.slot_pos.data_ptr()
         s.rope_table = self.rope_table.data_ptr()
         s.rope_pos_min, s.rope_pos_max, s.rope_base = int(pos_min), int(pos_max), float(base)
+        if rope3d is not None:
+            (s.rope_pairs_t, s.rope_pairs_h, s.rope_pairs_w, s.rope_grid_h,
+             s.rope_grid_w) = (int(x) for x in rope3d)
         self.s = s
         _check(lib().kv_ring_init(ctypes.byref(s)), "kv_ring_init")
 
@@ -211,6 +239,36 @@ def chunk_attention(ring: KvRing, q, q_pos0: int, n_current: int, mask=None,
                                  None if lse is None else _ptr(lse),
                                  KV_QK_FP8 if mode_b else 0, _stream(stream)),
            "chunk_attention")
+    return out, lse
+
+
+def chunk_attention_rows(ring: KvRing, q, q_pos0: int, n_current: int, rows, out, lse=None,
+                         mask=None, cache_bias: float = 0.0, softmax_scale: float | None = None,
+                         stream=None, mode_b: bool = False):
+    """chunk_attention for the listed query rows only: q is the whole chunk (bf16
+    [n_q][H][D]); rows is a device int32 tensor of chunk indices; out (bf16 [n_q][H][D])
+    and lse (fp32 [H][n_q], optional) receive the listed rows and keep every other row."""
+    import torch
+    assert q.is_cuda and q.dtype == torch.bfloat16 and q.is_contiguous()
+    n_q = int(q.shape[0])
+    assert q.shape == (n_q, ring.H, ring.D)
+    assert rows.is_cuda and rows.dtype == torch.int32 and rows.is_contiguous() and rows.dim() == 1
+    assert out.is_cuda and out.dtype == torch.bfloat16 and out.is_contiguous()
+    assert out.shape == q.shape
+    if lse is not None:
+        assert lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous()
+        assert lse.shape == (ring.H, n_q)
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(ring.D)
+    m = None if mask is None else kv_block_mask_t(*(int(x) for x in mask))
+    b = kv_cache_bias_t(float(cache_bias))
+    _check(lib().chunk_attention_rows(ring.ref, _ptr(q), n_q, int(q_pos0), int(n_current),
+                                      _ptr(rows), int(rows.numel()),
+                                      None if m is None else ctypes.byref(m), ctypes.byref(b),
+                                      float(softmax_scale), _ptr(out),
+                                      None if lse is None else _ptr(lse),
+                                      KV_QK_FP8 if mode_b else 0, _stream(stream)),
+           "chunk_attention_rows")
     return out, lse
 
 
@@ -284,14 +342,20 @@ def chunk_attention_multi(rings, q, q_pos0: int, n_current: int, n_splits: int, 
 
 def chunk_attention_split_noalloc(ring: KvRing, q, q_pos0: int, n_current: int, n_splits: int,
                                   out, lse=None, mask=None, cache_bias: float = 0.0,
-                                  softmax_scale: float | None = None, stream=None):
+                                  softmax_scale: float | None = None, stream=None,
+                                  mode_b: bool = False):
     """chunk_attention_split with the library's static per-device scratch instead of a
     workspace; `out` (and `lse`, if wanted) are caller-allocated, so the call allocates
     nothing.  Calls that overlap in time on one device race on the scratch."""
     import torch
     assert q.is_cuda and q.dtype == torch.bfloat16 and q.is_contiguous()
     n_q = int(q.shape[0])
-    assert q.shape == (n_q, ring.H, ring.D) and out.shape == q.shape
+    assert q.shape == (n_q, ring.H, ring.D)
+    assert out.is_cuda and out.dtype == torch.bfloat16 and out.is_contiguous()
+    assert out.shape == q.shape and out.device == q.device
+    if lse is not None:
+        assert lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous()
+        assert lse.shape == (ring.H, n_q) and lse.device == q.device
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(ring.D)
     m = None if mask is None else kv_block_mask_t(*(int(x) for x in mask))
@@ -299,7 +363,8 @@ def chunk_attention_split_noalloc(ring: KvRing, q, q_pos0: int, n_current: int, 
     _check(lib().chunk_attention_split_noalloc(
         ring.ref, _ptr(q), n_q, int(q_pos0), int(n_current),
         None if m is None else ctypes.byref(m), ctypes.byref(b), float(softmax_scale),
-        _ptr(out), None if lse is None else _ptr(lse), int(n_splits), 0, _stream(stream)),
+        _ptr(out), None if lse is None else _ptr(lse), int(n_splits),
+        KV_QK_FP8 if mode_b else 0, _stream(stream)),
         "chunk_attention_split_noalloc")
     return out, lse
 

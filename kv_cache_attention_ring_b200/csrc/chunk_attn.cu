@@ -394,13 +394,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 int launch_d(const AttnArgs& a, const void* tk, const void* tv, cudaStream_t s) {
   using S = Smem<D>;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(chunk_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)S::bytes) != cudaSuccess)
-      return KV_ECUDA;
-    configured = true;
-  }
+  static unsigned char configured[kMaxDevices] = {};
+  if (!smem_attr_set(reinterpret_cast<const void*>(chunk_attn_kernel<D>), (int)S::bytes,
+                     configured))
+    return KV_ECUDA;
   CUtensorMap mk, mv;
   memcpy(&mk, tk, sizeof(mk));
   memcpy(&mv, tv, sizeof(mv));

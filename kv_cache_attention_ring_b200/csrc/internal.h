@@ -47,14 +47,26 @@ struct AttnArgs {
   float bias_log2;          // history_bias * log2(e)
   unsigned int* timeouts;   // device counter of waits that gave up
   int mode_b;               // query quantised to e4m3 per row (one MMA set for Q.K^T)
+  // rows computed: the query indices rows[0 .. n_rows) (device int32), or 0 .. n_rows - 1
+  // when rows is null (then n_rows = n_q); indices outside [0, n_q) are skipped
+  const int32_t* rows;
+  int n_rows;
   // split over keys (gridDim.z splits): when part_o is set, each split writes its
   // unnormalised O [split][n_q][H][D] and (m, l) [split][H][n_q] (log2 units) there
   float* part_o;
   float* part_ml;
 };
 
-// Device address of the library's wait-timeout counter on the current device.
+// Largest device ordinal the per-device tables cover.
+constexpr int kMaxDevices = 64;
+
+// Device address of the library's wait-timeout counter on the current device (looked up
+// once per device, then cached).
 unsigned int* timeout_counter();
+
+// Set `func`'s dynamic shared-memory limit to `bytes` on the current device unless
+// done[device] says it is set already; false if the CUDA call fails.
+bool smem_attr_set(const void* func, int bytes, unsigned char (&done)[kMaxDevices]);
 
 int launch_write(const WriteArgs& a, int D, int in_dtype, cudaStream_t s);
 int launch_rotate(const RotateArgs& a, int D, cudaStream_t s);

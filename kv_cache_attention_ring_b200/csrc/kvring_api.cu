@@ -18,31 +18,50 @@
 namespace kvring {
 __device__ unsigned int g_wait_timeouts = 0;
 
-unsigned int* timeout_counter() {
-  void* p = nullptr;
-  if (cudaGetSymbolAddress(&p, g_wait_timeouts) != cudaSuccess) return nullptr;
-  return static_cast<unsigned int*>(p);
-}
-
 // Partials of chunk_attention_split_noalloc: part of the module image, so every device
 // that loads the library has its own copy and no call allocates.
 __device__ __align__(256) unsigned char g_noalloc_scratch[KV_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
+std::mutex g_symbol_mu;
+void* g_timeouts_ptr[kMaxDevices] = {};
 void* g_noalloc_ptr[kMaxDevices] = {};
 
-// Device address of the current device's scratch, looked up once per device.
-void* noalloc_scratch() {
+// Device address of `symbol` on the current device, looked up once per device (with that
+// device current) and cached in table[device].
+template <typename T>
+void* symbol_address(const T& symbol, void* (&table)[kMaxDevices]) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  std::lock_guard<std::mutex> lock(g_symbol_mu);
+  if (!table[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    g_noalloc_ptr[dev] = p;
+    if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess) return nullptr;
+    table[dev] = p;
   }
-  return g_noalloc_ptr[dev];
+  return table[dev];
+}
+
+unsigned int* timeout_counter() {
+  return static_cast<unsigned int*>(symbol_address(g_wait_timeouts, g_timeouts_ptr));
+}
+
+// Device address of the current device's no-alloc scratch.
+void* noalloc_scratch() { return symbol_address(g_noalloc_scratch, g_noalloc_ptr); }
+
+// Raise a kernel's dynamic shared-memory limit once per device (the attribute is per
+// device context, so a process that drives several GPUs sets it on each).
+std::mutex g_smem_mu;
+bool smem_attr_set(const void* func, int bytes, unsigned char (&done)[kMaxDevices]) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(g_smem_mu);
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess)
+      return false;
+    done[dev] = 1;
+  }
+  return true;
 }
 }
 
@@ -72,6 +91,46 @@ void rope_angles(int64_t p, int D, double base, float* out /* [D/2][2] */) {
     out[2 * i] = (float)cos(angle);
     out[2 * i + 1] = (float)sin(angle);
   }
+}
+
+bool rope_is_3d(const kv_ring_t* kv) {
+  return (kv->rope_pairs_t | kv->rope_pairs_h | kv->rope_pairs_w) != 0;
+}
+
+// 3-D form: token position p -> (frame, row, column) of a raster-ordered grid_h x grid_w
+// frame; pair k of the time/height/width run of n pairs turns by that coordinate times
+// base^(-2k/(2n)), binary64, rounded to binary32.
+void rope_angles_3d(int64_t p, int D, double base, const int (&pairs)[3], int64_t grid_h,
+                    int64_t grid_w, float* out /* [D/2][2] */) {
+  const int64_t hw = grid_h * grid_w;
+  int64_t f = p / hw;
+  if (p < 0 && f * hw != p) f -= 1;                          // floor division
+  const int64_t rest = p - f * hw;
+  const int64_t coord[3] = {f, rest / grid_w, rest % grid_w};
+  int i = 0;
+  for (int run = 0; run < 3; ++run) {
+    for (int k = 0; k < pairs[run] && i < D / 2; ++k, ++i) {
+      const double theta = pow(base, -(2.0 * (double)k) / (double)(2 * pairs[run]));
+      const double angle = (double)coord[run] * theta;
+      out[2 * i] = (float)cos(angle);
+      out[2 * i + 1] = (float)sin(angle);
+    }
+  }
+}
+
+// Angles of position p under the ring's rule.
+void ring_angles(const kv_ring_t* kv, int64_t p, float* out) {
+  if (!rope_is_3d(kv)) {
+    rope_angles(p, kv->head_dim, kv->rope_base, out);
+    return;
+  }
+  const int pairs[3] = {kv->rope_pairs_t, kv->rope_pairs_h, kv->rope_pairs_w};
+  rope_angles_3d(p, kv->head_dim, kv->rope_base, pairs, kv->rope_grid_h, kv->rope_grid_w, out);
+}
+
+bool rope3d_valid(int D, int pt, int ph, int pw, int gh, int gw) {
+  return pt >= 0 && ph >= 0 && pw >= 0 && (int64_t)pt + ph + pw == D / 2 && gh >= 1 &&
+         gw >= 1 && (int64_t)gh * gw <= ((int64_t)1 << 24);
 }
 
 int check_ring(const kv_ring_t* kv) {
@@ -159,6 +218,19 @@ int kv_rope_table_build(float* host_out, int64_t pos_min, int64_t pos_max, int h
   return KV_OK;
 }
 
+int kv_rope3d_table_build(float* host_out, int64_t pos_min, int64_t pos_max, int head_dim,
+                          double base, int pairs_t, int pairs_h, int pairs_w, int grid_h,
+                          int grid_w) {
+  if (!host_out || head_dim <= 0 || (head_dim & 1) || pos_max < pos_min || !(base > 0.0))
+    return KV_EINVAL;
+  if (!rope3d_valid(head_dim, pairs_t, pairs_h, pairs_w, grid_h, grid_w)) return KV_EINVAL;
+  const int pairs[3] = {pairs_t, pairs_h, pairs_w};
+  for (int64_t p = pos_min; p <= pos_max; ++p)
+    rope_angles_3d(p, head_dim, base, pairs, grid_h, grid_w,
+                   host_out + (size_t)(p - pos_min) * head_dim);
+  return KV_OK;
+}
+
 int kv_ring_init(kv_ring_t* kv) {
   if (!kv) return KV_EINVAL;
   kv->initialized = 0;
@@ -170,6 +242,9 @@ int kv_ring_init(kv_ring_t* kv) {
   if (!aligned16(kv->k_codes) || !aligned16(kv->v_codes) || !aligned16(kv->rope_table))
     return KV_EINVAL;
   if (kv->rope_pos_max < kv->rope_pos_min || !(kv->rope_base > 0.0)) return KV_EINVAL;
+  if (rope_is_3d(kv) && !rope3d_valid(kv->head_dim, kv->rope_pairs_t, kv->rope_pairs_h,
+                                      kv->rope_pairs_w, kv->rope_grid_h, kv->rope_grid_w))
+    return KV_EINVAL;
   if ((int64_t)kv->capacity * kv->n_heads > (int64_t)1 << 31) return KV_ERANGE;
   if (kv->n_heads > 65535) return KV_ERANGE;          // heads index grid dimension y
   int dev = 0, major = 0, minor = 0;
@@ -250,6 +325,8 @@ int kv_ring_delta_rotate(kv_ring_t* kv, int64_t delta, void* stream) {
   const int64_t committed = nv - kv->pending;              // history still in the ring
   const int64_t lo = kv->next_pos - committed + delta;     // oldest valid position after
   const int64_t hi = kv->next_pos + (kv->pending > 0 ? kv->pending - 1 : 0) + delta;
+  if (rope_is_3d(kv) && delta % ((int64_t)kv->rope_grid_h * kv->rope_grid_w) != 0)
+    return KV_EINVAL;                                      // resets move whole frames
   if (delta < INT32_MIN || delta > INT32_MAX || lo < INT32_MIN || hi > INT32_MAX)
     return KV_ERANGE;
   if (nv > 0) {
@@ -262,7 +339,7 @@ int kv_ring_delta_rotate(kv_ring_t* kv, int64_t delta, void* stream) {
     a.first_slot = mod_c(kv->write_slot + kv->pending - nv, kv->capacity);
     a.count = nv;
     a.delta = (int32_t)delta;
-    rope_angles(delta, kv->head_dim, kv->rope_base, a.cs);
+    ring_angles(kv, delta, a.cs);
     rc = launch_rotate(a, kv->head_dim, static_cast<cudaStream_t>(stream));
     if (rc) return rc;
   }
@@ -322,6 +399,8 @@ int attention_args(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0, 
   a->part_o = nullptr;
   a->part_ml = nullptr;
   a->mode_b = (flags & KV_QK_FP8) ? 1 : 0;
+  a->rows = nullptr;
+  a->n_rows = n_q;
   return KV_OK;
 }
 
@@ -347,6 +426,27 @@ int chunk_attention(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
   return launch_attention(a, kv->head_dim, kv->opaque + kOpaqueTmapK,
                           kv->opaque + kOpaqueTmapV, kv->opaque + kOpaqueTmapKsw,
                           kv->opaque + kOpaqueTmapVsw, static_cast<cudaStream_t>(stream));
+}
+
+int chunk_attention_rows(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
+                         int n_current, const int32_t* rows, int n_rows,
+                         const kv_block_mask_t* mask, const kv_cache_bias_t* bias,
+                         float softmax_scale, void* out, float* lse, uint32_t flags,
+                         void* stream) {
+  AttnArgs a;
+  int rc = attention_args(kv, q, n_q, q_pos0, n_current, mask, bias, softmax_scale, out, lse,
+                          flags, &a);
+  if (rc) return rc;
+  if (n_rows < 0) return KV_EINVAL;
+  if (n_q == 0 || n_rows == 0) return KV_OK;
+  if (kv->head_dim != 128) return KV_EUNSUPPORTED;
+  if (!rows || (reinterpret_cast<uintptr_t>(rows) & 3u)) return KV_EINVAL;
+  if ((int64_t)n_rows * kv->n_heads > ((int64_t)1 << 31)) return KV_ERANGE;
+  if ((rc = attach_timeouts(&a))) return rc;
+  a.rows = rows;
+  a.n_rows = n_rows;
+  return launch_attention_sm100_d128(a, kv->opaque + kOpaqueTmapKsw, kv->opaque + kOpaqueTmapVsw,
+                                     static_cast<cudaStream_t>(stream), 1);
 }
 
 size_t chunk_attention_workspace_size(int n_q, int n_heads, int head_dim, int n_splits) {

@@ -9,14 +9,31 @@ import kv_cache_attention_ring_b200 as kv
 from kv_cache_attention_ring_b200 import inputs
 
 # Attention acceptance against the fp64 oracle evaluated on the same dequantised FP8
-# values: relative L2 <= 5e-3, and per element |o - ref| <= 2e-2 * max(1, |ref| / 4) --
-# the stated 2e-2 max-abs bound, kept absolute where a bf16 output can resolve it
-# (|o| < 4) and 5e-3 relative above, since a bf16 value of magnitude |o| is itself only
-# exact to 2^-9 |o| (an absolute 2e-2 is unreachable for |o| >= 8).
+# values: relative L2 <= 5e-3, and per element
+#     |o - ref| <= max(2e-2, hulp(ref) + 2^-10 |ref|),
+# the stated 2e-2 max-abs bound, widened only where a bf16 output cannot meet it.
+#   hulp(ref) = 2^(floor(log2 |ref|) - 8) is half a bf16 ulp at |ref|: the rounding of
+#     the output itself, which no bf16-output kernel avoids (it passes 2e-2 at |ref| >= 8).
+#   2^-10 |ref| is the kernel's own rounding budget: P and the scaled V operand are each
+#     rounded once to f16 (2^-11 relative each) before the fp32-accumulated P.V.
+# Below |ref| = 4 the right side is under 1.2e-2, so the bound there is 2e-2 absolute;
+# in [4, 8) it is 2e-2 to 2.3e-2; from 8 on it follows the bf16 grid.
 ATOL = 2e-2
-ATOL_KNEE = 4.0
+F16_BUDGET = 2.0 ** -10
 REL_L2 = 5e-3
 LSE_ATOL = 2e-3
+
+
+def half_ulp_bf16(x: np.ndarray) -> np.ndarray:
+    """Half a bf16 ulp at |x| (8 significant bits): 2^(floor(log2|x|) - 8); 0 at x = 0."""
+    ax = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
+    return np.where(ax > 0, np.exp2(e - 8.0), 0.0)
+
+
+def attention_bound(ref: np.ndarray) -> np.ndarray:
+    """Per-element max-abs bound of a bf16 attention output against the fp64 oracle."""
+    return np.maximum(ATOL, half_ulp_bf16(ref) + F16_BUDGET * np.abs(ref))
 
 
 def to_dev(t: torch.Tensor) -> torch.Tensor:
@@ -67,7 +84,7 @@ def assert_attention_close(out, lse, ref_out, ref_lse, rows=None, what=""):
             l = l[:, np.asarray(rows)]
     assert np.isfinite(o).all(), (what, "non-finite output")
     err = np.abs(o - ref_out)
-    bound = ATOL * np.maximum(1.0, np.abs(ref_out) / ATOL_KNEE)
+    bound = attention_bound(ref_out)
     rel = np.linalg.norm(o - ref_out) / max(np.linalg.norm(ref_out), 1e-30)
     worst = np.unravel_index(np.argmax(err / bound), err.shape)
     assert (err <= bound).all(), (what, "max abs", float(err[worst]), "at |ref|",

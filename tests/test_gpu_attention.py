@@ -70,16 +70,16 @@ def _runway_ring(orc, with_oracle=True, start_slot=1234):
 
 
 @pytest.mark.parametrize("mask", [(1, 1, 1, 1), (inputs.BIG,) * 4])
-def test_runway_shape_sampled_rows(orc, mask):
+def test_runway_shape_all_rows(orc, mask):
     """H=40, D=128, 757 new tokens over a full 5,788-slot FP8 ring, bias 0: token-causal
-    inside the new chunk, and the whole-chunk block variant."""
+    inside the new chunk, and the whole-chunk block variant; every row and head."""
     w = inputs.RUNWAY
     ring, o, q = _runway_ring(orc)
     assert ring.n_valid == w.C
     out, lse = kv.chunk_attention(ring, to_dev(q), ring.next_pos, w.n, mask, 0.0)
-    rows = sample_rows(w.n, 40, seed=5)
-    ro, rl = o.attention(inputs.as_f32(q), o.next_pos, w.n, mask, 0.0, rows=rows)
-    assert_attention_close(out, lse, ro, rl, rows=rows, what=f"runway {mask}")
+    ro, rl = o.attention(inputs.as_f32(q), o.next_pos, w.n, mask, 0.0)
+    e, r = assert_attention_close(out, lse, ro, rl, what=f"runway {mask}")
+    print(f"runway {mask}: max-abs {e:.3e} rel-L2 {r:.3e}")
 
 
 @pytest.mark.parametrize("n_q", [1, 127, 129, 300])
