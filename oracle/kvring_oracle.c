@@ -401,6 +401,107 @@ ORC_API void orc_chunk_attention(const orc_ring* r, const float* q, int n_q, int
                             k_block, cache_bias, softmax_scale, flags, rows, n_rows, out, lse);
 }
 
+/* ---------------------------------------------------------------- content memory */
+
+/* Attention mass that history slots of rings[ri] receive in one attention call over
+ * rings[0..n_rings) (same arguments as orc_chunk_attention_multi): for candidate c (the
+ * slot of age ages[c] in rings[ri], a history slot), mass[c] = sum over heads h and query
+ * rows i of exp(s_ihc - lse_ih), the softmax probability row i of head h gives the slot,
+ * with lse the call's own log-sum-exp over every visible key of every ring.  This is the
+ * "attention quality" of "Stream LTX", Inference (each layer scores its own keys), read
+ * as the probability mass the keys received from the newest chunk's queries. */
+ORC_API void orc_key_mass(const orc_ring* const* rings, int n_rings, const float* q, int n_q,
+                          int64_t q_pos0, int n_current, int q_first, int q_block,
+                          int k_first, int k_block, float cache_bias, float softmax_scale,
+                          int ri, const int64_t* ages, int n_cand, double* mass) {
+  const orc_ring* r0 = rings[0];
+  const orc_ring* rk = rings[ri];
+  const int H = r0->H, D = r0->D;
+  double* out = (double*)malloc(sizeof(double) * (size_t)n_q * H * D);
+  double* lse = (double*)malloc(sizeof(double) * (size_t)H * n_q);
+  orc_chunk_attention_multi(rings, n_rings, q, n_q, q_pos0, n_current, q_first, q_block,
+                            k_first, k_block, cache_bias, softmax_scale, 0, NULL, n_q, out, lse);
+  for (int c = 0; c < n_cand; ++c) mass[c] = 0.0;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int c = 0; c < n_cand; ++c) {
+    const int64_t slot = orc_slot_of_age(rk, ages[c]);
+    double acc = 0.0;
+    for (int h = 0; h < H; ++h) {
+      const uint8_t* kr = rk->kc + ((size_t)h * rk->C + slot) * D;
+      const double ksc = (double)rk->ks[(size_t)h * rk->C + slot];
+      for (int i = 0; i < n_q; ++i) {
+        if (!isfinite(lse[(size_t)h * n_q + i])) continue;
+        float cc[256], ss[256], y[512];
+        orc_rope_cs_ring(r0, q_pos0 + i, cc, ss);
+        orc_rope_apply(q + ((size_t)i * H + h) * D, D, cc, ss, y);
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d)
+          dot += (double)orc_bf16_round(y[d]) * (orc_e4m3_decode(kr[d]) * ksc);
+        const double sv = (double)softmax_scale * dot + (double)cache_bias;
+        acc += exp(sv - lse[(size_t)h * n_q + i]);
+      }
+    }
+    mass[c] = acc;
+  }
+  free(out);
+  free(lse);
+}
+
+/* Top-M selection with temporal diversity ("Stream LTX", Inference: keys scored on
+ * attention quality and temporal diversity, evicted down to a top-M budget).  Read as a
+ * greedy choice in which every key already kept from a frame multiplies the remaining
+ * keys of that frame by gamma: equivalently, the k-th best key of its frame (by quality,
+ * k = 0, 1, ...) scores quality * gamma^k, and the M best scores are kept.  Ties break
+ * toward the lower position, then the lower candidate index, so the choice is unique.
+ * Writes the kept candidate indices in ascending order and returns how many (min(n, M)). */
+typedef struct { double key; int64_t pos; int idx; int64_t frame; } orc_cand;
+
+static int cmp_frame_then_quality(const void* a, const void* b) {
+  const orc_cand *x = (const orc_cand*)a, *y = (const orc_cand*)b;
+  if (x->frame != y->frame) return x->frame < y->frame ? -1 : 1;
+  if (x->key != y->key) return x->key > y->key ? -1 : 1;
+  if (x->pos != y->pos) return x->pos < y->pos ? -1 : 1;
+  return x->idx < y->idx ? -1 : (x->idx > y->idx);
+}
+
+static int cmp_score(const void* a, const void* b) {
+  const orc_cand *x = (const orc_cand*)a, *y = (const orc_cand*)b;
+  if (x->key != y->key) return x->key > y->key ? -1 : 1;
+  if (x->pos != y->pos) return x->pos < y->pos ? -1 : 1;
+  return x->idx < y->idx ? -1 : (x->idx > y->idx);
+}
+
+static int cmp_int(const void* a, const void* b) {
+  const int x = *(const int*)a, y = *(const int*)b;
+  return x < y ? -1 : (x > y);
+}
+
+ORC_API int orc_memory_select(const double* quality, const int64_t* frame, const int64_t* pos,
+                              int n, int M, double gamma, int32_t* kept) {
+  orc_cand* c = (orc_cand*)malloc(sizeof(orc_cand) * (size_t)(n > 0 ? n : 1));
+  for (int i = 0; i < n; ++i) {
+    c[i].key = quality[i];
+    c[i].pos = pos[i];
+    c[i].idx = i;
+    c[i].frame = frame[i];
+  }
+  qsort(c, (size_t)n, sizeof(orc_cand), cmp_frame_then_quality);
+  double scale = 1.0;
+  for (int i = 0; i < n; ++i) {
+    scale = (i > 0 && c[i].frame == c[i - 1].frame) ? scale * gamma : 1.0;
+    c[i].key = c[i].key * scale;                     /* quality * gamma^(rank in frame) */
+  }
+  qsort(c, (size_t)n, sizeof(orc_cand), cmp_score);
+  const int m = n < M ? n : M;
+  int* ids = (int*)malloc(sizeof(int) * (size_t)(m > 0 ? m : 1));
+  for (int i = 0; i < m; ++i) ids[i] = c[i].idx;
+  qsort(ids, (size_t)m, sizeof(int), cmp_int);
+  for (int i = 0; i < m; ++i) kept[i] = ids[i];
+  free(ids);
+  free(c);
+  return m;
+}
+
 /* ---------------------------------------------------------------- array helpers for tests */
 
 ORC_API void orc_e4m3_encode_n(const float* v, int64_t n, uint8_t* out) {

@@ -69,6 +69,12 @@ def lib() -> ctypes.CDLL:
             P, ctypes.c_int, P, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_float,
             ctypes.c_int, P, ctypes.c_int, P, P]
+        L.orc_key_mass.argtypes = [
+            P, ctypes.c_int, P, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_float,
+            ctypes.c_int, P, ctypes.c_int, P]
+        L.orc_memory_select.argtypes = [P, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_double, P]
+        L.orc_memory_select.restype = ctypes.c_int
         L.orc_e4m3_encode_n.argtypes = [P, ctypes.c_int64, P]
         L.orc_e4m3_decode_n.argtypes = [P, ctypes.c_int64, P]
         L.orc_bf16_round_n.argtypes = [P, ctypes.c_int64, P]
@@ -279,3 +285,35 @@ def attention_multi(main: OracleRing, history_rings, q, q_pos0: int, n_current: 
                                     float(cache_bias), float(softmax_scale), int(bool(mode_b)),
                                     rp, n_rows, _p(out), _p(lse))
     return out, lse
+
+
+def key_mass(main: OracleRing, history_rings, q, q_pos0: int, n_current: int, ring_index: int,
+             ages, mask=(1 << 30, 1 << 30, 1 << 30, 1 << 30), cache_bias: float = 0.0,
+             softmax_scale: float | None = None) -> np.ndarray:
+    """Attention mass (sum over heads and query rows of the softmax probability) that the
+    history slots of ring ``ring_index`` at the given ages receive in the attention call
+    over ``main`` and ``history_rings`` (see ``orc_key_mass``)."""
+    rings = [main, *history_rings]
+    q = _f32(q)
+    n_q = q.shape[0]
+    if softmax_scale is None:
+        softmax_scale = float(np.float32(1.0 / np.sqrt(main.D)))
+    ages = np.ascontiguousarray(np.asarray(ages, dtype=np.int64))
+    out = np.zeros(ages.size, np.float64)
+    ptrs = (ctypes.c_void_p * len(rings))(*[ctypes.addressof(r._s) for r in rings])
+    qf, qb, kf, kb = (int(x) for x in mask)
+    lib().orc_key_mass(ctypes.cast(ptrs, ctypes.c_void_p), len(rings), _p(q), n_q, int(q_pos0),
+                       int(n_current), qf, qb, kf, kb, float(cache_bias), float(softmax_scale),
+                       int(ring_index), _p(ages), ages.size, _p(out))
+    return out
+
+
+def memory_select(quality, frame, pos, M: int, gamma: float = 0.5) -> np.ndarray:
+    """Indices (ascending) of the candidates kept by the top-M rule with temporal
+    diversity (see ``orc_memory_select``)."""
+    qv = np.ascontiguousarray(np.asarray(quality, dtype=np.float64))
+    fr = np.ascontiguousarray(np.asarray(frame, dtype=np.int64))
+    ps = np.ascontiguousarray(np.asarray(pos, dtype=np.int64))
+    kept = np.zeros(max(1, qv.size), np.int32)
+    m = lib().orc_memory_select(_p(qv), _p(fr), _p(ps), qv.size, int(M), float(gamma), _p(kept))
+    return kept[:m].copy()
