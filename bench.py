@@ -194,10 +194,10 @@ class RunwayStep:
             for r, ring in enumerate(self.rings):
                 if "write" in parts:
                     kv.kv_ring_write(ring, self.k[r][p], self.v[r][p], commit=(p == PASSES - 1))
-                if "attn" in parts or "attn_b" in parts:
+                if "attn" in parts or "attn_b" in parts or "attn_pv8" in parts:
                     kv.chunk_attention(ring, self.q[r][p], self._q_pos(ring, p, parts), n,
                                        self.mask, 0.0, out=self.out[r], want_lse=False,
-                                       mode_b="attn_b" in parts)
+                                       mode_b="attn_b" in parts, pv_fp8="attn_pv8" in parts)
 
     def _q_pos(self, ring, p, parts):
         # the new chunk starts at next_pos while pending, and at next_pos - n once committed
@@ -607,6 +607,7 @@ def main():
     g_full = step.graph(("write", "attn"))
     g_attn = step.graph(("attn",))
     g_attn_b = step.graph(("attn_b",))     # mode B (e4m3 query), reported beside mode A
+    g_attn_8 = step.graph(("attn_pv8",))   # e4m3 P.V, reported beside mode A
     g_write = step.graph(("write",))
 
     def barrier():
@@ -631,11 +632,13 @@ def main():
     # per-kernel averages: the same launches, split into attention-only / write-only graphs
     ms_attn = timed(torch, g_attn.replay, args.steps, stream) / (R * PASSES)
     ms_attn_b = timed(torch, g_attn_b.replay, args.steps, stream) / (R * PASSES)
+    ms_attn_8 = timed(torch, g_attn_8.replay, args.steps, stream) / (R * PASSES)
     ms_write = timed(torch, g_write.replay, args.steps, stream) / (R * PASSES)
     clk = clocks.stop()
     ms_step = max_over_ranks(torch, dist, ms_step)
     ms_attn = max_over_ranks(torch, dist, ms_attn)
     ms_attn_b = max_over_ranks(torch, dist, ms_attn_b)
+    ms_attn_8 = max_over_ranks(torch, dist, ms_attn_8)
     ms_write = max_over_ranks(torch, dist, ms_write)
     if args.no_extras:
         rot = {"us_per_launch": float("nan"), "bytes_per_launch": 0}
@@ -650,7 +653,7 @@ def main():
     rot_us = max_over_ranks(torch, dist, rot["us_per_launch"])
     e2e_ms = max_over_ranks(torch, dist, e2e["ms_per_step"])
     timeouts = kv.kv_wait_timeout_count()
-    del g_full, g_attn, g_attn_b, g_write
+    del g_full, g_attn, g_attn_b, g_attn_8, g_write
 
     w = inputs.RUNWAY
     value = ms_step * 1e3 / (R * PASSES)              # us per call (each rank: R*4 calls)
@@ -686,6 +689,11 @@ def main():
             "frac_bf16_sustained": flop / (ms_attn_b * 1e-3) / 1e12 / peaks["bf16_sus"],
             "note": "KV_QK_FP8: query quantised to e4m3 per row, one e4m3 MMA set for Q.K^T; "
                     "matches the definition on the quantised query, not the headline"},
+        "attention_pv_fp8": {
+            "us_per_call": ms_attn_8 * 1e3, "tflops": flop / (ms_attn_8 * 1e-3) / 1e12,
+            "frac_bf16_sustained": flop / (ms_attn_8 * 1e-3) / 1e12 / peaks["bf16_sus"],
+            "note": "KV_PV_FP8: P rounded to e4m3, P.V on the raw V codes; its error against "
+                    "the oracle is reported by the tests, not held to the tolerance"},
         "write": {"us_per_call": ms_write * 1e3, "bytes_per_call": wbytes, "gbs": write_gbs,
                   "frac_hbm": write_gbs / peaks["hbm"]},
         "rotate": {"shape": "32768 slots x 40 heads x 128", "us_per_launch": rot_us,

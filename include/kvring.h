@@ -85,6 +85,13 @@ extern "C" {
                                  also quantised to e4m3 by the write's row rule (one fp32
                                  scale per row) and Q.K^T runs as one e4m3 MMA set instead
                                  of the exact hi + lo pair; head_dim 128 only */
+#define KV_PV_FP8 2u          /* chunk_attention*: the fast, less exact P.V -- P (times the
+                                 key's V scale) is rounded to e4m3 (2^-4 relative) and P.V
+                                 runs as e4m3 MMAs on the raw V codes.  Its error against
+                                 the definition is measured and reported, not bounded by
+                                 the acceptance tolerance ("KREA Real-Time 14B /
+                                 video-conductor", "What didn't": FP8 by default cost
+                                 quality); head_dim 128 only */
 
 /* Per-stream ring-head state.  Plain data: the caller fills the shape, the device
  * pointers, the RoPE table fields and next_pos, then calls kv_ring_init.  Copying the
@@ -214,10 +221,11 @@ KV_API int kv_ring_delta_rotate(kv_ring_t* kv, int64_t delta, void* stream);
  * chunk (masked by `mask`, no bias), the rest are history (bias added, always visible).
  * out: device bf16 [n_q][H][D]; lse: device fp32 [H][n_q] natural-log sum of exp, or
  * NULL.  A row with no visible key gets out = 0 and lse = -inf.  softmax_scale > 0.
- * flags: 0 (the query stays bf16: exact, "mode A") or KV_QK_FP8 (mode B; its result
- * matches the definition evaluated on the quantised-then-dequantised query).  Errors:
- * KV_EINVAL (also an unknown flag), KV_ERANGE (n_current > valid slots, a query position
- * outside the table), KV_EUNSUPPORTED (KV_QK_FP8 at head_dim 64), KV_ESTATE, KV_ECUDA. */
+ * flags: 0 (the query stays bf16: exact, "mode A"), KV_QK_FP8 (mode B; its result
+ * matches the definition evaluated on the quantised-then-dequantised query) and/or
+ * KV_PV_FP8 (e4m3 P.V, see above).  Errors: KV_EINVAL (also an unknown flag), KV_ERANGE
+ * (n_current > valid slots, a query position outside the table), KV_EUNSUPPORTED
+ * (KV_QK_FP8 or KV_PV_FP8 at head_dim 64), KV_ESTATE, KV_ECUDA. */
 KV_API int chunk_attention(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
                     int n_current, const kv_block_mask_t* mask, const kv_cache_bias_t* bias,
                     float softmax_scale, void* out, float* lse, uint32_t flags, void* stream);
@@ -322,6 +330,57 @@ KV_API int chunk_attention_split_noalloc(const kv_ring_t* kv, const void* q, int
                                          const kv_cache_bias_t* bias, float softmax_scale,
                                          void* out, float* lse, int n_splits, uint32_t flags,
                                          void* stream);
+
+/* ------------------------------------------------------------------ content memory
+ * "Stream LTX", Inference: the long-context cache is an anchor, a content memory and a
+ * FIFO of recent blocks; each layer scores its own keys on attention quality and temporal
+ * diversity and evicts down to a top-M budget.  Here the FIFO is the stream's ring, the
+ * anchor and the content memory are history-only rings read by chunk_attention_multi, and
+ * the two calls below score and select.  The pages give no formula; the reading:
+ *   quality of a key = the softmax probability it receives in the newest chunk's
+ *     attention call, summed over heads and query rows (chunk_key_mass);
+ *   diversity: the k-th best key of a frame (frame = floor(slot position / frame_len))
+ *     scores quality * gamma^k; the budget keeps the best M (kv_memory_select). */
+
+/* Attention mass of n_cand slots of cand_ring, the slots (slot_first + c) mod capacity,
+ * c < n_cand: mass[h * n_cand + c] = sum over query rows i of exp(s_ihc - lse[h * n_q + i])
+ * with s the call's score (softmax_scale * <q~_i, k~_c> + history bias), q~ rotated from
+ * main_ring's RoPE table at q_pos0 + i.  q, n_q, q_pos0, bias and softmax_scale must be
+ * those of the attention call whose lse [H][n_q] (device, natural log) is passed; the
+ * slots must be history keys of that call (always visible, bias added).  Rows whose lse
+ * is not finite add nothing.  mass: device fp32 [H][n_cand].  head_dim 128; both rings
+ * initialised with equal n_heads, head_dim and rope_base.  Errors: KV_EINVAL (null or
+ * misaligned pointers, rings that differ, n_cand < 0 or > capacity, slot_first outside
+ * [0, capacity), softmax_scale), KV_ERANGE (a query position outside main_ring's table),
+ * KV_EUNSUPPORTED (head_dim 64), KV_ESTATE, KV_ECUDA. */
+KV_API int chunk_key_mass(const kv_ring_t* main_ring, const kv_ring_t* cand_ring, const void* q,
+                          int n_q, int64_t q_pos0, const float* lse,
+                          const kv_cache_bias_t* bias, float softmax_scale,
+                          int64_t slot_first, int n_cand, float* mass, void* stream);
+
+/* Largest candidate count (memory slots + FIFO block) of one kv_memory_select call. */
+#define KV_MEMORY_MAX_CANDIDATES 8192
+
+/* Content-memory eviction: the candidates are the valid slots of `memory` (oldest first;
+ * memory may be NULL for none) and the n_fifo slots (fifo_slot_first + c) mod capacity of
+ * `fifo` (the block that the FIFO's next write overwrites), with their masses from
+ * chunk_key_mass (device [H][n_mem] and [H][n_fifo]).  quality = sum over heads of the
+ * masses (binary32, heads in order); frame = floor(slot_pos / frame_len); the k-th best
+ * key of a frame (quality descending, ties toward the lower position, then the lower
+ * candidate index) scores quality * gamma^k (binary32); the best min(n, budget) are kept.
+ * kept: device int32 workspace of at least min(n_mem + n_fifo, budget) entries; it
+ * receives the kept candidate indices (memory slots first, then the FIFO block), in
+ * ascending order.  Their K and V codes, scales and positions are copied into slots
+ * 0 .. kept - 1 of memory_out (a different ring with the same n_heads and head_dim and
+ * capacity >= budget), whose state becomes write_slot = kept mod capacity, live = kept,
+ * pending = 0 (next_pos unchanged).  Errors: KV_EINVAL (null or aligned pointers,
+ * budget < 1, frame_len < 1, gamma outside (0, 1], memory_out aliasing memory or fifo,
+ * rings that differ), KV_ERANGE (more than KV_MEMORY_MAX_CANDIDATES candidates,
+ * memory_out too small, n_fifo outside [0, capacity]), KV_ESTATE, KV_ECUDA. */
+KV_API int kv_memory_select(const kv_ring_t* memory, const float* mass_memory,
+                            const kv_ring_t* fifo, const float* mass_fifo,
+                            int64_t fifo_slot_first, int n_fifo, int budget, int64_t frame_len,
+                            float gamma, kv_ring_t* memory_out, int32_t* kept, void* stream);
 
 /* Static description of a status code.  Never NULL. */
 KV_API const char* kv_status_string(int status);

@@ -26,12 +26,15 @@ KV_OK, KV_EINVAL, KV_ERANGE, KV_EUNSUPPORTED, KV_ECUDA, KV_ESTATE = 0, -1, -2, -
 KV_DTYPE_BF16, KV_DTYPE_FP32 = 1, 2
 KV_COMMIT = 1
 KV_QK_FP8 = 1
+KV_PV_FP8 = 2
 
 EXPORTS = ("kv_rope_table_build", "kv_rope3d_table_build", "kv_ring_init", "kv_ring_write", "kv_ring_commit",
            "kv_ring_delta_rotate", "chunk_attention", "chunk_attention_workspace_size",
            "chunk_attention_split", "chunk_attention_split_noalloc", "chunk_attention_multi",
-           "chunk_attention_rows", "kv_status_string", "kv_wait_timeout_count")
+           "chunk_attention_rows", "chunk_key_mass", "kv_memory_select", "kv_status_string",
+           "kv_wait_timeout_count")
 KV_NOALLOC_SCRATCH_BYTES = 16 << 20
+KV_MEMORY_MAX_CANDIDATES = 8192
 KV_MAX_RINGS = 8
 
 
@@ -88,6 +91,8 @@ def lib() -> ctypes.CDLL:
                                       ctypes.c_uint32, P]
         L.chunk_attention_rows.argtypes = [P, P, I, I64, I, P, I, P, P, ctypes.c_float, P, P,
                                            ctypes.c_uint32, P]
+        L.chunk_key_mass.argtypes = [P, P, P, I, I64, P, P, ctypes.c_float, I64, I, P, P]
+        L.kv_memory_select.argtypes = [P, P, P, P, I64, I, I, I64, ctypes.c_float, P, P, P]
         L.kv_status_string.argtypes = [I]
         L.kv_status_string.restype = ctypes.c_char_p
         L.kv_wait_timeout_count.argtypes = [P]
@@ -216,9 +221,14 @@ def kv_ring_delta_rotate(ring: KvRing, delta: int, stream=None) -> None:
            "kv_ring_delta_rotate")
 
 
+def _flags(mode_b: bool, pv_fp8: bool) -> int:
+    return (KV_QK_FP8 if mode_b else 0) | (KV_PV_FP8 if pv_fp8 else 0)
+
+
 def chunk_attention(ring: KvRing, q, q_pos0: int, n_current: int, mask=None,
                     cache_bias: float = 0.0, softmax_scale: float | None = None, out=None,
-                    lse=None, want_lse: bool = True, stream=None, mode_b: bool = False):
+                    lse=None, want_lse: bool = True, stream=None, mode_b: bool = False,
+                    pv_fp8: bool = False):
     """q: bf16 [n_q][H][D] on the GPU.  mask: (q_first, q_block, k_first, k_block) or None.
     Returns (out bf16 [n_q][H][D], lse fp32 [H][n_q] or None)."""
     import torch
@@ -237,7 +247,7 @@ def chunk_attention(ring: KvRing, q, q_pos0: int, n_current: int, mask=None,
                                  None if m is None else ctypes.byref(m), ctypes.byref(b),
                                  float(softmax_scale), _ptr(out),
                                  None if lse is None else _ptr(lse),
-                                 KV_QK_FP8 if mode_b else 0, _stream(stream)),
+                                 _flags(mode_b, pv_fp8), _stream(stream)),
            "chunk_attention")
     return out, lse
 
@@ -280,7 +290,8 @@ def chunk_attention_workspace_size(n_q: int, n_heads: int, head_dim: int, n_spli
 def chunk_attention_split(ring: KvRing, q, q_pos0: int, n_current: int, n_splits: int,
                           workspace, mask=None, cache_bias: float = 0.0,
                           softmax_scale: float | None = None, out=None, lse=None,
-                          want_lse: bool = True, stream=None, mode_b: bool = False):
+                          want_lse: bool = True, stream=None, mode_b: bool = False,
+                          pv_fp8: bool = False):
     """chunk_attention with the keys split over n_splits groups; `workspace` is a device
     tensor of at least chunk_attention_workspace_size(...) bytes."""
     import torch
@@ -300,7 +311,7 @@ def chunk_attention_split(ring: KvRing, q, q_pos0: int, n_current: int, n_splits
                                        None if m is None else ctypes.byref(m), ctypes.byref(b),
                                        float(softmax_scale), _ptr(out),
                                        None if lse is None else _ptr(lse), int(n_splits),
-                                       _ptr(workspace), nbytes, KV_QK_FP8 if mode_b else 0,
+                                       _ptr(workspace), nbytes, _flags(mode_b, pv_fp8),
                                        _stream(stream)),
            "chunk_attention_split")
     return out, lse
@@ -373,3 +384,44 @@ def kv_wait_timeout_count() -> int:
     v = ctypes.c_uint32(0)
     _check(lib().kv_wait_timeout_count(ctypes.byref(v)), "kv_wait_timeout_count")
     return int(v.value)
+
+
+def chunk_key_mass(main: KvRing, cand: KvRing, q, q_pos0: int, lse, slot_first: int,
+                   n_cand: int, cache_bias: float = 0.0, softmax_scale: float | None = None,
+                   mass=None, stream=None):
+    """Attention mass [H][n_cand] (fp32, device) that slots (slot_first + c) mod C of
+    `cand` receive in the attention call with these q, q_pos0, bias and its lse [H][n_q]."""
+    import torch
+    assert q.is_cuda and q.dtype == torch.bfloat16 and q.is_contiguous()
+    assert lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous()
+    n_q = int(q.shape[0])
+    if mass is None:
+        mass = torch.empty((main.H, int(n_cand)), dtype=torch.float32, device=q.device)
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(main.D)
+    b = kv_cache_bias_t(float(cache_bias))
+    _check(lib().chunk_key_mass(main.ref, cand.ref, _ptr(q), n_q, int(q_pos0), _ptr(lse),
+                                ctypes.byref(b), float(softmax_scale), int(slot_first),
+                                int(n_cand), _ptr(mass), _stream(stream)),
+           "chunk_key_mass")
+    return mass
+
+
+def kv_memory_select(memory, mass_memory, fifo: KvRing, mass_fifo, fifo_slot_first: int,
+                     n_fifo: int, budget: int, frame_len: int, memory_out: KvRing,
+                     gamma: float = 0.5, kept=None, stream=None):
+    """Keep the best min(n, budget) of the memory's valid slots and the FIFO block by the
+    temporal-diversity rule; copy them into memory_out's slots 0 .. kept - 1.  Returns the
+    kept candidate indices (device int32, ascending)."""
+    import torch
+    n_mem = 0 if memory is None else memory.n_valid
+    m = min(n_mem + int(n_fifo), int(budget))
+    if kept is None:
+        kept = torch.empty((max(1, m),), dtype=torch.int32, device=fifo.k_codes.device)
+    _check(lib().kv_memory_select(None if memory is None else memory.ref,
+                                  None if mass_memory is None else _ptr(mass_memory), fifo.ref,
+                                  None if mass_fifo is None else _ptr(mass_fifo),
+                                  int(fifo_slot_first), int(n_fifo), int(budget), int(frame_len),
+                                  float(gamma), memory_out.ref, _ptr(kept), _stream(stream)),
+           "kv_memory_select")
+    return kept[:m]

@@ -12,7 +12,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libkvring.so")
-SOURCES = ["kvring_api.cu", "kv_write.cu", "kv_rotate.cu", "chunk_attn.cu", "chunk_attn_sm100.cu"]
+SOURCES = ["kvring_api.cu", "kv_write.cu", "kv_rotate.cu", "chunk_attn.cu", "chunk_attn_sm100.cu",
+           "key_mass.cu"]
 HEADERS = ["common.cuh", "internal.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

@@ -96,7 +96,7 @@ struct Layout {
   static constexpr uint32_t info = vh + NB * 2 * kVPanel;      // NI x Info
   static constexpr uint32_t rows = info + NI * sizeof(Info);    // int gi[256], float rowmul[256]
   static constexpr uint32_t bars = rows + 2 * BM * 4;           // mbarriers
-  static constexpr int kNumBars = 2 * NK + 2 * NV + 2 * NB + 2 * NI + 4 + 4 + 1;
+  static constexpr int kNumBars = 2 * NK + 2 * NV + 2 * NB + 2 * NI + 4 + 4 + 1 + NV;
   static constexpr uint32_t misc = bars + 8 * kNumBars;         // tmem addr, abort flag, G
   static constexpr uint32_t bytes = misc + 16 + 1024;           // + alignment slack
 };
@@ -121,6 +121,8 @@ struct Bars {
   __device__ uint64_t* sfull(int g, int buf) { return b + 2 * (NK + NV + NB + NI) + 2 * g + buf; }
   __device__ uint64_t* pfull(int g, int buf) { return b + 2 * (NK + NV + NB + NI) + 4 + 2 * g + buf; }
   __device__ uint64_t* ofinal() { return b + 2 * (NK + NV + NB + NI) + 8; }
+  // e4m3-P mode: V code stage s checked (rows of invalid slots zeroed) for the MMAs
+  __device__ uint64_t* vready(int s) { return b + 2 * (NK + NV + NB + NI) + 9 + s; }
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -273,9 +275,15 @@ __device__ __forceinline__ float q_quant16(const float (&y)[16], float amax, uin
   return div_rn(amax, 448.f);
 }
 
+// kPv8 (KV_PV_FP8): P is quantised to e4m3 as P'' = e4m3(p * vs / G * 2^8) with an exact
+// running maximum (p <= 1), and P''.V runs as kind::f8f6f4 MMAs that read the V codes
+// straight from their TMA stage (an MN-major e4m3 operand): no converter work, half the
+// tensor time of the f16 product, and e4m3's 2^-4 relative rounding on every P element.
+template <bool kPv8>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_attn_sm100_kernel(const __grid_constant__ CUtensorMap tmk,
                             const __grid_constant__ CUtensorMap tmv, const AttnArgs a) {
+  constexpr float kThr = kPv8 ? 0.f : kRescaleLog2;   // lazy-maximum threshold (log2)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -309,7 +317,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid == 32) {
     for (int s = 0; s < NK; ++s) { mbar_init(bars.kfull(s), 1); mbar_init(bars.kempty(s), 1); }
-    for (int s = 0; s < NV; ++s) { mbar_init(bars.vfull(s), 1); mbar_init(bars.vempty(s), kConvThreads); }
+    for (int s = 0; s < NV; ++s) {
+      mbar_init(bars.vfull(s), 1);
+      mbar_init(bars.vempty(s), kPv8 ? 1 : kConvThreads);  // released by the MMAs (kPv8)
+    }
     for (int s = 0; s < NB; ++s) { mbar_init(bars.vhfull(s), kConvThreads); mbar_init(bars.vhempty(s), 1); }
     for (int s = 0; s < NI; ++s) { mbar_init(bars.ifull(s), 32); mbar_init(bars.iempty(s), 256); }
     for (int g = 0; g < 2; ++g) {
@@ -319,6 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bars.pfull(g, 1), 128);
     }
     mbar_init(bars.ofinal(), 1);
+    for (int s = 0; s < NV; ++s) mbar_init(bars.vready(s), kConvThreads);
     *abort_flag = 0;
     *vmax_bits = 0u;
     *n_issued = 0;
@@ -424,7 +436,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   // mx < 2^(b - 126) for biased exponent b; b clamped so that G and 1/G are normal
   const int gexp = max(1, min(252, (int)((*vmax_bits >> 23) & 0xFFu)));
-  const float vnorm = __uint_as_float((uint32_t)(gexp + 1) << 23);        // G
+  // G (times 2^-8 for kPv8, whose P carries 2^8)
+  const float vnorm = __uint_as_float((uint32_t)(gexp + 1 - (kPv8 ? 8 : 0)) << 23);
   const float vnorm_inv = __uint_as_float((uint32_t)(253 - gexp) << 23);  // 1 / G
 
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -486,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int age = slot_age(slot, newest, C);
           if (age < n_valid) {
             ksv = pks[e] * a.score_scale_log2;
-            wv = pvs[e] * vnorm_inv;
+            wv = pvs[e] * vnorm_inv * (kPv8 ? 256.f : 1.f);   // exact: powers of two
             if (age < a.n_current) {
               kbv = 0.f;
               tok = a.n_current - 1 - age;
@@ -512,11 +525,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_e4m3_f32(128, BN);
       constexpr uint32_t idO = idesc_f16_f32(128, D, 0, 1);
+      constexpr uint32_t idO8 = idesc_e4m3_f32(128, D, 1);     // e4m3 P (TMEM) x V codes (MN)
       const uint32_t sQhi = smem_u32(sm + Layout::qhi), sQlo = smem_u32(sm + Layout::qlo);
       const uint32_t sK = smem_u32(sm + Layout::kbuf), sV = smem_u32(sm + Layout::vh);
       // descriptors are built once; a step of s bytes adds s >> 4 to the start field
       const uint64_t dQhi = smem_desc_sw128(sQhi, 16, 1024), dQlo = smem_desc_sw128(sQlo, 16, 1024);
       const uint64_t dK = smem_desc_sw128(sK, 16, 1024), dV = smem_desc_sw128(sV, kVPanel, 1024);
+      // V codes as the B operand: 64 key rows of 128 one-byte d values, 128-byte swizzled
+      // (one swizzle atom across d, 8-row groups 1024 bytes apart along the keys)
+      const uint64_t dVc = smem_desc_sw128(smem_u32(sm + Layout::vcode), kVPanel, 1024);
       const int n_halves = a.mode_b ? 1 : 2;       // hi and lo, or the one e4m3 operand
       // S_g(j) = Q_g K(j)^T into buffer j & 1 of tile g
       auto issue_s = [&](int gg, int jj) {
@@ -534,10 +551,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_pv = [&](int gg, int jj) {
         const uint32_t d = tmem + 256 + 128 * gg;
         const uint32_t p = tmem + 128 * gg + 64 * (jj & 1);
-        const uint64_t vd = dV + (((jj % NB) * 2 * kVPanel) >> 4);
+        if (kPv8) {
+          const uint64_t vd = dVc + (((jj % NV) * BN * D) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          tc_mma_f16_ts(d, p + 8 * kk, vd + 128 * kk, idO, (jj > 0) | (kk > 0));
+          for (int kk = 0; kk < BN / 32; ++kk)         // 32 keys = 8 columns = 32 code rows
+            tc_mma_f8_ts(d, p + 8 * kk, vd + 256 * kk, idO8, (jj > 0) | (kk > 0));
+        } else {
+          const uint64_t vd = dV + (((jj % NB) * 2 * kVPanel) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            tc_mma_f16_ts(d, p + 8 * kk, vd + 128 * kk, idO, (jj > 0) | (kk > 0));
+        }
       };
       bool ok = true;
       // S of the first two tiles for both query tiles
@@ -558,14 +582,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int gg = 0; gg < 2; ++gg) {
           const int j = jp[gg];
           if (j >= n_mine) continue;
-          if (!mbar_try_wait(bars.pfull(gg, j & 1), (j >> 1) & 1)) continue;
-          if (!mbar_try_wait(bars.vhfull(j % NB), (j / NB) & 1)) continue;
+          if (!mbar_test_wait(bars.pfull(gg, j & 1), (j >> 1) & 1)) continue;
+          if (kPv8 ? !mbar_test_wait(bars.vready(j % NV), (j / NV) & 1)
+                   : !mbar_test_wait(bars.vhfull(j % NB), (j / NB) & 1))
+            continue;
           const bool more = j + 2 < n_mine;
-          if (more && !mbar_try_wait(bars.kfull((j + 2) % NK), ((j + 2) / NK) & 1)) continue;
+          if (more && !mbar_test_wait(bars.kfull((j + 2) % NK), ((j + 2) / NK) & 1)) continue;
           tc_fence_after();
           issue_pv(gg, j);
           const bool second = jp[gg ^ 1] > j;       // the other tile is past j already
-          if (second) tc_commit(bars.vhempty(j % NB));
+          if (second) tc_commit(kPv8 ? bars.vempty(j % NV) : bars.vhempty(j % NB));
           if (more) {
             issue_s(gg, j + 2);
             if (second) tc_commit(bars.kempty((j + 2) % NK));
@@ -595,6 +621,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ V converters
     // 64 threads; thread ct owns key slot ct of every tile: its V row widened to f16
     // (exact) into the swizzled MN-major operand; rows of invalid slots become zero.
+    // e4m3-P mode: the MMAs read the V codes in place; thread ct only zeroes row ct of the
+    // stage when its slot is invalid (stale memory must not reach the MMA: 0 * NaN = NaN).
     const int ct = tid - 32 * kWarpConv;          // 0..63
     for (int j = 0; j < n_mine; ++j) {
       const int t = seq.tile(j0 + j);
@@ -602,8 +630,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool dead = !(slot < C && slot_age(slot, newest, C) < n_valid);
       const int sv = j % NV, b = j % NB;
       bool ok = wait(bars.vfull(sv), (j / NV) & 1);
-      ok = ok && (j < NB || wait(bars.vhempty(b), ((j / NB) - 1) & 1));
+      if (!kPv8) ok = ok && (j < NB || wait(bars.vhempty(b), ((j / NB) - 1) & 1));
       if (!named_bar_and(2, kConvThreads, ok)) break;
+      if (kPv8) {
+        if (dead) {
+          uint4* row = reinterpret_cast<uint4*>(sm + Layout::vcode + sv * BN * D + ct * 128);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) row[c] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bars.vready(sv));
+        continue;
+      }
       const uint8_t* vc = sm + Layout::vcode + sv * BN * D + ct * 128;
       uint8_t* vb = sm + Layout::vh + b * 2 * kVPanel;
 #pragma unroll
@@ -671,6 +709,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float off = a.bias_log2 - m_run;
         const uint64_t off2 = f2_pack(off, off);
         float m0 = -INFINITY, m1 = -INFINITY;
+        uint32_t p8[16];                               // kPv8: e4m3 P, four keys per word
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t pk[16];
@@ -695,14 +734,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             float a0, a1, a2, a3;
             f2_unpack(f2_mul(p01, f2_pack(ww.x, ww.y)), a0, a1);
             f2_unpack(f2_mul(p23, f2_pack(ww.z, ww.w)), a2, a3);
-            pk[2 * q8] = pack_f16x2(a0, a1);
-            pk[2 * q8 + 1] = pack_f16x2(a2, a3);
+            if (kPv8) {
+              p8[q] = e4m3x2(a0, a1) | (e4m3x2(a2, a3) << 16);
+            } else {
+              pk[2 * q8] = pack_f16x2(a0, a1);
+              pk[2 * q8 + 1] = pack_f16x2(a2, a3);
+            }
           }
           // P over S columns already read into registers; a recomputation overwrites it
-          tmem_st16(t_s + 16 * c, pk);
+          if (!kPv8) tmem_st16(t_s + 16 * c, pk);
         }
+        if (kPv8) tmem_st16(t_s, p8);
         const float mloc = fmaf(fmaxf(m0, m1), rowmul, a.bias_log2);
-        single = !__any_sync(0xffffffffu, mloc > m_run + kRescaleLog2);
+        single = !__any_sync(0xffffffffu, mloc > m_run + kThr);
       }
       if (!single) {
         // pass 1, in place: t = S * kscl (* r + bias later) for fast tiles, masked t for the
@@ -757,7 +801,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float mloc = special ? fmaxf(m0, m1) : fmaf(fmaxf(m0, m1), rowmul, a.bias_log2);
         // lazy reference maximum: move m only when the tile maximum exceeds it by more than
         // 2^8 (rows of a tile may differ; everything below is per row)
-        move = mloc > m_old + kRescaleLog2 || (m_old == -INFINITY && mloc > -INFINITY);
+        move = mloc > m_old + kThr || (m_old == -INFINITY && mloc > -INFINITY);
         if (move) m_run = mloc;
         const float mref = (m_run == -INFINITY) ? 0.f : m_run;
         // pass 2: p = 2^(t - m); P' = f16(p * w) over the S columns of tensor memory
@@ -766,6 +810,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t off2 = f2_pack(off, off);
         sum01 = f2_pack(0.f, 0.f);
         sum23 = sum01;
+        uint32_t p8[16];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t pk[16];
@@ -785,11 +830,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             float a0, a1, a2, a3;
             f2_unpack(f2_mul(p01, f2_pack(ww.x, ww.y)), a0, a1);
             f2_unpack(f2_mul(p23, f2_pack(ww.z, ww.w)), a2, a3);
-            pk[2 * q8] = pack_f16x2(a0, a1);
-            pk[2 * q8 + 1] = pack_f16x2(a2, a3);
+            if (kPv8) {
+              p8[q] = e4m3x2(a0, a1) | (e4m3x2(a2, a3) << 16);
+            } else {
+              pk[2 * q8] = pack_f16x2(a0, a1);
+              pk[2 * q8 + 1] = pack_f16x2(a2, a3);
+            }
           }
-          tmem_st16(t_s + 16 * c, pk);
+          if (!kPv8) tmem_st16(t_s + 16 * c, pk);
         }
+        if (kPv8) tmem_st16(t_s, p8);
       }
       float s0, s1, s2, s3;
       f2_unpack(sum01, s0, s1);
@@ -800,7 +850,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // rescale O_g once the previous P.V of this tile has landed (rare; warp-collective)
       if (__any_sync(0xffffffffu, scale_o)) {
         // P.V(j - 1) of both tiles has completed once V buffer (j - 1) is released
-        ok = wait(bars.vhempty((j - 1) % NB), ((j - 1) / NB) & 1);
+        ok = kPv8 ? wait(bars.vempty((j - 1) % NV), ((j - 1) / NV) & 1)
+                  : wait(bars.vhempty((j - 1) % NB), ((j - 1) / NB) & 1);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
 #pragma unroll 1
@@ -962,15 +1013,18 @@ int launch_split_combine(const AttnArgs& a, int D_, int n_splits, cudaStream_t s
 
 int launch_attention_sm100_d128(const AttnArgs& a, const void* tmap_k_sw128,
                                 const void* tmap_v_sw128, cudaStream_t s, int n_splits) {
-  static unsigned char configured[kMaxDevices] = {};
-  if (!smem_attr_set(reinterpret_cast<const void*>(chunk_attn_sm100_kernel), (int)Layout::bytes,
-                     configured))
-    return KV_ECUDA;
+  static unsigned char configured[2][kMaxDevices] = {};
+  const void* fn = a.pv_fp8 ? reinterpret_cast<const void*>(chunk_attn_sm100_kernel<true>)
+                            : reinterpret_cast<const void*>(chunk_attn_sm100_kernel<false>);
+  if (!smem_attr_set(fn, (int)Layout::bytes, configured[a.pv_fp8 ? 1 : 0])) return KV_ECUDA;
   CUtensorMap mk, mv;
   memcpy(&mk, tmap_k_sw128, sizeof(mk));
   memcpy(&mv, tmap_v_sw128, sizeof(mv));
   dim3 grid((a.n_rows + BM - 1) / BM, a.H, n_splits);
-  chunk_attn_sm100_kernel<<<grid, kThreads, Layout::bytes, s>>>(mk, mv, a);
+  if (a.pv_fp8)
+    chunk_attn_sm100_kernel<true><<<grid, kThreads, Layout::bytes, s>>>(mk, mv, a);
+  else
+    chunk_attn_sm100_kernel<false><<<grid, kThreads, Layout::bytes, s>>>(mk, mv, a);
   return cudaPeekAtLastError() == cudaSuccess ? KV_OK : KV_ECUDA;
 }
 

@@ -114,6 +114,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity (never suspends the thread, unlike
+// try_wait): for a thread that polls several barriers in turn.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Returns false after about a
 // second without completion (the event is counted in *timeouts, the library's device
 // counter, whose address the host passes in).
@@ -201,6 +215,18 @@ __device__ __forceinline__ void tc_mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, u
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::f8f6f4 (e4m3 A from tensor memory, four
+// consecutive K elements per 32-bit column; e4m3 B; f32 accumulate).
+__device__ __forceinline__ void tc_mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -429,10 +455,12 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, int a_mn_majo
          | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-// Instruction descriptor of kind::f8f6f4 with e4m3 A and B (both K-major), f32 D, M x N.
-__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+// Instruction descriptor of kind::f8f6f4 with e4m3 A and B, f32 D, M x N; A K-major, B
+// K-major (b_mn_major = 0) or MN-major (1, allowed for e4m3).
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, int b_mn_major = 0) {
   return (1u << 4)                        // D format f32
          | (0u << 7) | (0u << 10)         // A, B e4m3
+         | ((uint32_t)b_mn_major << 16)   // B major
          | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 

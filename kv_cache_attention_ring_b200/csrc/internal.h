@@ -47,6 +47,7 @@ struct AttnArgs {
   float bias_log2;          // history_bias * log2(e)
   unsigned int* timeouts;   // device counter of waits that gave up
   int mode_b;               // query quantised to e4m3 per row (one MMA set for Q.K^T)
+  int pv_fp8;               // P quantised to e4m3, P.V on the raw V codes (fast, less exact)
   // rows computed: the query indices rows[0 .. n_rows) (device int32), or 0 .. n_rows - 1
   // when rows is null (then n_rows = n_q); indices outside [0, n_q) are skipped
   const int32_t* rows;
@@ -56,6 +57,46 @@ struct AttnArgs {
   float* part_o;
   float* part_ml;
 };
+
+// Attention mass received by n_cand consecutive slots (from slot_first, mod C) of one
+// ring: mass [H][n_cand] (see key_mass.cu).
+struct KeyMassArgs {
+  const uint16_t* q;        // bf16 [n_q][H][D]
+  const float* rope_q0;     // main ring's table row of q_pos0
+  const float* lse;         // [H][n_q] natural log, from the attention call
+  const uint8_t* kc;        // candidate ring codes [H][C][D]
+  const float* ks;          // candidate ring scales [H][C]
+  float* mass;              // [H][n_cand]
+  int n_q, H, C, n_cand, slot_first;
+  float score_scale_log2;   // softmax_scale * log2(e)
+  float bias_log2;          // history_bias * log2(e)
+  unsigned int* timeouts;
+};
+
+// Top-M selection over a memory ring's slots and a FIFO block, and the gather of the kept
+// entries into a fresh ring (see key_mass.cu).
+struct SelectArgs {
+  const float* mass_mem;    // [H][n_mem]
+  const float* mass_fifo;   // [H][n_fifo]
+  const uint8_t *mem_kc, *mem_vc, *fifo_kc, *fifo_vc;
+  const float *mem_ks, *mem_vs, *fifo_ks, *fifo_vs;
+  const int32_t *mem_pos, *fifo_pos;
+  int n_mem, mem_slot_first, mem_C;
+  int n_fifo, fifo_slot_first, fifo_C;
+  int H, M;
+  long long frame_len;
+  float gamma;
+  int32_t* kept;            // [min(n_mem + n_fifo, M)] candidate indices, ascending
+  uint8_t *out_kc, *out_vc;
+  float *out_ks, *out_vs;
+  int32_t* out_pos;
+  int out_C;
+};
+
+int launch_key_mass(const KeyMassArgs& a, cudaStream_t s);
+int launch_memory_select(const SelectArgs& a, cudaStream_t s);
+// Shared memory of the selection for n candidates (n rounded up to a power of two).
+size_t select_smem_bytes(int n);
 
 // Largest device ordinal the per-device tables cover.
 constexpr int kMaxDevices = 64;

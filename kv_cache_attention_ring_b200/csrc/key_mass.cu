@@ -1,0 +1,380 @@
+// key_mass.cu -- attention mass received by history keys, and the content memory's top-M
+// selection ("Stream LTX", Inference: the long-context cache is an anchor, a content
+// memory and a FIFO of recent blocks; each layer scores its own keys on attention quality
+// and temporal diversity and evicts down to a top-M budget).
+//
+// key_mass_kernel: mass_h[h][c] = sum over query rows i of exp(s_ihc - lse_ih), the
+// probability head h of row i gives candidate key c in the attention call whose
+// log-sum-exp `lse` the caller passes.  One CTA takes 128 candidate keys of one head and
+// computes S^T = K Q^T on the tensor core (M = 128 keys, N = 128 queries per tile, the
+// query split exactly into e4m3 hi + lo as in the attention kernel), so every thread owns
+// one key as its tensor-memory lane and sums its own row: no cross-thread reduction.
+//
+// memory_select_kernel: one CTA ranks the candidates (quality = sum over heads of the
+// masses; the k-th best key of a frame scores quality * gamma^k; ties toward the lower
+// position, then the lower candidate index) and keeps the best M, written as a list of
+// source (ring, slot) in ascending candidate order.  memory_gather_kernel copies them
+// (K and V codes, scales, positions) into the new memory ring's slots 0 .. kept - 1.
+#include <cuda.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "../../include/kvring.h"
+
+namespace kvring {
+
+namespace {
+
+constexpr int D = 128;
+constexpr int KM = 128;          // candidate keys per CTA (tensor-memory lanes)
+constexpr int QN = 128;          // query rows per tile (MMA N)
+constexpr int kThreads = 128;
+
+struct MassLayout {
+  static constexpr uint32_t k = 0;                    // e4m3 [128 keys][128], sw128
+  static constexpr uint32_t qhi = k + KM * D;         // e4m3 [128 queries][128], sw128
+  static constexpr uint32_t qlo = qhi + QN * D;
+  static constexpr uint32_t rq = qlo + QN * D;        // per query: r (the split's power of two)
+  static constexpr uint32_t lq = rq + QN * 4;         // per query: lse * log2(e), or +inf
+  static constexpr uint32_t bar = lq + QN * 4;        // one mbarrier
+  static constexpr uint32_t misc = bar + 8;           // tmem address, abort flag
+  static constexpr uint32_t bytes = misc + 8 + 1024;  // + alignment slack
+};
+
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) key_mass_kernel(const KeyMassArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + MassLayout::bar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + MassLayout::misc);
+  float* rq = reinterpret_cast<float*>(sm + MassLayout::rq);
+  float* lq = reinterpret_cast<float*>(sm + MassLayout::lq);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int h = blockIdx.y;
+  const int c = blockIdx.x * KM + tid;                 // this thread's candidate
+  const bool live_c = c < a.n_cand;
+
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  if (tid == 32) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  // candidate key row: 8 16-byte chunks into the swizzled K-major operand (zero past the
+  // candidates); its scale times softmax_scale * log2(e)
+  float kscl = 0.f;
+  {
+    uint4 w[8];
+    if (live_c) {
+      int slot = a.slot_first + c;
+      slot = slot >= a.C ? slot - a.C : slot;
+      const uint4* src = reinterpret_cast<const uint4*>(a.kc + ((size_t)h * a.C + slot) * D);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[i] = __ldg(src + i);
+      kscl = __ldg(a.ks + (size_t)h * a.C + slot) * a.score_scale_log2;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      *reinterpret_cast<uint4*>(sm + MassLayout::k + tid * 128 + ((i ^ (tid & 7)) << 4)) = w[i];
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+  constexpr uint32_t idS = idesc_e4m3_f32(KM, QN);
+  const uint64_t dK = smem_desc_sw128(smem_u32(sm + MassLayout::k), 16, 1024);
+  const uint64_t dQhi = smem_desc_sw128(smem_u32(sm + MassLayout::qhi), 16, 1024);
+  const uint64_t dQlo = smem_desc_sw128(smem_u32(sm + MassLayout::qlo), 16, 1024);
+
+  float acc = 0.f;
+  bool ok = true;
+  const int lc = tid & 7;                              // prologue: 8 lanes per query row
+  int phase = 0;
+  for (int q0 = 0; q0 < a.n_q && ok; q0 += QN, phase ^= 1) {
+    // query tile: rotate, round to bf16, split exactly into e4m3 hi + lo (per-row power
+    // of two r), 16 rows per pass of the 128 threads
+    for (int rr = tid >> 3; rr < QN; rr += kThreads / 8) {
+      const int i = q0 + rr;
+      float y[16];
+      if (i < a.n_q) {
+        const uint4* qp = reinterpret_cast<const uint4*>(a.q + ((size_t)i * a.H + h) * D + 16 * lc);
+        const uint4 q0v = __ldg(qp), q1v = __ldg(qp + 1);
+        const float4* tb = reinterpret_cast<const float4*>(a.rope_q0 + (size_t)i * D + 16 * lc);
+        const uint32_t w[8] = {q0v.x, q0v.y, q0v.z, q0v.w, q1v.x, q1v.y, q1v.z, q1v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float4 cs = __ldg(tb + j);
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const uint32_t pr = w[2 * j + u];
+            const float c = u ? cs.z : cs.x, s = u ? cs.w : cs.y;
+            const float x0 = bf16_bits_to_float(pr & 0xFFFFu), x1 = bf16_bits_to_float(pr >> 16);
+            const uint32_t b = pack_bf16x2(sub_rn(mul_rn(x0, c), mul_rn(x1, s)),
+                                           add_rn(mul_rn(x0, s), mul_rn(x1, c)));
+            y[4 * j + 2 * u] = bf16_bits_to_float(b & 0xFFFFu);
+            y[4 * j + 2 * u + 1] = bf16_bits_to_float(b >> 16);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) y[e] = 0.f;
+      }
+      float amax = 0.f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) amax = max_nan(amax, fabsf(y[e]));
+#pragma unroll
+      for (int off = 4; off > 0; off >>= 1) amax = max_nan(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      int k = 0;
+      if (amax > 0.f && amax <= 3.402823466e38f) {
+        int e;
+        const float m = frexpf(amax, &e);
+        k = max(-126, min(127, (e - 1) - 8 + (m > 0.875f ? 1 : 0)));
+      }
+      const float inv_r = ldexpf(1.f, -k);
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float x[4], lv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = y[4 * j + e] * inv_r;
+        const uint32_t h01 = e4m3x2(x[0], x[1]), h23 = e4m3x2(x[2], x[3]);
+        const float2 d01 = f16x2_to_float2(e4m3x2_to_f16x2((uint16_t)h01));
+        const float2 d23 = f16x2_to_float2(e4m3x2_to_f16x2((uint16_t)h23));
+        lv[0] = x[0] - d01.x;
+        lv[1] = x[1] - d01.y;
+        lv[2] = x[2] - d23.x;
+        lv[3] = x[3] - d23.y;
+        hw[j] = h01 | (h23 << 16);
+        lw[j] = e4m3x2(lv[0], lv[1]) | (e4m3x2(lv[2], lv[3]) << 16);
+      }
+      const uint32_t off = (uint32_t)rr * 128u + ((uint32_t)(lc ^ (rr & 7)) << 4);
+      *reinterpret_cast<uint4*>(sm + MassLayout::qhi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(sm + MassLayout::qlo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      if (lc == 0) {
+        // rows past n_q, rows that attended nothing (lse not finite): no contribution
+        const float l = i < a.n_q ? __ldg(a.lse + (size_t)h * a.n_q + i) : INFINITY;
+        const bool use = isfinite(l);
+        rq[rr] = use ? ldexpf(1.f, k) : 0.f;
+        lq[rr] = use ? l * 1.4426950408889634f : INFINITY;
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const uint64_t qd = hf == 0 ? dQhi : dQlo;
+#pragma unroll
+        for (int kk = 0; kk < D / 32; ++kk)
+          tc_mma_f8_ss(tmem, dK + 2 * kk, qd + 2 * kk, idS, (hf | kk) != 0);
+      }
+      tc_commit(bar);
+    }
+    ok = mbar_wait(bar, phase, a.timeouts);
+    tc_fence_after();
+    if (__all_sync(0xffffffffu, ok)) {
+#pragma unroll 1
+      for (int cb = 0; cb < QN; cb += 32) {
+        uint32_t sr[32];
+        tmem_ld32(tmem + lane_base + cb, sr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          // s' = S kscl r + bias - lse (log2 units); 2^-inf = 0 for unused rows
+          const float t = fmaf(__uint_as_float(sr[u]) * kscl, rq[cb + u], a.bias_log2) - lq[cb + u];
+          acc += ex2f(t);
+        }
+      }
+    }
+    tc_fence_before();
+    ok = __syncthreads_and(ok);
+    tc_fence_after();
+  }
+  if (!ok) {
+    mbar_wait(bar, phase ^ 1, a.timeouts);             // bounded: let an issued MMA land
+    acc = __uint_as_float(0x7FC00000u);
+  }
+  if (live_c) a.mass[(size_t)h * a.n_cand + c] = acc;
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// ------------------------------------------------------------------ selection
+constexpr int kSelThreads = 1024;
+
+// Candidates of a selection: quality, position, frame, index; kept in shared memory.
+struct Cand {
+  float q;
+  int idx;
+  long long pos;
+  long long frame;
+};
+
+// (frame asc, quality desc, position asc, index asc)
+__device__ __forceinline__ bool before_in_frame(const Cand& x, const Cand& y) {
+  if (x.frame != y.frame) return x.frame < y.frame;
+  if (x.q != y.q) return x.q > y.q;
+  if (x.pos != y.pos) return x.pos < y.pos;
+  return x.idx < y.idx;
+}
+// (score desc, position asc, index asc)
+__device__ __forceinline__ bool before_in_score(const Cand& x, const Cand& y) {
+  if (x.q != y.q) return x.q > y.q;
+  if (x.pos != y.pos) return x.pos < y.pos;
+  return x.idx < y.idx;
+}
+
+// In-place bitonic sort of n_pow2 entries (padding entries sort last), all threads.
+template <bool kByFrame>
+__device__ void bitonic(Cand* v, int n_pow2) {
+  for (int size = 2; size <= n_pow2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < n_pow2; i += blockDim.x) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool up = (i & size) == 0;
+          const bool swap = kByFrame ? (up ? before_in_frame(v[j], v[i]) : before_in_frame(v[i], v[j]))
+                                     : (up ? before_in_score(v[j], v[i]) : before_in_score(v[i], v[j]));
+          if (swap) {
+            const Cand t = v[i];
+            v[i] = v[j];
+            v[j] = t;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kSelThreads) memory_select_kernel(const SelectArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  Cand* v = reinterpret_cast<Cand*>(smem_raw);
+  const int n = a.n_mem + a.n_fifo;
+  int n_pow2 = 1;
+  while (n_pow2 < n) n_pow2 <<= 1;
+  for (int i = threadIdx.x; i < n_pow2; i += blockDim.x) {
+    Cand c;
+    if (i < n) {
+      const bool mem = i < a.n_mem;
+      const float* m = mem ? a.mass_mem : a.mass_fifo;
+      const int ci = mem ? i : i - a.n_mem;
+      const int nc = mem ? a.n_mem : a.n_fifo;
+      float q = 0.f;
+      for (int h = 0; h < a.H; ++h) q += m[(size_t)h * nc + ci];   // fixed order over heads
+      int slot = (mem ? a.mem_slot_first : a.fifo_slot_first) + ci;
+      const int C = mem ? a.mem_C : a.fifo_C;
+      slot = slot >= C ? slot - C : slot;
+      const long long pos = (mem ? a.mem_pos : a.fifo_pos)[slot];
+      c.q = q;
+      c.idx = i;
+      c.pos = pos;
+      c.frame = pos >= 0 ? pos / a.frame_len : -((-pos + a.frame_len - 1) / a.frame_len);
+    } else {
+      c.q = -INFINITY;                               // padding sorts last in both orders
+      c.idx = 0x7FFFFFFF;
+      c.pos = 0x7FFFFFFFFFFFFFFFll;
+      c.frame = 0x7FFFFFFFFFFFFFFFll;
+    }
+    v[i] = c;
+  }
+  __syncthreads();
+  bitonic<true>(v, n_pow2);
+  // rank within the frame: the k-th entry of a frame run scores quality * gamma^k
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    int first = i;
+    while (first > 0 && v[first - 1].frame == v[i].frame) --first;
+    float s = v[i].q;
+    for (int k = first; k < i; ++k) s *= a.gamma;
+    v[i].q = s;                                      // frames and positions stay as keys
+  }
+  __syncthreads();
+  bitonic<false>(v, n_pow2);
+  // the best min(n, M), listed in ascending candidate index
+  const int m = n < a.M ? n : a.M;
+  for (int i = threadIdx.x; i < m; i += blockDim.x) {
+    // position of v[i] among the kept in ascending idx order = count of kept with lower idx
+    int rank = 0;
+    for (int k = 0; k < m; ++k) rank += v[k].idx < v[i].idx;
+    a.kept[rank] = v[i].idx;
+  }
+}
+
+// Copy kept candidate r (source: memory ring slot or FIFO slot) into memory_out slot r.
+__global__ void __launch_bounds__(256) memory_gather_kernel(const SelectArgs a) {
+  const int r = blockIdx.x;                          // kept entry = destination slot
+  const int idx = a.kept[r];
+  const bool mem = idx < a.n_mem;
+  int slot = mem ? a.mem_slot_first + idx : a.fifo_slot_first + (idx - a.n_mem);
+  const int C = mem ? a.mem_C : a.fifo_C;
+  slot = slot >= C ? slot - C : slot;
+  const uint8_t* kc = mem ? a.mem_kc : a.fifo_kc;
+  const uint8_t* vc = mem ? a.mem_vc : a.fifo_vc;
+  const float* ks = mem ? a.mem_ks : a.fifo_ks;
+  const float* vs = mem ? a.mem_vs : a.fifo_vs;
+  // 8 lanes per (head, K or V) row of 128 bytes
+  for (int t = threadIdx.x; t < a.H * 2 * 8; t += blockDim.x) {
+    const int hh = t / 16, which = (t / 8) & 1, part = t & 7;
+    const uint8_t* src = (which ? vc : kc) + ((size_t)hh * C + slot) * D;
+    uint8_t* dst = (which ? a.out_vc : a.out_kc) + ((size_t)hh * a.out_C + r) * D;
+    reinterpret_cast<uint4*>(dst)[part] = reinterpret_cast<const uint4*>(src)[part];
+  }
+  for (int hh = threadIdx.x; hh < a.H; hh += blockDim.x) {
+    a.out_ks[(size_t)hh * a.out_C + r] = ks[(size_t)hh * C + slot];
+    a.out_vs[(size_t)hh * a.out_C + r] = vs[(size_t)hh * C + slot];
+  }
+  if (threadIdx.x == 0) a.out_pos[r] = (mem ? a.mem_pos : a.fifo_pos)[slot];
+}
+
+}  // namespace
+
+int launch_key_mass(const KeyMassArgs& a, cudaStream_t s) {
+  static unsigned char configured[kMaxDevices] = {};
+  if (!smem_attr_set(reinterpret_cast<const void*>(key_mass_kernel), (int)MassLayout::bytes,
+                     configured))
+    return KV_ECUDA;
+  const dim3 grid((unsigned)((a.n_cand + KM - 1) / KM), (unsigned)a.H);
+  key_mass_kernel<<<grid, kThreads, MassLayout::bytes, s>>>(a);
+  return cudaPeekAtLastError() == cudaSuccess ? KV_OK : KV_ECUDA;
+}
+
+size_t select_smem_bytes(int n) {
+  size_t p = 1;
+  while ((int)p < n) p <<= 1;
+  return p * sizeof(Cand);
+}
+
+int launch_memory_select(const SelectArgs& a, cudaStream_t s) {
+  const int n = a.n_mem + a.n_fifo;
+  const size_t bytes = select_smem_bytes(n);
+  static unsigned char configured[kMaxDevices] = {};
+  if (!smem_attr_set(reinterpret_cast<const void*>(memory_select_kernel), 232448, configured))
+    return KV_ECUDA;
+  memory_select_kernel<<<1, kSelThreads, bytes, s>>>(a);
+  if (cudaPeekAtLastError() != cudaSuccess) return KV_ECUDA;
+  const int m = n < a.M ? n : a.M;
+  if (m > 0) memory_gather_kernel<<<m, 256, 0, s>>>(a);
+  return cudaPeekAtLastError() == cudaSuccess ? KV_OK : KV_ECUDA;
+}
+
+}  // namespace kvring

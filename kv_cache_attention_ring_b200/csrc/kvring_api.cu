@@ -357,9 +357,9 @@ int attention_args(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0, 
                    float softmax_scale, void* out, float* lse, uint32_t flags, AttnArgs* a) {
   int rc = check_ring(kv);
   if (rc) return rc;
-  if (flags & ~KV_QK_FP8) return KV_EINVAL;
+  if (flags & ~(KV_QK_FP8 | KV_PV_FP8)) return KV_EINVAL;
   if (n_q < 0 || n_current < 0) return KV_EINVAL;
-  if ((flags & KV_QK_FP8) && kv->head_dim != 128) return KV_EUNSUPPORTED;
+  if ((flags & (KV_QK_FP8 | KV_PV_FP8)) && kv->head_dim != 128) return KV_EUNSUPPORTED;
   if (n_q == 0) return KV_OK;
   if (!q || !out || !aligned16(q) || !aligned16(out)) return KV_EINVAL;
   if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return KV_EINVAL;
@@ -399,6 +399,7 @@ int attention_args(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0, 
   a->part_o = nullptr;
   a->part_ml = nullptr;
   a->mode_b = (flags & KV_QK_FP8) ? 1 : 0;
+  a->pv_fp8 = (flags & KV_PV_FP8) ? 1 : 0;
   a->rows = nullptr;
   a->n_rows = n_q;
   return KV_OK;
@@ -544,6 +545,110 @@ int chunk_attention_multi(const kv_ring_t* const* rings, int n_rings, const void
   m.part_o = part_o;
   m.part_ml = part_ml;
   return launch_split_combine(m, D, S, s);
+}
+
+int chunk_key_mass(const kv_ring_t* main_ring, const kv_ring_t* cand_ring, const void* q,
+                   int n_q, int64_t q_pos0, const float* lse, const kv_cache_bias_t* bias,
+                   float softmax_scale, int64_t slot_first, int n_cand, float* mass,
+                   void* stream) {
+  int rc = check_ring(main_ring);
+  if (rc) return rc;
+  if ((rc = check_ring(cand_ring))) return rc;
+  if (main_ring->n_heads != cand_ring->n_heads || main_ring->head_dim != cand_ring->head_dim ||
+      main_ring->rope_base != cand_ring->rope_base)
+    return KV_EINVAL;
+  if (main_ring->head_dim != 128) return KV_EUNSUPPORTED;
+  if (n_q < 0 || n_cand < 0 || n_cand > cand_ring->capacity) return KV_EINVAL;
+  if (slot_first < 0 || slot_first >= cand_ring->capacity) return KV_EINVAL;
+  if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return KV_EINVAL;
+  const float b = bias ? bias->history_bias : 0.f;
+  if (isnan(b) || b == INFINITY) return KV_EINVAL;
+  if (n_q == 0 || n_cand == 0) return KV_OK;
+  if (!q || !lse || !mass || !aligned16(q) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(mass) & 3u))
+    return KV_EINVAL;
+  if (!in_table(main_ring, q_pos0, q_pos0 + n_q - 1)) return KV_ERANGE;
+  KeyMassArgs a;
+  a.q = static_cast<const uint16_t*>(q);
+  a.rope_q0 = main_ring->rope_table + (size_t)(q_pos0 - main_ring->rope_pos_min) * 128;
+  a.lse = lse;
+  a.kc = cand_ring->k_codes;
+  a.ks = cand_ring->k_scale;
+  a.mass = mass;
+  a.n_q = n_q;
+  a.H = main_ring->n_heads;
+  a.C = cand_ring->capacity;
+  a.n_cand = n_cand;
+  a.slot_first = (int)slot_first;
+  a.score_scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.bias_log2 = b * 1.4426950408889634f;
+  a.timeouts = timeout_counter();
+  if (!a.timeouts) return KV_ECUDA;
+  return launch_key_mass(a, static_cast<cudaStream_t>(stream));
+}
+
+int kv_memory_select(const kv_ring_t* memory, const float* mass_memory, const kv_ring_t* fifo,
+                     const float* mass_fifo, int64_t fifo_slot_first, int n_fifo, int budget,
+                     int64_t frame_len, float gamma, kv_ring_t* memory_out, int32_t* kept,
+                     void* stream) {
+  int rc = check_ring(fifo);
+  if (rc) return rc;
+  if ((rc = check_ring(memory_out))) return rc;
+  if (memory && (rc = check_ring(memory))) return rc;
+  if (memory_out == memory || memory_out == fifo) return KV_EINVAL;
+  if (memory_out->k_codes == fifo->k_codes || (memory && memory_out->k_codes == memory->k_codes))
+    return KV_EINVAL;
+  const kv_ring_t* others[2] = {memory, memory_out};
+  for (const kv_ring_t* r : others) {
+    if (r && (r->n_heads != fifo->n_heads || r->head_dim != fifo->head_dim)) return KV_EINVAL;
+  }
+  if (budget < 1 || frame_len < 1 || !(gamma > 0.f) || gamma > 1.f) return KV_EINVAL;
+  if (n_fifo < 0 || n_fifo > fifo->capacity) return KV_ERANGE;
+  if (fifo_slot_first < 0 || fifo_slot_first >= fifo->capacity) return KV_EINVAL;
+  if (budget > memory_out->capacity) return KV_ERANGE;
+  const int64_t n_mem = memory ? valid_slots(memory) : 0;
+  if (n_mem + n_fifo > KV_MEMORY_MAX_CANDIDATES) return KV_ERANGE;
+  if (!kept || (n_mem > 0 && !mass_memory) || (n_fifo > 0 && !mass_fifo)) return KV_EINVAL;
+  const int64_t m = n_mem + n_fifo < budget ? n_mem + n_fifo : budget;
+  SelectArgs a;
+  a.mass_mem = mass_memory;
+  a.mass_fifo = mass_fifo;
+  a.mem_kc = memory ? memory->k_codes : nullptr;
+  a.mem_vc = memory ? memory->v_codes : nullptr;
+  a.mem_ks = memory ? memory->k_scale : nullptr;
+  a.mem_vs = memory ? memory->v_scale : nullptr;
+  a.mem_pos = memory ? memory->slot_pos : nullptr;
+  a.mem_C = memory ? memory->capacity : 1;
+  a.n_mem = (int)n_mem;
+  a.mem_slot_first =
+      memory ? (int)mod_c(memory->write_slot + memory->pending - n_mem, memory->capacity) : 0;
+  a.fifo_kc = fifo->k_codes;
+  a.fifo_vc = fifo->v_codes;
+  a.fifo_ks = fifo->k_scale;
+  a.fifo_vs = fifo->v_scale;
+  a.fifo_pos = fifo->slot_pos;
+  a.fifo_C = fifo->capacity;
+  a.n_fifo = n_fifo;
+  a.fifo_slot_first = (int)fifo_slot_first;
+  a.H = fifo->n_heads;
+  a.M = budget;
+  a.frame_len = frame_len;
+  a.gamma = gamma;
+  a.kept = kept;
+  a.out_kc = memory_out->k_codes;
+  a.out_vc = memory_out->v_codes;
+  a.out_ks = memory_out->k_scale;
+  a.out_vs = memory_out->v_scale;
+  a.out_pos = memory_out->slot_pos;
+  a.out_C = memory_out->capacity;
+  if (m > 0) {
+    rc = launch_memory_select(a, static_cast<cudaStream_t>(stream));
+    if (rc) return rc;
+  }
+  memory_out->write_slot = mod_c(m, memory_out->capacity);
+  memory_out->live = m;
+  memory_out->pending = 0;
+  return KV_OK;
 }
 
 int kv_wait_timeout_count(uint32_t* host_count) {

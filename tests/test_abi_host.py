@@ -174,7 +174,8 @@ def test_attention_validation_before_launch(L):
     ok_args = (r, 16, 8, 0, 8, None, None, 0.125, 16, None)
     assert L.chunk_attention(*ok_args[:1], 16, 0, 0, 0, None, None, 0.125, 16, None, 0,
                              None) == kv.KV_OK                            # n_q = 0: no launch
-    assert L.chunk_attention(*ok_args, 2, None) == kv.KV_EINVAL           # unknown flag
+    assert L.chunk_attention(*ok_args, 4, None) == kv.KV_EINVAL           # unknown flag
+    assert L.chunk_attention(*ok_args, kv.KV_PV_FP8, None) == kv.KV_EUNSUPPORTED  # e4m3 P, D 64
     assert L.chunk_attention(*ok_args, kv.KV_QK_FP8, None) == kv.KV_EUNSUPPORTED  # mode B, D 64
     assert L.chunk_attention(r, 16, 8, 0, 65, None, None, 0.125, 16, None, 0,
                              None) == kv.KV_ERANGE                        # n_current > valid
@@ -206,11 +207,47 @@ def test_rows_validation_before_launch(L):
     assert call(n_q=0) == kv.KV_OK
     assert call(rows=None) == kv.KV_EINVAL
     assert call(rows=18) == kv.KV_EINVAL               # not 4-byte aligned
-    assert call(flags=2) == kv.KV_EINVAL
+    assert call(flags=4) == kv.KV_EINVAL
     s64 = _fake_ring(D=64)
     s64.live = 64
     assert call(ring=ctypes.byref(s64)) == kv.KV_EUNSUPPORTED
     assert call() == kv.KV_ECUDA                       # valid: reaches the device (none here)
+
+
+def test_content_memory_validation(L):
+    main, cand = _fake_ring(D=128), _fake_ring(C=64, D=128)
+    main.live, cand.live = 64, 64
+    rm, rc = ctypes.byref(main), ctypes.byref(cand)
+
+    def mass(n_q=8, slot_first=0, n_cand=16, scale=0.125, ring=rc, lse=16, m=16):
+        return L.chunk_key_mass(rm, ring, 16, n_q, 0, lse, None, scale, slot_first, n_cand, m,
+                                None)
+
+    assert mass(n_cand=0) == kv.KV_OK and mass(n_q=0) == kv.KV_OK     # nothing to do
+    assert mass(n_cand=65) == kv.KV_EINVAL
+    assert mass(slot_first=64) == kv.KV_EINVAL
+    assert mass(scale=0.0) == kv.KV_EINVAL
+    assert mass(lse=None) == kv.KV_EINVAL and mass(m=18) == kv.KV_EINVAL
+    wide = _fake_ring(C=64, H=4, D=128)
+    assert mass(ring=ctypes.byref(wide)) == kv.KV_EINVAL
+    assert mass() == kv.KV_ECUDA                                        # reaches the device
+    out = _fake_ring(C=32, D=128)
+    out.k_codes = 0x200000
+
+    def sel(memory=None, n_fifo=16, budget=32, frame=8, gamma=0.5, dst=None, kept=16):
+        return L.kv_memory_select(memory, 16, rc, 16, 0, n_fifo, budget, frame, gamma,
+                                  ctypes.byref(out) if dst is None else dst, kept, None)
+
+    assert sel(budget=0) == kv.KV_EINVAL and sel(frame=0) == kv.KV_EINVAL
+    assert sel(gamma=0.0) == kv.KV_EINVAL and sel(gamma=1.5) == kv.KV_EINVAL
+    assert sel(budget=33) == kv.KV_ERANGE                              # memory_out too small
+    assert sel(n_fifo=65) == kv.KV_ERANGE
+    assert sel(dst=rc) == kv.KV_EINVAL                                 # aliases the FIFO
+    assert sel(kept=None) == kv.KV_EINVAL
+    assert out.live == 0
+    big = _fake_ring(C=8192, D=128)
+    big.live = 8192
+    assert sel(memory=ctypes.byref(big)) == kv.KV_ERANGE               # > 8,192 candidates
 
 
 def test_split_workspace_size_and_validation(L):
@@ -273,7 +310,7 @@ def test_multi_ring_validation_before_launch(L):
     assert call(two, 2, ws=17) == kv.KV_EINVAL                          # misaligned
     assert call(two, 2, nbytes=need - 1) == kv.KV_ERANGE                # sized for 8 splits
     assert call(two, 2, n_current=65) == kv.KV_ERANGE                   # main ring: 64 valid
-    assert call(two, 2, flags=2) == kv.KV_EINVAL
+    assert call(two, 2, flags=4) == kv.KV_EINVAL
     wide = _fake_ring(C=64, H=4, D=128)
     assert call(arr(main, wide), 2) == kv.KV_EINVAL                     # heads differ
     other_base = _fake_ring(C=64, D=128)
