@@ -54,6 +54,9 @@ def parse_args():
                     help="rings per step (60 = the Runway step; fewer for profiler captures)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the rotate, end-to-end and CPU legs (profiler captures)")
+    ap.add_argument("--leg", choices=["all", "rotate"], default="all",
+                    help="rotate: time only the delta rotation of a full 32,768 x 40 ring "
+                         "(one JSON line; for profiler captures of that kernel)")
     return ap.parse_args()
 
 
@@ -601,6 +604,14 @@ def main():
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
     peaks = load_peaks()
+    if args.leg == "rotate":
+        rot = rotate_timing(torch, kv, inputs, dev, reps=max(3, args.steps))
+        rot["gbs"] = rot["bytes_per_launch"] / (rot["us_per_launch"] * 1e-6) / 1e9
+        rot["frac_hbm"] = rot["gbs"] / peaks["hbm"]
+        if rank == 0:
+            print(json.dumps({"leg": "rotate", "shape": "32768 slots x 40 heads x 128", **rot}),
+                  flush=True)
+        return
 
     step = RunwayStep(torch, kv, inputs, dev, seed=1000 + 2 + rank, rings=args.rings)
     R = args.rings
