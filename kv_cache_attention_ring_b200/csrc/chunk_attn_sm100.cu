@@ -29,10 +29,10 @@
 //    the first K/V tile loads.
 //  * Tensor memory (512 columns): tile g owns two S/P buffers of 64 columns,
 //    [128g, 128g+64) and [128g+64, 128g+128), and O_g = [256+128g, 384+128g).  The MMA
-//    issuer serves the two query tiles independently: as soon as P_g(j) is in tensor
-//    memory (and V(j) is widened) it runs P.V_g(j), then S_g(j+2) into the buffer P_g(j)
-//    occupied (tensor-core operations of one thread run in issue order).  A K stage and
-//    a V buffer are released by the second query tile to use them.
+//    issuer serves the two query tiles in lockstep: for key tile j it waits for P_0(j)
+//    (and V(j) widened), runs P.V_0(j) and S_0(j+2) into the buffer P_0(j) occupied,
+//    then does the same for tile 1 (tensor-core operations of one thread run in issue
+//    order).  Query tile 1 releases the K stage and the V buffer.
 //  * Warps: 0 producer (lane 0 issues the TMA loads of K and V codes; all lanes build the
 //    per-key info of each tile: scale, P factor, bias, mask token), 1 MMA issuer,
 //    2-3 V converters, 4-7 softmax of tile 0, 8-11 softmax of tile 1 (thread = query
@@ -67,8 +67,8 @@ constexpr int BM = 256;                 // query rows per CTA
 constexpr int BN = 64;                  // key slots per tile
 constexpr int NK = 4;                   // K code stages
 constexpr int NV = 4;                   // V code stages
-constexpr int NB = 3;                   // V f16 buffers
-constexpr int NI = 6;                   // per-key info stages
+constexpr int NB = 2;                   // V f16 buffers
+constexpr int NI = 4;                   // per-key info stages
 constexpr int kThreads = 12 * 32;
 constexpr int kWarpProd = 0, kWarpMma = 1, kWarpConv = 2, kWarpSoft = 4;
 constexpr int kConvThreads = 64;        // one converter thread per key slot of a tile
@@ -572,45 +572,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_s(1, jj);
         tc_commit(bars.kempty(jj % NK));           // both tiles have read K(jj)
       }
-      // then serve the two query tiles as their P tiles arrive: P.V_g(j), S_g(j + 2)
-      int jp[2] = {0, 0};
-      unsigned long long t_idle = 0;
-      uint32_t spins = 0;
-      while (ok && (jp[0] < n_mine || jp[1] < n_mine)) {
-        bool progressed = false;
-#pragma unroll
-        for (int gg = 0; gg < 2; ++gg) {
-          const int j = jp[gg];
-          if (j >= n_mine) continue;
-          if (!mbar_test_wait(bars.pfull(gg, j & 1), (j >> 1) & 1)) continue;
-          if (kPv8 ? !mbar_test_wait(bars.vready(j % NV), (j / NV) & 1)
-                   : !mbar_test_wait(bars.vhfull(j % NB), (j / NB) & 1))
-            continue;
+      // lockstep: per key tile j, query tile 0 then query tile 1, blocking waits
+      for (int j = 0; ok && j < n_mine; ++j) {
+        for (int gg = 0; gg < 2 && ok; ++gg) {
+          ok = wait(bars.pfull(gg, j & 1), (j >> 1) & 1) &&
+               (kPv8 ? wait(bars.vready(j % NV), (j / NV) & 1) : wait(bars.vhfull(j % NB), (j / NB) & 1));
           const bool more = j + 2 < n_mine;
-          if (more && !mbar_test_wait(bars.kfull((j + 2) % NK), ((j + 2) / NK) & 1)) continue;
+          if (ok && more) ok = wait(bars.kfull((j + 2) % NK), ((j + 2) / NK) & 1);
+          if (!ok) break;
           tc_fence_after();
           issue_pv(gg, j);
-          const bool second = jp[gg ^ 1] > j;       // the other tile is past j already
-          if (second) tc_commit(kPv8 ? bars.vempty(j % NV) : bars.vhempty(j % NB));
+          if (gg == 1) tc_commit(kPv8 ? bars.vempty(j % NV) : bars.vhempty(j % NB));
           if (more) {
             issue_s(gg, j + 2);
-            if (second) tc_commit(bars.kempty((j + 2) % NK));
-          }
-          jp[gg] = j + 1;
-          progressed = true;
-        }
-        if (progressed) {
-          spins = 0;
-        } else if ((++spins & 63u) == 0) {
-          // bounded: give up after about a second without progress
-          const unsigned long long now = global_ns();
-          if (spins == 64) t_idle = now;
-          if (*abort_flag) {
-            ok = false;
-          } else if (now - t_idle > kWaitLimitNs) {
-            atomicAdd(a.timeouts, 1u);
-            *abort_flag = 1;
-            ok = false;
+            if (gg == 1) tc_commit(bars.kempty((j + 2) % NK));
           }
         }
       }
