@@ -47,7 +47,8 @@
 //  * Split over keys (gridDim.z > 1): each CTA takes a contiguous share of the valid
 //    tiles and writes fp32 partials (O G, m, l); split_combine_kernel merges them.
 //  * Keys are visited in physical slot order; the ring wrap costs nothing (attention
-//    does not depend on key order once bias and mask are per key).
+//    does not depend on key order once bias and mask are per key).  A CTA skips the
+//    newest current-chunk keys that the block-causal mask hides from all of its rows.
 // Every mbarrier wait is bounded (about a second); on a timeout the CTA abandons the
 // work, writes NaN to its rows, waits (bounded again) for the copies and MMAs it has
 // issued, frees its tensor memory and exits.
@@ -302,8 +303,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int C = a.C;
   const int newest = (int)a.newest_slot, n_valid = (int)a.n_valid;
 
-  // this CTA's slice of the valid tiles (all of them unless split over keys)
-  const TileSeq seq(C, newest, n_valid);
+  // Keys this CTA visits: the valid slots, less the newest current-chunk keys that the
+  // block-causal mask hides from every one of its rows (the mask limit grows with the row
+  // index, so its last row decides; a row list can hold any index, so all are kept then).
+  int newest_v = newest, n_visit = n_valid;
+  if (!a.rows && a.n_current > 0) {
+    const int last = min(q0 + BM, min(a.n_rows, a.n_q)) - 1;
+    if (last >= 0) {
+      const int64_t qb = last < a.q_first ? 0 : 1 + (int64_t)(last - a.q_first) / a.q_block;
+      const int64_t l = (int64_t)a.k_first + qb * (int64_t)a.k_block;
+      const int hidden = a.n_current - (int)(l < (int64_t)a.n_current ? l : (int64_t)a.n_current);
+      n_visit = n_valid - hidden;
+      newest_v = newest - hidden;
+      if (newest_v < 0) newest_v += C;
+    }
+  }
+  // this CTA's slice of the visited tiles (all of them unless split over keys)
+  const TileSeq seq(C, newest_v, n_visit);
   int j0, n_mine;
   {
     const int per = (seq.count + (int)gridDim.z - 1) / (int)gridDim.z;
