@@ -280,7 +280,7 @@ __device__ __forceinline__ float q_quant16(const float (&y)[16], float amax, uin
 // running maximum (p <= 1), and P''.V runs as kind::f8f6f4 MMAs that read the V codes
 // straight from their TMA stage (an MN-major e4m3 operand): no converter work, half the
 // tensor time of the f16 product, and e4m3's 2^-4 relative rounding on every P element.
-template <bool kPv8>
+template <bool kPv8, bool kModeB>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_attn_sm100_kernel(const __grid_constant__ CUtensorMap tmk,
                             const __grid_constant__ CUtensorMap tmv, const AttnArgs a) {
@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // written for such a row).  Two rows per lane group in flight.
   {
     const int lc = tid % kRowLanes;
-    const bool mode_b = a.mode_b != 0;
+    constexpr bool mode_b = kModeB;
     for (int base = 0; base < BM; base += 2 * kRowsPerPass) {
       int gi[2], r[2];
       uint4 qr[2][2];
@@ -538,7 +538,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop and waits; one elected lane issues each tensor-core
+    // instruction (el_*), so every operand is warp-uniform.
+    {
       constexpr uint32_t idS = idesc_e4m3_f32(128, BN);
       constexpr uint32_t idO = idesc_f16_f32(128, D, 0, 1);
       constexpr uint32_t idO8 = idesc_e4m3_f32(128, D, 1);     // e4m3 P (TMEM) x V codes (MN)
@@ -550,18 +552,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       // V codes as the B operand: 64 key rows of 128 one-byte d values, 128-byte swizzled
       // (one swizzle atom across d, 8-row groups 1024 bytes apart along the keys)
       const uint64_t dVc = smem_desc_sw128(smem_u32(sm + Layout::vcode), kVPanel, 1024);
-      const int n_halves = a.mode_b ? 1 : 2;       // hi and lo, or the one e4m3 operand
+      constexpr int kHalves = kModeB ? 1 : 2;      // hi and lo, or the one e4m3 operand
       // S_g(j) = Q_g K(j)^T into buffer j & 1 of tile g
       auto issue_s = [&](int gg, int jj) {
         const uint32_t d = tmem + 128 * gg + 64 * (jj & 1);
         const uint64_t kd = dK + (((jj % NK) * BN * D) >> 4);
-        for (int hf = 0; hf < n_halves; ++hf) {
+#pragma unroll
+        for (int hf = 0; hf < kHalves; ++hf) {
           const uint64_t qd = (hf == 0 ? dQhi : dQlo) + ((gg * 128 * D) >> 4);
 #pragma unroll
           for (int kk = 0; kk < D / 32; ++kk)
-            tc_mma_f8_ss(d, qd + 2 * kk, kd + 2 * kk, idS, (hf | kk) != 0);
+            el_mma_f8_ss(d, qd + 2 * kk, kd + 2 * kk, idS, (hf | kk) != 0);
         }
-        tc_commit(bars.sfull(gg, jj & 1));
+        el_commit(bars.sfull(gg, jj & 1));
       };
       // O_g (+)= P_g(j) V(j) with P_g read from tensor memory (buffer j & 1)
       auto issue_pv = [&](int gg, int jj) {
@@ -571,42 +574,47 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t vd = dVc + (((jj % NV) * BN * D) >> 4);
 #pragma unroll
           for (int kk = 0; kk < BN / 32; ++kk)         // 32 keys = 8 columns = 32 code rows
-            tc_mma_f8_ts(d, p + 8 * kk, vd + 256 * kk, idO8, (jj > 0) | (kk > 0));
+            el_mma_f8_ts(d, p + 8 * kk, vd + 256 * kk, idO8, (jj > 0) | (kk > 0));
         } else {
           const uint64_t vd = dV + (((jj % NB) * 2 * kVPanel) >> 4);
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk)
-            tc_mma_f16_ts(d, p + 8 * kk, vd + 128 * kk, idO, (jj > 0) | (kk > 0));
+            el_mma_f16_ts(d, p + 8 * kk, vd + 128 * kk, idO, (jj > 0) | (kk > 0));
         }
+      };
+      auto wait_w = [&](uint64_t* bar, uint32_t parity) -> bool {
+        return mbar_wait_warp(bar, parity, abort_flag, a.timeouts);
       };
       bool ok = true;
       // S of the first two tiles for both query tiles
       for (int jj = 0; jj < 2 && jj < n_mine && ok; ++jj) {
-        if (!(ok = wait(bars.kfull(jj % NK), (jj / NK) & 1))) break;
+        if (!(ok = wait_w(bars.kfull(jj % NK), (jj / NK) & 1))) break;
         tc_fence_after();
         issue_s(0, jj);
         issue_s(1, jj);
-        tc_commit(bars.kempty(jj % NK));           // both tiles have read K(jj)
+        el_commit(bars.kempty(jj % NK));           // both tiles have read K(jj)
       }
       // lockstep: per key tile j, query tile 0 then query tile 1, blocking waits
       for (int j = 0; ok && j < n_mine; ++j) {
-        for (int gg = 0; gg < 2 && ok; ++gg) {
-          ok = wait(bars.pfull(gg, j & 1), (j >> 1) & 1) &&
-               (kPv8 ? wait(bars.vready(j % NV), (j / NV) & 1) : wait(bars.vhfull(j % NB), (j / NB) & 1));
-          const bool more = j + 2 < n_mine;
-          if (ok && more) ok = wait(bars.kfull((j + 2) % NK), ((j + 2) / NK) & 1);
+        const bool more = j + 2 < n_mine;
+#pragma unroll
+        for (int gg = 0; gg < 2; ++gg) {
+          ok = wait_w(bars.pfull(gg, j & 1), (j >> 1) & 1) &&
+               (kPv8 ? wait_w(bars.vready(j % NV), (j / NV) & 1)
+                     : wait_w(bars.vhfull(j % NB), (j / NB) & 1)) &&
+               (!more || wait_w(bars.kfull((j + 2) % NK), ((j + 2) / NK) & 1));
           if (!ok) break;
           tc_fence_after();
           issue_pv(gg, j);
-          if (gg == 1) tc_commit(kPv8 ? bars.vempty(j % NV) : bars.vhempty(j % NB));
+          if (gg == 1) el_commit(kPv8 ? bars.vempty(j % NV) : bars.vhempty(j % NB));
           if (more) {
             issue_s(gg, j + 2);
-            if (gg == 1) tc_commit(bars.kempty((j + 2) % NK));
+            if (gg == 1) el_commit(bars.kempty((j + 2) % NK));
           }
         }
       }
-      if (n_mine > 0) tc_commit(bars.ofinal());    // tracks every MMA issued above
-      else mbar_arrive(bars.ofinal());
+      if (n_mine > 0) el_commit(bars.ofinal());    // tracks every MMA issued above
+      else if (lane == 0) mbar_arrive(bars.ofinal());
     }
   } else if (warp < kWarpSoft) {
     // ------------------------------------------------------------ V converters
@@ -1004,18 +1012,22 @@ int launch_split_combine(const AttnArgs& a, int D_, int n_splits, cudaStream_t s
 
 int launch_attention_sm100_d128(const AttnArgs& a, const void* tmap_k_sw128,
                                 const void* tmap_v_sw128, cudaStream_t s, int n_splits) {
-  static unsigned char configured[2][kMaxDevices] = {};
-  const void* fn = a.pv_fp8 ? reinterpret_cast<const void*>(chunk_attn_sm100_kernel<true>)
-                            : reinterpret_cast<const void*>(chunk_attn_sm100_kernel<false>);
-  if (!smem_attr_set(fn, (int)Layout::bytes, configured[a.pv_fp8 ? 1 : 0])) return KV_ECUDA;
+  // one instance per (e4m3 P, mode B) pair
+  using Kernel = void (*)(const CUtensorMap, const CUtensorMap, const AttnArgs);
+  static const Kernel kernels[4] = {chunk_attn_sm100_kernel<false, false>,
+                                    chunk_attn_sm100_kernel<false, true>,
+                                    chunk_attn_sm100_kernel<true, false>,
+                                    chunk_attn_sm100_kernel<true, true>};
+  static unsigned char configured[4][kMaxDevices] = {};
+  const int which = (a.pv_fp8 ? 2 : 0) + (a.mode_b ? 1 : 0);
+  const Kernel fn = kernels[which];
+  if (!smem_attr_set(reinterpret_cast<const void*>(fn), (int)Layout::bytes, configured[which]))
+    return KV_ECUDA;
   CUtensorMap mk, mv;
   memcpy(&mk, tmap_k_sw128, sizeof(mk));
   memcpy(&mv, tmap_v_sw128, sizeof(mv));
   dim3 grid((a.n_rows + BM - 1) / BM, a.H, n_splits);
-  if (a.pv_fp8)
-    chunk_attn_sm100_kernel<true><<<grid, kThreads, Layout::bytes, s>>>(mk, mv, a);
-  else
-    chunk_attn_sm100_kernel<false><<<grid, kThreads, Layout::bytes, s>>>(mk, mv, a);
+  fn<<<grid, kThreads, Layout::bytes, s>>>(mk, mv, a);
   return cudaPeekAtLastError() == cudaSuccess ? KV_OK : KV_ECUDA;
 }
 
