@@ -389,7 +389,78 @@ def config_timings(torch, kv, inputs, dev, stream, peaks, reps: int = 10) -> dic
                                 "write_us": t_w * 1e3, "write_gbs": wb / (t_w * 1e-3) / 1e9,
                                 "write_frac_hbm": wb / (t_w * 1e-3) / 1e9 / peaks["hbm"],
                                 "inputs": "K, V Student-t(4); Q N(0,1); bias -4"}
-    del ring
+    # the same chunk with the keys split four ways: 640 CTAs fill the SMs in even waves
+    splits = 4
+    ws = torch.empty(kv.chunk_attention_workspace_size(w.n, w.H, w.D, splits),
+                     dtype=torch.uint8, device=dev)
+    def at4():
+        kv.chunk_attention_split(ring, q, ring.next_pos, w.n, splits, ws, cache_bias=-4.0,
+                                 out=o, want_lse=False)
+    at4()
+    t_a4 = timed(torch, at4, reps, stream)
+    out["stress_1024x32768"]["attn_split4_us"] = t_a4 * 1e3
+    out["stress_1024x32768"]["attn_split4_tflops"] = f_a / (t_a4 * 1e-3) / 1e12
+    del ring, ws
+    torch.cuda.synchronize()
+    return out
+
+
+def next_rows_timing(torch, kv, inputs, dev, stream, reps: int = 10) -> dict:
+    """The paths beyond the chunk step, on the Runway shape (757 new tokens, 5,788-slot
+    ring, 40 heads x 128): gathered-row attention of a quarter of the rows, and one
+    content-memory eviction (attention over the FIFO ring and a 2,048-key memory ring,
+    key masses of the memory and of the FIFO block the next write overwrites, top-M
+    selection and gather)."""
+    w = inputs.RUNWAY
+    out = {}
+    fifo = _filled_ring(torch, kv, inputs, w, dev, -(-w.C // w.n) + 1)
+    q, k, v = inputs.chunk_qkv_torch(w, 100, device=dev)
+    kv.kv_ring_write(fifo, k, v)                           # the pending chunk
+    o = torch.empty_like(q)
+    rows = torch.arange(0, w.n, 4, dtype=torch.int32, device=dev)
+    def rw():
+        kv.chunk_attention_rows(fifo, q, fifo.next_pos, w.n, rows, o, mask=(1, 1, 1, 1))
+    rw()
+    t_r = timed(torch, rw, reps, stream)
+    out["rows_quarter_runway"] = {"us_per_call": t_r * 1e3, "rows": int(rows.numel()),
+                                  "of": w.n, "mask": "token-causal"}
+    # content memory: M = 2,048 keys drawn as history at earlier positions
+    M, frame_len = 2048, 256
+    mem = kv.KvRing(M, w.H, w.D, -2 * w.C, 2 * w.C, device=dev)
+    dst = kv.KvRing(M, w.H, w.D, -2 * w.C, 2 * w.C, device=dev)
+    for ch in range(-(-M // w.n)):
+        _, mk, mv = inputs.chunk_qkv_torch(w, 200 + ch, device=dev)
+        kv.kv_ring_write(mem, mk, mv, commit=True)
+    ws = torch.empty(kv.chunk_attention_workspace_size(w.n, w.H, w.D, 2), dtype=torch.uint8,
+                     device=dev)
+    lse = torch.empty((w.H, w.n), dtype=torch.float32, device=dev)
+    def att():
+        kv.chunk_attention_multi([fifo, mem], q, fifo.next_pos, w.n, 1, ws, mask=(1, 1, 1, 1),
+                                 out=o, lse=lse)
+    att()
+    first = (fifo.s.write_slot + w.n) % w.C                # the block the next write overwrites
+    n_mem = mem.n_valid
+    mem_first = (mem.s.write_slot + mem.s.pending - n_mem) % M
+    mf = torch.empty((w.H, w.n), dtype=torch.float32, device=dev)
+    mm = torch.empty((w.H, n_mem), dtype=torch.float32, device=dev)
+    kept = torch.empty((M,), dtype=torch.int32, device=dev)
+    def mass():
+        kv.chunk_key_mass(fifo, fifo, q, fifo.next_pos, lse, first, w.n, mass=mf)
+        kv.chunk_key_mass(fifo, mem, q, fifo.next_pos, lse, mem_first, n_mem, mass=mm)
+    def select():
+        kv.kv_memory_select(mem, mm, fifo, mf, first, w.n, M, frame_len, dst, kept=kept)
+    mass()
+    select()
+    t_att = timed(torch, att, reps, stream)
+    t_mass = timed(torch, mass, reps, stream)
+    t_sel = timed(torch, select, reps, stream)
+    out["content_memory_runway"] = {
+        "attention_fifo_plus_memory_us": t_att * 1e3, "key_mass_us": t_mass * 1e3,
+        "select_and_gather_us": t_sel * 1e3, "memory_keys": M, "fifo_block": w.n,
+        "frame_len": frame_len,
+        "note": "one eviction: masses of 2,048 memory keys and 757 FIFO keys over 757 queries "
+                "x 40 heads, then top-2,048 of 2,805 candidates"}
+    del fifo, mem, dst, ws
     torch.cuda.synchronize()
     return out
 
@@ -654,13 +725,14 @@ def main():
     if args.no_extras:
         rot = {"us_per_launch": float("nan"), "bytes_per_launch": 0}
         e2e = {"ms_per_step": float("nan"), "h2d": 0, "d2h": 0}
-        per_call, fp8, configs = None, None, None
+        per_call, fp8, configs, nxt = None, None, None, None
     else:
         rot = rotate_timing(torch, kv, inputs, dev)
         e2e = e2e_timing(torch, kv, step, args.e2e_steps, stream)
         per_call = per_call_percentiles(torch, step, stream)
         fp8 = fp8_gemm_peak(torch)
         configs = config_timings(torch, kv, inputs, dev, stream, peaks)
+        nxt = next_rows_timing(torch, kv, inputs, dev, stream)
     rot_us = max_over_ranks(torch, dist, rot["us_per_launch"])
     e2e_ms = max_over_ranks(torch, dist, e2e["ms_per_step"])
     timeouts = kv.kv_wait_timeout_count()
@@ -721,6 +793,7 @@ def main():
         "e2e": {"value": e2e_ms * 1e3 / (R * PASSES) / world, "unit": UNIT,
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
         "configs": configs,
+        "next_rows": nxt,
         "gpu_launches": 2 * R * PASSES * args.steps,
         "clocks": clk,
         "wait_timeouts": timeouts,

@@ -253,15 +253,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
 
     // S = Q K^T
-    if (tid == 0) {
+    if (tid < 32) {                                   // warp 0; one elected lane issues
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-        tc_mma_f16_ss(tmem, smem_desc_sw128(sQ + off, 16, 1024),
+        el_mma_f16_ss(tmem, smem_desc_sw128(sQ + off, 16, 1024),
                       smem_desc_sw128(sK + off, 16, 1024), idS, kk > 0);
       }
-      tc_commit(mma_bar);
+      el_commit(mma_bar);
     }
     ok = mbar_wait(mma_bar, mma_phase, a.timeouts);
     mma_phase ^= 1u;
@@ -336,16 +336,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
 
     // O += P' V
-    if (tid == 0) {
+    if (tid < 32) {                                   // warp 0; one elected lane issues
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < BN / 16; ++kk) {
         const uint32_t pa = sP + (kk >> 2) * kPanel + (kk & 3) * 32;   // K-major P
         const uint32_t vb = sV + kk * 2048;                            // 16 keys = 2 atoms
-        tc_mma_f16_ss(tmem + 128, smem_desc_sw128(pa, 16, 1024),
+        el_mma_f16_ss(tmem + 128, smem_desc_sw128(pa, 16, 1024),
                       smem_desc_sw128(vb, kPanel, 1024), idO, 1);
       }
-      tc_commit(mma_bar);
+      el_commit(mma_bar);
     }
     ok = mbar_wait(mma_bar, mma_phase, a.timeouts);
     mma_phase ^= 1u;

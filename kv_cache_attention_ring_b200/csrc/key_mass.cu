@@ -176,15 +176,15 @@ __global__ void __launch_bounds__(kThreads, 1) key_mass_kernel(const KeyMassArgs
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (tid == 0) {
+    if (tid < 32) {                                   // warp 0; one elected lane issues
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         const uint64_t qd = hf == 0 ? dQhi : dQlo;
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk)
-          tc_mma_f8_ss(tmem, dK + 2 * kk, qd + 2 * kk, idS, (hf | kk) != 0);
+          el_mma_f8_ss(tmem, dK + 2 * kk, qd + 2 * kk, idS, (hf | kk) != 0);
       }
-      tc_commit(bar);
+      el_commit(bar);
     }
     ok = mbar_wait(bar, phase, a.timeouts);
     tc_fence_after();
