@@ -222,12 +222,13 @@ __global__ void __launch_bounds__(kThreads, 1) key_mass_kernel(const KeyMassArgs
 // ------------------------------------------------------------------ selection
 constexpr int kSelThreads = 1024;
 
-// Candidates of a selection: quality, position, frame, index; kept in shared memory.
-struct Cand {
+// Candidates of a selection: quality (then score), index, position, frame; 16 bytes, kept in
+// shared memory.  Positions are the rings' int32 slot positions, so frames fit in 32 bits.
+struct __align__(16) Cand {
   float q;
   int idx;
-  long long pos;
-  long long frame;
+  int pos;
+  int frame;
 };
 
 // (frame asc, quality desc, position asc, index asc)
@@ -249,17 +250,17 @@ template <bool kByFrame>
 __device__ void bitonic(Cand* v, int n_pow2) {
   for (int size = 2; size <= n_pow2; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = threadIdx.x; i < n_pow2; i += blockDim.x) {
-        const int j = i ^ stride;
-        if (j > i) {
-          const bool up = (i & size) == 0;
-          const bool swap = kByFrame ? (up ? before_in_frame(v[j], v[i]) : before_in_frame(v[i], v[j]))
-                                     : (up ? before_in_score(v[j], v[i]) : before_in_score(v[i], v[j]));
-          if (swap) {
-            const Cand t = v[i];
-            v[i] = v[j];
-            v[j] = t;
-          }
+      for (int t = threadIdx.x; t < (n_pow2 >> 1); t += blockDim.x) {
+        // t-th pair: i has bit `stride` clear, j = i + stride
+        const int i = ((t & ~(stride - 1)) << 1) | (t & (stride - 1));
+        const int j = i + stride;
+        const Cand x = v[i], y = v[j];
+        const bool up = (i & size) == 0;
+        const bool swap = kByFrame ? (up ? before_in_frame(y, x) : before_in_frame(x, y))
+                                   : (up ? before_in_score(y, x) : before_in_score(x, y));
+        if (swap) {
+          v[i] = y;
+          v[j] = x;
         }
       }
       __syncthreads();
@@ -267,56 +268,140 @@ __device__ void bitonic(Cand* v, int n_pow2) {
   }
 }
 
+// Block-wide inclusive max-scan of one int per thread (kSelThreads threads).
+__device__ int block_max_scan(int x, int* red) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x = max(x, y);
+  }
+  if (lane == 31) red[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    int w = red[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w = max(w, y);
+    }
+    red[lane] = w;
+  }
+  __syncthreads();
+  const int r = wid > 0 ? max(x, red[wid - 1]) : x;
+  __syncthreads();
+  return r;
+}
+
 __global__ void __launch_bounds__(kSelThreads) memory_select_kernel(const SelectArgs a) {
   extern __shared__ uint8_t smem_raw[];
   Cand* v = reinterpret_cast<Cand*>(smem_raw);
+  __shared__ int red[32];
+  __shared__ uint32_t kbits[KV_MEMORY_MAX_CANDIDATES / 32];
+  __shared__ int wpre[KV_MEMORY_MAX_CANDIDATES / 32];
+  const int tid = threadIdx.x;
   const int n = a.n_mem + a.n_fifo;
   int n_pow2 = 1;
   while (n_pow2 < n) n_pow2 <<= 1;
-  for (int i = threadIdx.x; i < n_pow2; i += blockDim.x) {
+  for (int i = tid; i < n_pow2; i += blockDim.x) {
     Cand c;
     if (i < n) {
       const bool mem = i < a.n_mem;
       const float* m = mem ? a.mass_mem : a.mass_fifo;
       const int ci = mem ? i : i - a.n_mem;
       const int nc = mem ? a.n_mem : a.n_fifo;
+      // quality: the heads' masses added in head order; loads issued eight at a time
       float q = 0.f;
-      for (int h = 0; h < a.H; ++h) q += m[(size_t)h * nc + ci];   // fixed order over heads
+      for (int h0 = 0; h0 < a.H; h0 += 8) {
+        float t[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) t[u] = h0 + u < a.H ? __ldg(m + (size_t)(h0 + u) * nc + ci) : 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (h0 + u < a.H) q += t[u];
+      }
       int slot = (mem ? a.mem_slot_first : a.fifo_slot_first) + ci;
       const int C = mem ? a.mem_C : a.fifo_C;
       slot = slot >= C ? slot - C : slot;
       const long long pos = (mem ? a.mem_pos : a.fifo_pos)[slot];
       c.q = q;
       c.idx = i;
-      c.pos = pos;
-      c.frame = pos >= 0 ? pos / a.frame_len : -((-pos + a.frame_len - 1) / a.frame_len);
+      c.pos = (int)pos;
+      c.frame = (int)(pos >= 0 ? pos / a.frame_len : -((-pos + a.frame_len - 1) / a.frame_len));
     } else {
       c.q = -INFINITY;                               // padding sorts last in both orders
       c.idx = 0x7FFFFFFF;
-      c.pos = 0x7FFFFFFFFFFFFFFFll;
-      c.frame = 0x7FFFFFFFFFFFFFFFll;
+      c.pos = 0x7FFFFFFF;
+      c.frame = 0x7FFFFFFF;
     }
     v[i] = c;
   }
   __syncthreads();
   bitonic<true>(v, n_pow2);
-  // rank within the frame: the k-th entry of a frame run scores quality * gamma^k
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    int first = i;
-    while (first > 0 && v[first - 1].frame == v[i].frame) --first;
-    float s = v[i].q;
-    for (int k = first; k < i; ++k) s *= a.gamma;
-    v[i].q = s;                                      // frames and positions stay as keys
+  // rank within the frame: the k-th entry of a frame run scores quality * gamma^k, gamma^k
+  // formed by repeated multiplication.  Each thread takes a contiguous chunk; the run in
+  // effect at its first entry comes from a max-scan of the chunks' last run starts.
+  {
+    const int per = (n + kSelThreads - 1) / kSelThreads;
+    const int lo = min(tid * per, n), hi = min(lo + per, n);
+    int last_start = -1;
+    for (int i = lo; i < hi; ++i)
+      if (i == 0 || v[i].frame != v[i - 1].frame) last_start = i;
+    const int incl = block_max_scan(last_start, red);
+    const int before = __shfl_up_sync(0xffffffffu, incl, 1);
+    // run start in effect before lo: the previous thread's inclusive value (for the first
+    // lane of a warp, the scanned total of the warps before it)
+    const int carry = (tid & 31) ? before : (tid > 0 ? red[(tid >> 5) - 1] : -1);
+    float scale = 1.f;
+    if (lo < hi) {
+      const int start = (lo == 0 || v[lo].frame != v[lo - 1].frame) ? lo : max(carry, 0);
+      for (int k = start; k < lo; ++k) scale *= a.gamma;
+    }
+    float qs[8];
+    for (int i = lo; i < hi; ++i) {
+      if (i > lo) scale = (v[i].frame == v[i - 1].frame) ? scale * a.gamma : 1.f;
+      qs[i - lo] = v[i].q * scale;
+    }
+    __syncthreads();                                 // every frame read before q changes
+    for (int i = lo; i < hi; ++i) v[i].q = qs[i - lo];
   }
   __syncthreads();
   bitonic<false>(v, n_pow2);
-  // the best min(n, M), listed in ascending candidate index
+  // the best min(n, M), listed in ascending candidate index: a bitmap of the kept indices
+  // and a prefix count over it
   const int m = n < a.M ? n : a.M;
-  for (int i = threadIdx.x; i < m; i += blockDim.x) {
-    // position of v[i] among the kept in ascending idx order = count of kept with lower idx
-    int rank = 0;
-    for (int k = 0; k < m; ++k) rank += v[k].idx < v[i].idx;
-    a.kept[rank] = v[i].idx;
+  const int n_words = (n + 31) >> 5;
+  for (int w = tid; w < n_words; w += blockDim.x) kbits[w] = 0u;
+  __syncthreads();
+  for (int i = tid; i < m; i += blockDim.x) atomicOr(&kbits[v[i].idx >> 5], 1u << (v[i].idx & 31));
+  __syncthreads();
+  if (tid < 32) {                                    // exclusive prefix of the words' counts
+    const int per_w = (n_words + 31) >> 5;
+    int run = 0;
+    for (int k = 0; k < per_w; ++k) {
+      const int w = tid * per_w + k;
+      run += w < n_words ? __popc(kbits[w]) : 0;
+    }
+    int incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (tid >= o) incl += y;
+    }
+    int base = incl - run;
+    for (int k = 0; k < per_w; ++k) {
+      const int w = tid * per_w + k;
+      if (w < n_words) {
+        wpre[w] = base;
+        base += __popc(kbits[w]);
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < m; i += blockDim.x) {
+    const int idx = v[i].idx;
+    const int r = wpre[idx >> 5] + __popc(kbits[idx >> 5] & ((1u << (idx & 31)) - 1u));
+    a.kept[r] = idx;
   }
 }
 
@@ -368,7 +453,8 @@ int launch_memory_select(const SelectArgs& a, cudaStream_t s) {
   const int n = a.n_mem + a.n_fifo;
   const size_t bytes = select_smem_bytes(n);
   static unsigned char configured[kMaxDevices] = {};
-  if (!smem_attr_set(reinterpret_cast<const void*>(memory_select_kernel), 232448, configured))
+  if (!smem_attr_set(reinterpret_cast<const void*>(memory_select_kernel),
+                     (int)select_smem_bytes(KV_MEMORY_MAX_CANDIDATES), configured))
     return KV_ECUDA;
   memory_select_kernel<<<1, kSelThreads, bytes, s>>>(a);
   if (cudaPeekAtLastError() != cudaSuccess) return KV_ECUDA;
