@@ -710,11 +710,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         float m0 = -INFINITY, m1 = -INFINITY;
         uint32_t p8[16];                               // kPv8: e4m3 P, four keys per word
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t pk[16];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[8];
 #pragma unroll
-          for (int q8 = 0; q8 < 8; ++q8) {
-            const int q = 8 * c + q8;
+          for (int q8 = 0; q8 < 4; ++q8) {
+            const int q = 4 * c + q8;
             const float4 ks = k4[q], ww = w4[q];
             const uint64_t u01 = f2_mul(f2_pack(__uint_as_float(sr[4 * q]), __uint_as_float(sr[4 * q + 1])),
                                         f2_pack(ks.x, ks.y));
@@ -741,7 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           // P over S columns already read into registers; a recomputation overwrites it
-          if (!kPv8) tmem_st16(t_s + 16 * c, pk);
+          if (!kPv8) tmem_st8(t_s + 8 * c, pk);
         }
         if (kPv8) tmem_st16(t_s, p8);
         const float mloc = fmaf(fmaxf(m0, m1), rowmul, a.bias_log2);
@@ -811,11 +811,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         sum23 = sum01;
         uint32_t p8[16];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t pk[16];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[8];
 #pragma unroll
-          for (int q8 = 0; q8 < 8; ++q8) {
-            const int q = 8 * c + q8;
+          for (int q8 = 0; q8 < 4; ++q8) {
+            const int q = 4 * c + q8;
             const float4 ww = w4[q];
             float t0, t1, t2, t3;
             f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[4 * q]), __uint_as_float(sr[4 * q + 1])), mul2,
@@ -836,7 +836,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               pk[2 * q8 + 1] = pack_f16x2(a2, a3);
             }
           }
-          if (!kPv8) tmem_st16(t_s + 16 * c, pk);
+          if (!kPv8) tmem_st8(t_s + 8 * c, pk);
         }
         if (kPv8) tmem_st16(t_s, p8);
       }
