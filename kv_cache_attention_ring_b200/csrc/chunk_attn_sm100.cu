@@ -905,31 +905,72 @@ __global__ void __launch_bounds__(kThreads, 1)
                   : make_float2(__uint_as_float(0x7FC00000u), __uint_as_float(0x7FC00000u));
       }
     } else {
-      uint16_t* dst = a.out + ((size_t)(row_ok ? gi : 0) * a.H + h) * D;
       const float inv_l = (l_run > 0.f) ? (1.f / l_run) * vnorm : 0.f;
+      // Rows go through shared memory (the K and V code stages are free once every MMA has
+      // completed) so that whole 256-byte rows are stored with coalesced 16-byte stores.
+      // After an abandoned wait in any softmax warp, every row is stored directly instead.
+      if (named_bar_and(1, 256, ok)) {
+        uint8_t* st = sm + Layout::kbuf;                      // [256 rows][256 B], swizzled
 #pragma unroll 1
-      for (int c = 0; c < D / 64; ++c) {
-        uint32_t o[64];
-        if (any) {
-          uint32_t (&lo)[32] = *reinterpret_cast<uint32_t (*)[32]>(o);
-          uint32_t (&hi)[32] = *reinterpret_cast<uint32_t (*)[32]>(o + 32);
-          tmem_ld32(t_o + 64 * c, lo);
-          tmem_ld32(t_o + 64 * c + 32, hi);
-          tmem_wait_ld();
-        }
-        uint32_t pk[32];
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t o[64];
+          if (any) {
+            uint32_t (&lo)[32] = *reinterpret_cast<uint32_t (*)[32]>(o);
+            uint32_t (&hi)[32] = *reinterpret_cast<uint32_t (*)[32]>(o + 32);
+            tmem_ld32(t_o + 64 * c, lo);
+            tmem_ld32(t_o + 64 * c + 32, hi);
+            tmem_wait_ld();
+          }
+          uint32_t pk[32];
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          float x0 = l_run > 0.f ? __uint_as_float(o[2 * k]) * inv_l : 0.f;
-          float x1 = l_run > 0.f ? __uint_as_float(o[2 * k + 1]) * inv_l : 0.f;
-          if (!ok) x0 = x1 = __uint_as_float(0x7FC00000u);
-          pk[k] = pack_bf16x2(x0, x1);
-        }
-        if (row_ok) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + 64 * c);
+          for (int k = 0; k < 32; ++k) {
+            const float x0 = l_run > 0.f ? __uint_as_float(o[2 * k]) * inv_l : 0.f;
+            const float x1 = l_run > 0.f ? __uint_as_float(o[2 * k + 1]) * inv_l : 0.f;
+            pk[k] = pack_bf16x2(x0, x1);
+          }
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            d4[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+          for (int k = 0; k < 8; ++k) {
+            const int cc = 8 * c + k;                           // 16-byte chunk of the row
+            *reinterpret_cast<uint4*>(st + row * 256 + ((cc ^ (row & 15)) << 4)) =
+                make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+          }
+        }
+        named_bar(1, 256);
+        const int sw = warp - kWarpSoft;                        // rows [32 sw, 32 sw + 32)
+#pragma unroll 4
+        for (int it = 0; it < 16; ++it) {
+          const int r = 32 * sw + 2 * it + (lane >> 4), cc = lane & 15;
+          const int gr = row_gi[r];
+          if (gr >= 0)
+            *reinterpret_cast<uint4*>(a.out + ((size_t)gr * a.H + h) * D + 8 * cc) =
+                *reinterpret_cast<const uint4*>(st + r * 256 + ((cc ^ (r & 15)) << 4));
+        }
+      } else {
+        uint16_t* dst = a.out + ((size_t)(row_ok ? gi : 0) * a.H + h) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t o[64];
+          if (any) {
+            uint32_t (&lo)[32] = *reinterpret_cast<uint32_t (*)[32]>(o);
+            uint32_t (&hi)[32] = *reinterpret_cast<uint32_t (*)[32]>(o + 32);
+            tmem_ld32(t_o + 64 * c, lo);
+            tmem_ld32(t_o + 64 * c + 32, hi);
+            tmem_wait_ld();
+          }
+          uint32_t pk[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            float x0 = l_run > 0.f ? __uint_as_float(o[2 * k]) * inv_l : 0.f;
+            float x1 = l_run > 0.f ? __uint_as_float(o[2 * k + 1]) * inv_l : 0.f;
+            if (!ok) x0 = x1 = __uint_as_float(0x7FC00000u);
+            pk[k] = pack_bf16x2(x0, x1);
+          }
+          if (row_ok) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + 64 * c);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              d4[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+          }
         }
       }
       if (row_ok && a.lse) {
