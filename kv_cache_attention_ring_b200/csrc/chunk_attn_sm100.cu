@@ -29,7 +29,8 @@
 //    the first K/V tile loads.
 //  * Tensor memory (512 columns): tile g owns two S/P buffers of 64 columns,
 //    [128g, 128g+64) and [128g+64, 128g+128), and O_g = [256+128g, 384+128g).  The MMA
-//    issuer serves the two query tiles in lockstep: for key tile j it waits for P_0(j)
+//    warp runs its loop converged and one elected lane issues each instruction; it
+//    serves the two query tiles in lockstep: for key tile j it waits for P_0(j)
 //    (and V(j) widened), runs P.V_0(j) and S_0(j+2) into the buffer P_0(j) occupied,
 //    then does the same for tile 1 (tensor-core operations of one thread run in issue
 //    order).  Query tile 1 releases the K stage and the V buffer.
@@ -38,12 +39,14 @@
 //    2-3 V converters, 4-7 softmax of tile 0, 8-11 softmax of tile 1 (thread = query
 //    row = TMEM lane).
 //  * Softmax in log2 units with paired fp32 instructions (f32x2) on the 64-column S row
-//    held in registers.  The reference maximum m moves lazily (only when the tile
+//    held in registers; P goes back to tensor memory in 8-column pieces.  The reference maximum m moves lazily (only when the tile
 //    maximum exceeds it by more than 8, a factor 256); O is then rescaled in tensor
 //    memory after the previous P.V has completed.  out = O / l is exact regardless of m.
 //    A history-only tile with m already set takes one pass (scale, 2^(t - m), P, tile
 //    maximum on the way); the first tile, tiles with current or invalid keys, and tiles
 //    whose maximum exceeds m by more than 8 take two (maximum first, then 2^(t - m)).
+//  * Epilogue: O / l in bf16 goes through the K/V code stages of shared memory (free once
+//    every MMA has completed), so whole 256-byte output rows leave in coalesced stores.
 //  * Split over keys (gridDim.z > 1): each CTA takes a contiguous share of the valid
 //    tiles and writes fp32 partials (O G, m, l); split_combine_kernel merges them.
 //  * Keys are visited in physical slot order; the ring wrap costs nothing (attention
