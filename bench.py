@@ -422,8 +422,16 @@ def next_rows_timing(torch, kv, inputs, dev, stream, reps: int = 10) -> dict:
         kv.chunk_attention_rows(fifo, q, fifo.next_pos, w.n, rows, o, mask=(1, 1, 1, 1))
     rw()
     t_r = timed(torch, rw, reps, stream)
-    out["rows_quarter_runway"] = {"us_per_call": t_r * 1e3, "rows": int(rows.numel()),
-                                  "of": w.n, "mask": "token-causal"}
+    # the same rows with the keys split three ways: 120 CTAs instead of 40
+    wsr = torch.empty(kv.chunk_attention_workspace_size(int(rows.numel()), w.H, w.D, 3),
+                      dtype=torch.uint8, device=dev)
+    def rw3():
+        kv.chunk_attention_rows(fifo, q, fifo.next_pos, w.n, rows, o, mask=(1, 1, 1, 1),
+                                n_splits=3, workspace=wsr)
+    rw3()
+    t_r3 = timed(torch, rw3, reps, stream)
+    out["rows_quarter_runway"] = {"us_per_call": t_r * 1e3, "us_per_call_3_key_splits": t_r3 * 1e3,
+                                  "rows": int(rows.numel()), "of": w.n, "mask": "token-causal"}
     # content memory: M = 2,048 keys drawn as history at earlier positions
     M, frame_len = 2048, 256
     mem = kv.KvRing(M, w.H, w.D, -2 * w.C, 2 * w.C, device=dev)

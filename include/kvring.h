@@ -241,13 +241,21 @@ KV_API int chunk_attention(const kv_ring_t* kv, const void* q, int n_q, int64_t 
  * every other row of out and lse is left as it was (the static regions keep their
  * previous outputs).  A listed index outside [0, n_q) is skipped: nothing is computed or
  * written for it (the indices live on the device, so the host cannot reject them).
- * n_rows = 0 enqueues nothing.  head_dim 128 only.  Errors: those of chunk_attention,
- * KV_EINVAL (rows null or misaligned, n_rows < 0), KV_ERANGE (n_rows * n_heads > 2^31),
- * KV_EUNSUPPORTED (head_dim 64). */
+ * n_rows = 0 enqueues nothing.  head_dim 128 only.
+ * n_splits (1..64) splits the keys as chunk_attention_split does, so that few listed rows
+ * still fill the SMs: each split writes fp32 partials per list entry into workspace
+ * (device, 16-byte aligned, caller-owned, at least
+ * chunk_attention_workspace_size(n_rows, n_heads, head_dim, n_splits) bytes), and one
+ * merge writes the listed rows.  With n_splits = 1 the workspace is not used (may be
+ * NULL).  Errors: those of chunk_attention, KV_EINVAL (rows null or misaligned,
+ * n_rows < 0, n_splits outside 1..64, workspace null or misaligned for n_splits > 1),
+ * KV_ERANGE (n_rows * n_heads > 2^31, workspace too small), KV_EUNSUPPORTED
+ * (head_dim 64). */
 KV_API int chunk_attention_rows(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
                                 int n_current, const int32_t* rows, int n_rows,
                                 const kv_block_mask_t* mask, const kv_cache_bias_t* bias,
-                                float softmax_scale, void* out, float* lse, uint32_t flags,
+                                float softmax_scale, void* out, float* lse, int n_splits,
+                                void* workspace, size_t workspace_bytes, uint32_t flags,
                                 void* stream);
 
 /* Bytes of workspace chunk_attention_split needs: n_splits * n_q * n_heads * (4*head_dim + 8).

@@ -90,7 +90,7 @@ def lib() -> ctypes.CDLL:
         L.chunk_attention.argtypes = [P, P, I, I64, I, P, P, ctypes.c_float, P, P,
                                       ctypes.c_uint32, P]
         L.chunk_attention_rows.argtypes = [P, P, I, I64, I, P, I, P, P, ctypes.c_float, P, P,
-                                           ctypes.c_uint32, P]
+                                           I, P, ctypes.c_size_t, ctypes.c_uint32, P]
         L.chunk_key_mass.argtypes = [P, P, P, I, I64, P, P, ctypes.c_float, I64, I, P, P]
         L.kv_memory_select.argtypes = [P, P, P, P, I64, I, I, I64, ctypes.c_float, P, P, P]
         L.kv_status_string.argtypes = [I]
@@ -254,10 +254,12 @@ def chunk_attention(ring: KvRing, q, q_pos0: int, n_current: int, mask=None,
 
 def chunk_attention_rows(ring: KvRing, q, q_pos0: int, n_current: int, rows, out, lse=None,
                          mask=None, cache_bias: float = 0.0, softmax_scale: float | None = None,
-                         stream=None, mode_b: bool = False):
+                         stream=None, mode_b: bool = False, n_splits: int = 1, workspace=None):
     """chunk_attention for the listed query rows only: q is the whole chunk (bf16
     [n_q][H][D]); rows is a device int32 tensor of chunk indices; out (bf16 [n_q][H][D])
-    and lse (fp32 [H][n_q], optional) receive the listed rows and keep every other row."""
+    and lse (fp32 [H][n_q], optional) receive the listed rows and keep every other row.
+    n_splits > 1 splits the keys (workspace: a device tensor of at least
+    chunk_attention_workspace_size(len(rows), H, D, n_splits) bytes)."""
     import torch
     assert q.is_cuda and q.dtype == torch.bfloat16 and q.is_contiguous()
     n_q = int(q.shape[0])
@@ -268,15 +270,19 @@ def chunk_attention_rows(ring: KvRing, q, q_pos0: int, n_current: int, rows, out
     if lse is not None:
         assert lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous()
         assert lse.shape == (ring.H, n_q)
+    if workspace is not None:
+        assert workspace.is_cuda and workspace.is_contiguous()
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(ring.D)
     m = None if mask is None else kv_block_mask_t(*(int(x) for x in mask))
     b = kv_cache_bias_t(float(cache_bias))
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().chunk_attention_rows(ring.ref, _ptr(q), n_q, int(q_pos0), int(n_current),
                                       _ptr(rows), int(rows.numel()),
                                       None if m is None else ctypes.byref(m), ctypes.byref(b),
                                       float(softmax_scale), _ptr(out),
-                                      None if lse is None else _ptr(lse),
+                                      None if lse is None else _ptr(lse), int(n_splits),
+                                      None if workspace is None else _ptr(workspace), nbytes,
                                       KV_QK_FP8 if mode_b else 0, _stream(stream)),
            "chunk_attention_rows")
     return out, lse

@@ -878,7 +878,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool any = j > 0;
     if (a.part_o) {
       // split over keys: unnormalised O (relative to m_run, times G) and (m_run, l_run)
-      const size_t prow = ((size_t)blockIdx.z * a.n_q + (row_ok ? gi : 0)) * a.H + h;
+      // partials are indexed by the row's list entry li (its own index without a list)
+      const int li = row_ok ? q0 + row : 0;
+      const size_t prow = ((size_t)blockIdx.z * a.n_rows + li) * a.H + h;
       float* po = a.part_o + prow * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
@@ -903,7 +905,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (row_ok) {
         float2* pml = reinterpret_cast<float2*>(a.part_ml) +
-                      ((size_t)blockIdx.z * a.H + h) * a.n_q + gi;
+                      ((size_t)blockIdx.z * a.H + h) * a.n_rows + li;
         *pml = ok ? make_float2(m_run, l_run)
                   : make_float2(__uint_as_float(0x7FC00000u), __uint_as_float(0x7FC00000u));
       }
@@ -1009,25 +1011,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 // with l_s > 0, w_s = 2^(m_s - M), out = sum w_s O_s / sum w_s l_s, lse = (M + log2 L) ln 2.
 __global__ void __launch_bounds__(256) split_combine_kernel(const AttnArgs a, int n_splits) {
   const int wid = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (wid >= a.n_q * a.H) return;                 // whole warp leaves together
-  const int gi = wid / a.H, h = wid % a.H;
+  if (wid >= a.n_rows * a.H) return;              // whole warp leaves together
+  // partials of list entry li; the output row is rows[li] (li itself without a list)
+  const int li = wid / a.H, h = wid % a.H;
+  const int gi = a.rows ? __ldg(a.rows + li) : li;
+  if (gi < 0 || gi >= a.n_q) return;
   const float2* pml = reinterpret_cast<const float2*>(a.part_ml);
   float M = -INFINITY;
   bool bad = false;                               // a split that gave up: NaN out
   for (int z = 0; z < n_splits; ++z) {
-    const float2 ml = pml[((size_t)z * a.H + h) * a.n_q + gi];
+    const float2 ml = pml[((size_t)z * a.H + h) * a.n_rows + li];
     bad |= isnan(ml.y);
     if (ml.y > 0.f) M = fmaxf(M, ml.x);
   }
   float L = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int z = 0; z < n_splits; ++z) {
-    const float2 ml = pml[((size_t)z * a.H + h) * a.n_q + gi];
+    const float2 ml = pml[((size_t)z * a.H + h) * a.n_rows + li];
     if (!(ml.y > 0.f)) continue;
     const float w = ex2(ml.x - M);
     L += w * ml.y;
     const float4 o = reinterpret_cast<const float4*>(
-        a.part_o + (((size_t)z * a.n_q + gi) * a.H + h) * D)[lane];
+        a.part_o + (((size_t)z * a.n_rows + li) * a.H + h) * D)[lane];
     acc.x += w * o.x;
     acc.y += w * o.y;
     acc.z += w * o.z;
@@ -1049,7 +1054,7 @@ __global__ void __launch_bounds__(256) split_combine_kernel(const AttnArgs a, in
 
 int launch_split_combine(const AttnArgs& a, int D_, int n_splits, cudaStream_t s) {
   if (D_ != D) return KV_EUNSUPPORTED;
-  const int warps = a.n_q * a.H;
+  const int warps = a.n_rows * a.H;
   split_combine_kernel<<<(warps + 7) / 8, 256, 0, s>>>(a, n_splits);
   return cudaPeekAtLastError() == cudaSuccess ? KV_OK : KV_ECUDA;
 }

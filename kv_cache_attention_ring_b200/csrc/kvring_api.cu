@@ -432,22 +432,36 @@ int chunk_attention(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
 int chunk_attention_rows(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
                          int n_current, const int32_t* rows, int n_rows,
                          const kv_block_mask_t* mask, const kv_cache_bias_t* bias,
-                         float softmax_scale, void* out, float* lse, uint32_t flags,
+                         float softmax_scale, void* out, float* lse, int n_splits,
+                         void* workspace, size_t workspace_bytes, uint32_t flags,
                          void* stream) {
   AttnArgs a;
   int rc = attention_args(kv, q, n_q, q_pos0, n_current, mask, bias, softmax_scale, out, lse,
                           flags, &a);
   if (rc) return rc;
-  if (n_rows < 0) return KV_EINVAL;
+  if (n_rows < 0 || n_splits < 1 || n_splits > 64) return KV_EINVAL;
   if (n_q == 0 || n_rows == 0) return KV_OK;
   if (kv->head_dim != 128) return KV_EUNSUPPORTED;
   if (!rows || (reinterpret_cast<uintptr_t>(rows) & 3u)) return KV_EINVAL;
   if ((int64_t)n_rows * kv->n_heads > ((int64_t)1 << 31)) return KV_ERANGE;
+  if (n_splits > 1) {
+    const size_t need = chunk_attention_workspace_size(n_rows, kv->n_heads, kv->head_dim, n_splits);
+    if (!workspace || !aligned16(workspace)) return KV_EINVAL;
+    if (workspace_bytes < need) return KV_ERANGE;
+  }
   if ((rc = attach_timeouts(&a))) return rc;
   a.rows = rows;
   a.n_rows = n_rows;
-  return launch_attention_sm100_d128(a, kv->opaque + kOpaqueTmapKsw, kv->opaque + kOpaqueTmapVsw,
-                                     static_cast<cudaStream_t>(stream), 1);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (n_splits == 1)
+    return launch_attention_sm100_d128(a, kv->opaque + kOpaqueTmapKsw,
+                                       kv->opaque + kOpaqueTmapVsw, s, 1);
+  a.part_o = static_cast<float*>(workspace);
+  a.part_ml = a.part_o + (size_t)n_splits * n_rows * kv->n_heads * kv->head_dim;
+  rc = launch_attention_sm100_d128(a, kv->opaque + kOpaqueTmapKsw, kv->opaque + kOpaqueTmapVsw,
+                                   s, n_splits);
+  if (rc) return rc;
+  return launch_split_combine(a, kv->head_dim, n_splits, s);
 }
 
 size_t chunk_attention_workspace_size(int n_q, int n_heads, int head_dim, int n_splits) {

@@ -198,10 +198,17 @@ def test_rows_validation_before_launch(L):
     s.live = 64
     r = ctypes.byref(s)
 
-    def call(rows=16, n_rows=4, n_q=8, flags=0, ring=r):
+    def call(rows=16, n_rows=4, n_q=8, flags=0, ring=r, splits=1, ws=None, ws_bytes=0):
         return L.chunk_attention_rows(ring, 16, n_q, 0, 8, rows, n_rows, None, None, 0.125, 16,
-                                      None, flags, None)
+                                      None, splits, ws, ws_bytes, flags, None)
 
+    need = kv.lib().chunk_attention_workspace_size(4, s.n_heads, 128, 3)
+    assert need == 3 * 4 * s.n_heads * (4 * 128 + 8)
+    assert call(splits=0) == kv.KV_EINVAL
+    assert call(splits=65) == kv.KV_EINVAL
+    assert call(splits=3) == kv.KV_EINVAL              # no workspace
+    assert call(splits=3, ws=24, ws_bytes=need) == kv.KV_EINVAL      # not 16-byte aligned
+    assert call(splits=3, ws=32, ws_bytes=need - 1) == kv.KV_ERANGE
     assert call(n_rows=-1) == kv.KV_EINVAL
     assert call(n_rows=0) == kv.KV_OK                  # nothing to do
     assert call(n_q=0) == kv.KV_OK

@@ -85,3 +85,32 @@ def test_out_of_range_indices_are_skipped_and_empty_list_is_a_no_op(orc):
     ro, rl = o.attention(inputs.as_f32(q), o.next_pos, n_q, (1, 1, 1, 1), rows=[3, 199])
     assert_attention_close(out, lse, ro, rl, rows=[3, 199], what="rows in range")
     assert kv.kv_wait_timeout_count() == 0
+
+
+@pytest.mark.parametrize("n_splits", [2, 5])
+def test_gathered_rows_with_key_splits(orc, n_splits):
+    """The rows path with the keys split over CTAs: partials per list entry, one merge.
+    Listed rows match the oracle (the merge adds in another order, so not bit for bit),
+    out-of-range entries are skipped, every other row is left as it was."""
+    ring, o, q = _ring(orc, seed=67)
+    n_q, H = q.shape[0], ring.H
+    rng = np.random.default_rng(9)
+    listed = np.concatenate([[0, 255, 256, 756, 40, 40, -3, n_q, 1 << 29],
+                             rng.choice(n_q, 90, replace=False)]).astype(np.int32)
+    rng.shuffle(listed)
+    qd = to_dev(q)
+    out = torch.full_like(qd, SENTINEL)
+    lse = torch.full((H, n_q), 123.0, dtype=torch.float32, device="cuda")
+    ws = torch.empty(kv.chunk_attention_workspace_size(len(listed), H, 128, n_splits),
+                     dtype=torch.uint8, device="cuda")
+    kv.chunk_attention_rows(ring, qd, ring.next_pos, n_q, to_dev(torch.from_numpy(listed)), out,
+                            lse, mask=(1, 1, 1, 1), cache_bias=-0.5, n_splits=n_splits,
+                            workspace=ws)
+    torch.cuda.synchronize()
+    uniq = np.unique(listed[(listed >= 0) & (listed < n_q)])
+    rest = np.setdiff1d(np.arange(n_q), uniq)
+    assert (out[torch.from_numpy(rest)].float() == SENTINEL).all()
+    assert (lse[:, torch.from_numpy(rest)] == 123.0).all()
+    ro, rl = o.attention(inputs.as_f32(q), o.next_pos, n_q, (1, 1, 1, 1), -0.5, rows=uniq)
+    assert_attention_close(out, lse, ro, rl, rows=uniq, what=f"rows, {n_splits} key splits")
+    assert kv.kv_wait_timeout_count() == 0
