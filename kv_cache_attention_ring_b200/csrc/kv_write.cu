@@ -17,7 +17,7 @@ namespace kvring {
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 64;         // small blocks: the grid's last partial wave is short
 constexpr int kRows = 1;        // rows per lane group (more in flight cost occupancy here)
 
 template <typename T>
