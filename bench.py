@@ -234,6 +234,23 @@ def timed(torch, fn, reps: int, stream) -> float:
     return a.elapsed_time(b) / reps
 
 
+def graph_timed(torch, fn, reps: int, stream, inner: int = 10) -> float:
+    """Milliseconds per call of fn, from a CUDA graph of `inner` calls replayed `reps`
+    times (no host launch overhead in the timed region); fn must leave the state it found
+    (attention calls, or rewrites of a pending chunk)."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        for _ in range(inner):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    ms = timed(torch, g.replay, reps, stream) / inner
+    del g
+    return ms
+
+
 def per_call_percentiles(torch, step: "RunwayStep", stream) -> dict:
     """Per-call device time (write + attention) of one eager pass over the step's 240
     calls: an event between consecutive calls (the host runs ahead of the device, so the
@@ -322,7 +339,7 @@ def config_timings(torch, kv, inputs, dev, stream, peaks, reps: int = 10) -> dic
         for b in w.biases:
             kv.chunk_attention(ring, q, ring.next_pos, w.n, w.mask, b, out=o, want_lse=False)
     wan()
-    ms = timed(torch, wan, reps, stream) / len(w.biases)
+    ms = graph_timed(torch, wan, reps, stream, inner=2) / len(w.biases)
     flop = 4 * w.D * w.H * attn_pairs(w.n, w.C - w.n, *w.mask, w.n)
     out["wan_4680x23400"] = {"us_per_call": ms * 1e3, "gflop_per_call": flop / 1e9,
                              "tflops": flop / (ms * 1e-3) / 1e12,
@@ -353,10 +370,10 @@ def config_timings(torch, kv, inputs, dev, stream, peaks, reps: int = 10) -> dic
         kv.chunk_attention(ra, qa, ra.next_pos, wa.n, None, 0.0, out=oa, want_lse=False)
     for f in (vv_, av_, va_, aa_):
         f()
-    t_vv = timed(torch, vv_, reps, stream)
-    t_av = timed(torch, av_, reps, stream)
-    t_va = timed(torch, va_, reps, stream)
-    t_aa = timed(torch, aa_, reps, stream)
+    t_vv = graph_timed(torch, vv_, reps, stream)
+    t_av = graph_timed(torch, av_, reps, stream)
+    t_va = graph_timed(torch, va_, reps, stream)
+    t_aa = graph_timed(torch, aa_, reps, stream)
     f_vv = 4 * wv.D * wv.H * wv.n * wv.C
     av_bytes = wv.C * wv.H * (2 * wv.D + 8)          # K, V codes and scales of the video ring
     out["av_v2v_1152x24192"] = {"us_per_call": t_vv * 1e3, "gflop_per_call": f_vv / 1e9,
@@ -379,8 +396,8 @@ def config_timings(torch, kv, inputs, dev, stream, peaks, reps: int = 10) -> dic
     def at():
         kv.chunk_attention(ring, q, ring.next_pos, w.n, None, -4.0, out=o, want_lse=False)
     at()
-    t_w = timed(torch, wr, reps, stream)
-    t_a = timed(torch, at, reps, stream)
+    t_w = graph_timed(torch, wr, reps, stream)
+    t_a = graph_timed(torch, at, reps, stream, inner=2)
     f_a = 4 * w.D * w.H * w.n * w.C
     wb = write_bytes(w.n, w.H, w.D)
     out["stress_1024x32768"] = {"attn_us": t_a * 1e3, "attn_gflop": f_a / 1e9,
@@ -397,7 +414,7 @@ def config_timings(torch, kv, inputs, dev, stream, peaks, reps: int = 10) -> dic
         kv.chunk_attention_split(ring, q, ring.next_pos, w.n, splits, ws, cache_bias=-4.0,
                                  out=o, want_lse=False)
     at4()
-    t_a4 = timed(torch, at4, reps, stream)
+    t_a4 = graph_timed(torch, at4, reps, stream, inner=2)
     out["stress_1024x32768"]["attn_split4_us"] = t_a4 * 1e3
     out["stress_1024x32768"]["attn_split4_tflops"] = f_a / (t_a4 * 1e-3) / 1e12
     del ring, ws
@@ -421,7 +438,7 @@ def next_rows_timing(torch, kv, inputs, dev, stream, reps: int = 10) -> dict:
     def rw():
         kv.chunk_attention_rows(fifo, q, fifo.next_pos, w.n, rows, o, mask=(1, 1, 1, 1))
     rw()
-    t_r = timed(torch, rw, reps, stream)
+    t_r = graph_timed(torch, rw, reps, stream)
     # the same rows with the keys split three ways: 120 CTAs instead of 40
     wsr = torch.empty(kv.chunk_attention_workspace_size(int(rows.numel()), w.H, w.D, 3),
                       dtype=torch.uint8, device=dev)
@@ -429,7 +446,7 @@ def next_rows_timing(torch, kv, inputs, dev, stream, reps: int = 10) -> dict:
         kv.chunk_attention_rows(fifo, q, fifo.next_pos, w.n, rows, o, mask=(1, 1, 1, 1),
                                 n_splits=3, workspace=wsr)
     rw3()
-    t_r3 = timed(torch, rw3, reps, stream)
+    t_r3 = graph_timed(torch, rw3, reps, stream)
     out["rows_quarter_runway"] = {"us_per_call": t_r * 1e3, "us_per_call_3_key_splits": t_r3 * 1e3,
                                   "rows": int(rows.numel()), "of": w.n, "mask": "token-causal"}
     # content memory: M = 2,048 keys drawn as history at earlier positions
@@ -459,9 +476,9 @@ def next_rows_timing(torch, kv, inputs, dev, stream, reps: int = 10) -> dict:
         kv.kv_memory_select(mem, mm, fifo, mf, first, w.n, M, frame_len, dst, kept=kept)
     mass()
     select()
-    t_att = timed(torch, att, reps, stream)
-    t_mass = timed(torch, mass, reps, stream)
-    t_sel = timed(torch, select, reps, stream)
+    t_att = graph_timed(torch, att, reps, stream)
+    t_mass = graph_timed(torch, mass, reps, stream)
+    t_sel = graph_timed(torch, select, reps, stream)
     out["content_memory_runway"] = {
         "attention_fifo_plus_memory_us": t_att * 1e3, "key_mass_us": t_mass * 1e3,
         "select_and_gather_us": t_sel * 1e3, "memory_keys": M, "fifo_block": w.n,
