@@ -5,10 +5,11 @@
 //
 // key_mass_kernel: mass_h[h][c] = sum over query rows i of exp(s_ihc - lse_ih), the
 // probability head h of row i gives candidate key c in the attention call whose
-// log-sum-exp `lse` the caller passes.  One CTA takes 128 candidate keys of one head and
-// computes S^T = K Q^T on the tensor core (M = 128 keys, N = 128 queries per tile, the
-// query split exactly into e4m3 hi + lo as in the attention kernel), so every thread owns
-// one key as its tensor-memory lane and sums its own row: no cross-thread reduction.
+// log-sum-exp `lse` the caller passes.  One CTA takes 4 groups of 128 candidate keys of
+// one head (512 threads) and computes S^T = K Q^T on the tensor core (M = 128 keys per
+// group, N = 128 queries per tile, the query split exactly into e4m3 hi + lo as in the
+// attention kernel, once per tile for all 512 keys), so every thread owns one key as its
+// tensor-memory lane and sums its own row: no cross-thread reduction.
 //
 // memory_select_kernel: one CTA ranks the candidates (quality = sum over heads of the
 // masses; the k-th best key of a frame scores quality * gamma^k; ties toward the lower
@@ -27,13 +28,14 @@ namespace kvring {
 namespace {
 
 constexpr int D = 128;
-constexpr int KM = 128;          // candidate keys per CTA (tensor-memory lanes)
+constexpr int KM = 128;          // candidate keys per group (tensor-memory lanes)
+constexpr int KG = 4;            // groups per CTA: 512 candidates share each query tile's split
 constexpr int QN = 128;          // query rows per tile (MMA N)
-constexpr int kThreads = 128;
+constexpr int kThreads = 32 * 4 * KG;   // warp w: lane quadrant w % 4 of group w / 4
 
 struct MassLayout {
-  static constexpr uint32_t k = 0;                    // e4m3 [128 keys][128], sw128
-  static constexpr uint32_t qhi = k + KM * D;         // e4m3 [128 queries][128], sw128
+  static constexpr uint32_t k = 0;                    // KG x e4m3 [128 keys][128], sw128
+  static constexpr uint32_t qhi = k + KG * KM * D;    // e4m3 [128 queries][128], sw128
   static constexpr uint32_t qlo = qhi + QN * D;
   static constexpr uint32_t rq = qlo + QN * D;        // per query: r (the split's power of two)
   static constexpr uint32_t lq = rq + QN * 4;         // per query: lse * log2(e), or +inf
@@ -56,13 +58,15 @@ __global__ void __launch_bounds__(kThreads, 1) key_mass_kernel(const KeyMassArgs
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + MassLayout::misc);
   float* rq = reinterpret_cast<float*>(sm + MassLayout::rq);
   float* lq = reinterpret_cast<float*>(sm + MassLayout::lq);
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int grp = warp >> 2, quad = warp & 3;
+  const int krow = 32 * quad + lane;                   // TMEM lane = row in group grp
   const int h = blockIdx.y;
-  const int c = blockIdx.x * KM + tid;                 // this thread's candidate
+  const int c = blockIdx.x * (KG * KM) + grp * KM + krow;   // this thread's candidate
   const bool live_c = c < a.n_cand;
 
   if (warp == 0) {
-    tmem_alloc(tmem_slot, 128);
+    tmem_alloc(tmem_slot, KG * 128);
     tmem_relinquish();
   }
   if (tid == 32) {
@@ -85,16 +89,17 @@ __global__ void __launch_bounds__(kThreads, 1) key_mass_kernel(const KeyMassArgs
 #pragma unroll
       for (int i = 0; i < 8; ++i) w[i] = make_uint4(0u, 0u, 0u, 0u);
     }
+    uint8_t* krow_sm = sm + MassLayout::k + grp * KM * D + krow * 128;
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-      *reinterpret_cast<uint4*>(sm + MassLayout::k + tid * 128 + ((i ^ (tid & 7)) << 4)) = w[i];
+      *reinterpret_cast<uint4*>(krow_sm + ((i ^ (krow & 7)) << 4)) = w[i];
   }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+  const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
   constexpr uint32_t idS = idesc_e4m3_f32(KM, QN);
   const uint64_t dK = smem_desc_sw128(smem_u32(sm + MassLayout::k), 16, 1024);
   const uint64_t dQhi = smem_desc_sw128(smem_u32(sm + MassLayout::qhi), 16, 1024);
@@ -178,11 +183,15 @@ __global__ void __launch_bounds__(kThreads, 1) key_mass_kernel(const KeyMassArgs
     tc_fence_after();
     if (tid < 32) {                                   // warp 0; one elected lane issues
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const uint64_t qd = hf == 0 ? dQhi : dQlo;
+      for (int gg = 0; gg < KG; ++gg) {
+        const uint64_t kd = dK + ((gg * KM * D) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < D / 32; ++kk)
-          el_mma_f8_ss(tmem, dK + 2 * kk, qd + 2 * kk, idS, (hf | kk) != 0);
+        for (int hf = 0; hf < 2; ++hf) {
+          const uint64_t qd = hf == 0 ? dQhi : dQlo;
+#pragma unroll
+          for (int kk = 0; kk < D / 32; ++kk)
+            el_mma_f8_ss(tmem + 128 * gg, kd + 2 * kk, qd + 2 * kk, idS, (hf | kk) != 0);
+        }
       }
       el_commit(bar);
     }
@@ -192,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1) key_mass_kernel(const KeyMassArgs
 #pragma unroll 1
       for (int cb = 0; cb < QN; cb += 32) {
         uint32_t sr[32];
-        tmem_ld32(tmem + lane_base + cb, sr);
+        tmem_ld32(tmem + lane_base + 128 * grp + cb, sr);
         tmem_wait_ld();
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
@@ -215,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1) key_mass_kernel(const KeyMassArgs
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, KG * 128);
   }
 }
 
@@ -438,7 +447,7 @@ int launch_key_mass(const KeyMassArgs& a, cudaStream_t s) {
   if (!smem_attr_set(reinterpret_cast<const void*>(key_mass_kernel), (int)MassLayout::bytes,
                      configured))
     return KV_ECUDA;
-  const dim3 grid((unsigned)((a.n_cand + KM - 1) / KM), (unsigned)a.H);
+  const dim3 grid((unsigned)((a.n_cand + KG * KM - 1) / (KG * KM)), (unsigned)a.H);
   key_mass_kernel<<<grid, kThreads, MassLayout::bytes, s>>>(a);
   return cudaPeekAtLastError() == cudaSuccess ? KV_OK : KV_ECUDA;
 }
