@@ -289,10 +289,13 @@ KV_API int chunk_attention_split(const kv_ring_t* kv, const void* q, int n_q, in
  * rings[1 .. n_rings) is history: always visible, cache_bias added.  The result is softmax
  * attention over the union of all rings' valid slots, with chunk_attention's contract for
  * out, lse, mask, softmax_scale and flags.
- * Each ring's keys are split over n_splits groups as in chunk_attention_split.  All
- * partials go to one workspace of at least chunk_attention_workspace_size(n_q, H, 128,
+ * One launch reads every ring (each CTA visits the main ring's key tiles, then the extra
+ * rings', under one online softmax).  The keys of all rings together are split over
+ * n_splits groups as in chunk_attention_split; with n_splits > 1 the partials go to the
+ * workspace and one merge writes out and lse, with n_splits = 1 the kernel writes them
+ * itself.  The workspace must hold at least chunk_attention_workspace_size(n_q, H, 128,
  * n_rings * n_splits) bytes (device, 16-byte aligned, caller-owned, uninitialised is
- * fine), and one merge writes out and lse.
+ * fine); the launch uses its first n_splits slices.
  * rings: host array of n_rings (1..KV_MAX_RINGS) initialised rings with equal n_heads,
  * head_dim (128) and rope_base.  Each ring's RoPE table must cover q_pos0 .. q_pos0 + n_q - 1;
  * the queries are rotated once per ring from that ring's table, so the tables must hold the

@@ -49,6 +49,10 @@
 //    every MMA has completed), so whole 256-byte output rows leave in coalesced stores.
 //  * Split over keys (gridDim.z > 1): each CTA takes a contiguous share of the valid
 //    tiles and writes fp32 partials (O G, m, l); split_combine_kernel merges them.
+//  * Several rings (kMulti): after the main ring's tiles a CTA visits the tiles of up to
+//    KV_MAX_RINGS - 1 history-only rings (a persistent anchor, a content memory) in the
+//    same pipeline, with each ring's tensor maps, scales and valid range; one softmax
+//    covers them all.
 //  * Keys are visited in physical slot order; the ring wrap costs nothing (attention
 //    does not depend on key order once bias and mask are per key).  A CTA skips the
 //    newest current-chunk keys that the block-causal mask hides from all of its rows.
@@ -178,6 +182,53 @@ __device__ __forceinline__ int slot_age(int slot, int newest, int C) {
   return age < 0 ? age + C : age;
 }
 
+// Tensor maps (K and V codes, 128-byte swizzle) of the history-only rings that follow the
+// main ring in one launch.
+struct ExtraMaps {
+  CUtensorMap k[KV_MAX_RINGS - 1];
+  CUtensorMap v[KV_MAX_RINGS - 1];
+};
+
+// One key tile of the launch: ring r (0 = main ring), tile t of that ring, and the ring's
+// scales, capacity and valid range.
+struct KeyTile {
+  int r, t, C, newest, n_valid;
+  const float* ks;
+  const float* vs;
+};
+
+// Tile k of the CTA's sequence: the main ring's visited tiles first, then each extra
+// ring's valid tiles in order (kMulti: the launch reads extra rings).
+template <bool kMulti>
+__device__ __forceinline__ KeyTile key_tile(const AttnArgs& a, const TileSeq& seq0, int k) {
+  KeyTile kt;
+  if (!kMulti || k < seq0.count) {
+    kt.r = 0;
+    kt.t = seq0.tile(k);
+    kt.C = a.C;
+    kt.newest = (int)a.newest_slot;
+    kt.n_valid = (int)a.n_valid;
+    kt.ks = a.k_scale;
+    kt.vs = a.v_scale;
+    return kt;
+  }
+  k -= seq0.count;
+  int x = 0;
+  for (; x < a.n_extra - 1; ++x) {
+    const int cnt = TileSeq(a.x_C[x], a.x_newest[x], a.x_n_valid[x]).count;
+    if (k < cnt) break;
+    k -= cnt;
+  }
+  kt.r = 1 + x;
+  kt.t = TileSeq(a.x_C[x], a.x_newest[x], a.x_n_valid[x]).tile(k);
+  kt.C = a.x_C[x];
+  kt.newest = a.x_newest[x];
+  kt.n_valid = a.x_n_valid[x];
+  kt.ks = a.x_k_scale[x];
+  kt.vs = a.x_v_scale[x];
+  return kt;
+}
+
 // ------------------------------------------------------------------ query prologue
 // 8 lanes per row, 16 consecutive elements per lane (one 16-byte chunk of the e4m3 row).
 __device__ __forceinline__ void q_load16(const AttnArgs& a, int gi, int h, int lc, uint4 (&qr)[2],
@@ -283,10 +334,11 @@ __device__ __forceinline__ float q_quant16(const float (&y)[16], float amax, uin
 // running maximum (p <= 1), and P''.V runs as kind::f8f6f4 MMAs that read the V codes
 // straight from their TMA stage (an MN-major e4m3 operand): no converter work, half the
 // tensor time of the f16 product, and e4m3's 2^-4 relative rounding on every P element.
-template <bool kPv8, bool kModeB>
+template <bool kPv8, bool kModeB, bool kMulti>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_attn_sm100_kernel(const __grid_constant__ CUtensorMap tmk,
-                            const __grid_constant__ CUtensorMap tmv, const AttnArgs a) {
+                            const __grid_constant__ CUtensorMap tmv,
+                            const __grid_constant__ ExtraMaps xm, const AttnArgs a) {
   constexpr float kThr = kPv8 ? 0.f : kRescaleLog2;   // lazy-maximum threshold (log2)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>(
@@ -321,14 +373,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (newest_v < 0) newest_v += C;
     }
   }
-  // this CTA's slice of the visited tiles (all of them unless split over keys)
+  // this CTA's slice of the visited tiles (all of them unless split over keys): the main
+  // ring's, then those of every extra (history-only) ring
   const TileSeq seq(C, newest_v, n_visit);
+  int n_total = seq.count;
+  if (kMulti)
+    for (int x = 0; x < a.n_extra; ++x)
+      n_total += TileSeq(a.x_C[x], a.x_newest[x], a.x_n_valid[x]).count;
   int j0, n_mine;
   {
-    const int per = (seq.count + (int)gridDim.z - 1) / (int)gridDim.z;
-    j0 = min(seq.count, (int)blockIdx.z * per);
-    n_mine = min(seq.count, j0 + per) - j0;
+    const int per = (n_total + (int)gridDim.z - 1) / (int)gridDim.z;
+    j0 = min(n_total, (int)blockIdx.z * per);
+    n_mine = min(n_total, j0 + per) - j0;
   }
+  auto tmap_k = [&](int r) -> const CUtensorMap* { return !kMulti || r == 0 ? &tmk : &xm.k[r - 1]; };
+  auto tmap_v = [&](int r) -> const CUtensorMap* { return !kMulti || r == 0 ? &tmv : &xm.v[r - 1]; };
 
   if (warp == 0) {
     tmem_alloc(tmem_slot, 512);
@@ -364,11 +423,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmk);
     prefetch_tmap(&tmv);
     for (int j = 0; j < n_pre; ++j) {
-      const int t = seq.tile(j0 + j);
+      const KeyTile kt = key_tile<kMulti>(a, seq, j0 + j);
       mbar_arrive_expect_tx(bars.kfull(j), BN * D);
-      tma_load_3d(sm + Layout::kbuf + j * BN * D, &tmk, bars.kfull(j), 0, t * BN, h);
+      tma_load_3d(sm + Layout::kbuf + j * BN * D, tmap_k(kt.r), bars.kfull(j), 0, kt.t * BN, h);
       mbar_arrive_expect_tx(bars.vfull(j), BN * D);
-      tma_load_3d(sm + Layout::vcode + j * BN * D, &tmv, bars.vfull(j), 0, t * BN, h);
+      tma_load_3d(sm + Layout::vcode + j * BN * D, tmap_v(kt.r), bars.vfull(j), 0, kt.t * BN, h);
     }
     *n_issued = n_pre;
   }
@@ -378,7 +437,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   // their bits.  Up to 16 loads per thread are in flight at once.
   {
     float mx = 0.f;
-    const float* vsrow = a.v_scale + (size_t)h * C;
     const int n_slots = n_mine * BN;
     for (int base = 0; base < n_slots; base += 16 * kThreads) {
       float v[16];
@@ -387,8 +445,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int i = base + u * kThreads + tid;
         v[u] = 0.f;
         if (i < n_slots) {
-          const int slot = seq.tile(j0 + i / BN) * BN + (i % BN);
-          if (slot < C && slot_age(slot, newest, C) < n_valid) v[u] = __ldg(vsrow + slot);
+          const KeyTile kt = key_tile<kMulti>(a, seq, j0 + i / BN);
+          const int slot = kt.t * BN + (i % BN);
+          if (slot < kt.C && slot_age(slot, kt.newest, kt.C) < kt.n_valid)
+            v[u] = __ldg(kt.vs + (size_t)h * kt.C + slot);
         }
       }
 #pragma unroll
@@ -473,31 +533,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the prologue); all lanes: the per-key info of tile j, two keys per lane, with the
     // next tile's scales loaded while this one is written.
     auto load_scales = [&](int j, float (&ks)[2], float (&vs)[2]) {
-      const int t = j < n_mine ? seq.tile(j0 + j) : 0;
+      const KeyTile kt = key_tile<kMulti>(a, seq, j < n_mine ? j0 + j : 0);
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int slot = t * BN + lane + 32 * e;
-        const bool in_ring = j < n_mine && slot < C;
-        ks[e] = in_ring ? __ldg(a.k_scale + (size_t)h * C + slot) : 0.f;
-        vs[e] = in_ring ? __ldg(a.v_scale + (size_t)h * C + slot) : 0.f;
+        const int slot = kt.t * BN + lane + 32 * e;
+        const bool in_ring = j < n_mine && slot < kt.C;
+        ks[e] = in_ring ? __ldg(kt.ks + (size_t)h * kt.C + slot) : 0.f;
+        vs[e] = in_ring ? __ldg(kt.vs + (size_t)h * kt.C + slot) : 0.f;
       }
     };
     float pks[2], pvs[2];
     load_scales(0, pks, pvs);
     for (int j = 0; j < n_mine; ++j) {
-      const int t = seq.tile(j0 + j);
+      const KeyTile kt = key_tile<kMulti>(a, seq, j0 + j);
+      const int t = kt.t;
       bool ok = true;
       if (lane == 0 && j >= n_pre) {
         const int sk = j % NK, sv = j % NV;
         ok = j < NK || wait(bars.kempty(sk), ((j / NK) - 1) & 1);
         if (ok) {
           mbar_arrive_expect_tx(bars.kfull(sk), BN * D);
-          tma_load_3d(sm + Layout::kbuf + sk * BN * D, &tmk, bars.kfull(sk), 0, t * BN, h);
+          tma_load_3d(sm + Layout::kbuf + sk * BN * D, tmap_k(kt.r), bars.kfull(sk), 0, t * BN, h);
           ok = j < NV || wait(bars.vempty(sv), ((j / NV) - 1) & 1);
         }
         if (ok) {
           mbar_arrive_expect_tx(bars.vfull(sv), BN * D);
-          tma_load_3d(sm + Layout::vcode + sv * BN * D, &tmv, bars.vfull(sv), 0, t * BN, h);
+          tma_load_3d(sm + Layout::vcode + sv * BN * D, tmap_v(kt.r), bars.vfull(sv), 0, t * BN, h);
           *n_issued = j + 1;          // tile j's K and V loads are both out
         } else if (*n_issued == j) {
           // K(j) went out but V(j) did not: count K(j) alone (the drain waits on it)
@@ -514,12 +575,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kk = lane + 32 * e, slot = t * BN + kk;
         float ksv = 0.f, kbv = -INFINITY, wv = 0.f;
         int tok = kInvalidTok;
-        if (slot < C) {
-          const int age = slot_age(slot, newest, C);
-          if (age < n_valid) {
+        if (slot < kt.C) {
+          const int age = slot_age(slot, kt.newest, kt.C);
+          if (age < kt.n_valid) {
             ksv = pks[e] * a.score_scale_log2;
             wv = pvs[e] * vnorm_inv * (kPv8 ? 256.f : 1.f);   // exact: powers of two
-            if (age < a.n_current) {
+            if (kt.r == 0 && age < a.n_current) {           // current chunk: main ring only
               kbv = 0.f;
               tok = a.n_current - 1 - age;
             } else {
@@ -627,9 +688,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // stage when its slot is invalid (stale memory must not reach the MMA: 0 * NaN = NaN).
     const int ct = tid - 32 * kWarpConv;          // 0..63
     for (int j = 0; j < n_mine; ++j) {
-      const int t = seq.tile(j0 + j);
-      const int slot = t * BN + ct;
-      const bool dead = !(slot < C && slot_age(slot, newest, C) < n_valid);
+      const KeyTile kt = key_tile<kMulti>(a, seq, j0 + j);
+      const int slot = kt.t * BN + ct;
+      const bool dead = !(slot < kt.C && slot_age(slot, kt.newest, kt.C) < kt.n_valid);
       const int sv = j % NV, b = j % NB;
       bool ok = wait(bars.vfull(sv), (j / NV) & 1);
       if (!kPv8) ok = ok && (j < NB || wait(bars.vhempty(b), ((j / NB) - 1) & 1));
@@ -1060,23 +1121,33 @@ int launch_split_combine(const AttnArgs& a, int D_, int n_splits, cudaStream_t s
 }
 
 int launch_attention_sm100_d128(const AttnArgs& a, const void* tmap_k_sw128,
-                                const void* tmap_v_sw128, cudaStream_t s, int n_splits) {
-  // one instance per (e4m3 P, mode B) pair
-  using Kernel = void (*)(const CUtensorMap, const CUtensorMap, const AttnArgs);
-  static const Kernel kernels[4] = {chunk_attn_sm100_kernel<false, false>,
-                                    chunk_attn_sm100_kernel<false, true>,
-                                    chunk_attn_sm100_kernel<true, false>,
-                                    chunk_attn_sm100_kernel<true, true>};
-  static unsigned char configured[4][kMaxDevices] = {};
-  const int which = (a.pv_fp8 ? 2 : 0) + (a.mode_b ? 1 : 0);
+                                const void* tmap_v_sw128, cudaStream_t s, int n_splits,
+                                const void* const* x_tmap_k, const void* const* x_tmap_v) {
+  // one instance per (e4m3 P, mode B, extra rings) triple
+  using Kernel = void (*)(const CUtensorMap, const CUtensorMap, const ExtraMaps, const AttnArgs);
+  static const Kernel kernels[8] = {
+      chunk_attn_sm100_kernel<false, false, false>, chunk_attn_sm100_kernel<false, true, false>,
+      chunk_attn_sm100_kernel<true, false, false>,  chunk_attn_sm100_kernel<true, true, false>,
+      chunk_attn_sm100_kernel<false, false, true>,  chunk_attn_sm100_kernel<false, true, true>,
+      chunk_attn_sm100_kernel<true, false, true>,   chunk_attn_sm100_kernel<true, true, true>};
+  static unsigned char configured[8][kMaxDevices] = {};
+  const int which = (a.n_extra > 0 ? 4 : 0) + (a.pv_fp8 ? 2 : 0) + (a.mode_b ? 1 : 0);
   const Kernel fn = kernels[which];
   if (!smem_attr_set(reinterpret_cast<const void*>(fn), (int)Layout::bytes, configured[which]))
     return KV_ECUDA;
+  if (a.n_extra < 0 || a.n_extra > KV_MAX_RINGS - 1 || (a.n_extra > 0 && (!x_tmap_k || !x_tmap_v)))
+    return KV_EINVAL;
   CUtensorMap mk, mv;
   memcpy(&mk, tmap_k_sw128, sizeof(mk));
   memcpy(&mv, tmap_v_sw128, sizeof(mv));
+  ExtraMaps xm;
+  memset(&xm, 0, sizeof(xm));
+  for (int x = 0; x < a.n_extra; ++x) {
+    memcpy(&xm.k[x], x_tmap_k[x], sizeof(CUtensorMap));
+    memcpy(&xm.v[x], x_tmap_v[x], sizeof(CUtensorMap));
+  }
   dim3 grid((a.n_rows + BM - 1) / BM, a.H, n_splits);
-  fn<<<grid, kThreads, Layout::bytes, s>>>(mk, mv, a);
+  fn<<<grid, kThreads, Layout::bytes, s>>>(mk, mv, xm, a);
   return cudaPeekAtLastError() == cudaSuccess ? KV_OK : KV_ECUDA;
 }
 

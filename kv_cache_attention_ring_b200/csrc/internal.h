@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/kvring.h"
+
 namespace kvring {
 
 struct WriteArgs {
@@ -56,6 +58,14 @@ struct AttnArgs {
   // unnormalised O [split][n_q][H][D] and (m, l) [split][H][n_q] (log2 units) there
   float* part_o;
   float* part_ml;
+  // history-only rings read after the main ring in the same launch (chunk_attention_multi):
+  // their scales [H][C], capacity, newest valid slot and number of valid slots
+  int n_extra;
+  const float* x_k_scale[KV_MAX_RINGS - 1];
+  const float* x_v_scale[KV_MAX_RINGS - 1];
+  int x_C[KV_MAX_RINGS - 1];
+  int x_newest[KV_MAX_RINGS - 1];
+  int x_n_valid[KV_MAX_RINGS - 1];
 };
 
 // Attention mass received by n_cand consecutive slots (from slot_first, mod C) of one
@@ -116,7 +126,9 @@ int launch_rotate(const RotateArgs& a, int D, cudaStream_t s);
 int launch_attention(const AttnArgs& a, int D, const void* tmap_k, const void* tmap_v,
                      const void* tmap_k_sw128, const void* tmap_v_sw128, cudaStream_t s);
 int launch_attention_sm100_d128(const AttnArgs& a, const void* tmap_k_sw128,
-                                const void* tmap_v_sw128, cudaStream_t s, int n_splits = 1);
+                                const void* tmap_v_sw128, cudaStream_t s, int n_splits = 1,
+                                const void* const* x_tmap_k = nullptr,
+                                const void* const* x_tmap_v = nullptr);
 // Merge split partials into out (bf16) and lse.
 int launch_split_combine(const AttnArgs& a, int D, int n_splits, cudaStream_t s);
 

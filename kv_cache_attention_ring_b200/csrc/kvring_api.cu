@@ -398,6 +398,7 @@ int attention_args(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0, 
   a->timeouts = nullptr;
   a->part_o = nullptr;
   a->part_ml = nullptr;
+  a->n_extra = 0;
   a->mode_b = (flags & KV_QK_FP8) ? 1 : 0;
   a->pv_fp8 = (flags & KV_PV_FP8) ? 1 : 0;
   a->rows = nullptr;
@@ -541,24 +542,32 @@ int chunk_attention_multi(const kv_ring_t* const* rings, int n_rings, const void
   const size_t need = chunk_attention_workspace_size(n_q, H, D, S);
   if (!workspace || !aligned16(workspace)) return KV_EINVAL;
   if (workspace_bytes < need) return KV_ERANGE;
-  // partials of all rings in one workspace: O as [S][n_q][H][D], then (m, l) as
-  // [S][H][n_q]; ring r owns splits [r * n_splits, (r + 1) * n_splits)
-  float* const part_o = static_cast<float*>(workspace);
-  float* const part_ml = part_o + (size_t)S * n_q * H * D;
   if (int rc = attach_timeouts(&a[0])) return rc;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  for (int r = 0; r < n_rings; ++r) {
-    a[r].timeouts = a[0].timeouts;
-    a[r].part_o = part_o + (size_t)r * n_splits * n_q * H * D;
-    a[r].part_ml = part_ml + (size_t)r * n_splits * n_q * H * 2;
-    const int rc = launch_attention_sm100_d128(a[r], rings[r]->opaque + kOpaqueTmapKsw,
-                                               rings[r]->opaque + kOpaqueTmapVsw, s, n_splits);
-    if (rc) return rc;
-  }
+  // One launch reads every ring: each CTA visits the main ring's tiles, then the extra
+  // rings' (all history).  The CTAs' fp32 partials go to the workspace only when the
+  // keys are split; otherwise the kernel writes out and lse itself.
   AttnArgs m = a[0];
-  m.part_o = part_o;
-  m.part_ml = part_ml;
-  return launch_split_combine(m, D, S, s);
+  const void* xk[KV_MAX_RINGS - 1];
+  const void* xv[KV_MAX_RINGS - 1];
+  m.n_extra = n_rings - 1;
+  for (int r = 1; r < n_rings; ++r) {
+    m.x_k_scale[r - 1] = a[r].k_scale;
+    m.x_v_scale[r - 1] = a[r].v_scale;
+    m.x_C[r - 1] = a[r].C;
+    m.x_newest[r - 1] = (int)a[r].newest_slot;
+    m.x_n_valid[r - 1] = (int)a[r].n_valid;
+    xk[r - 1] = rings[r]->opaque + kOpaqueTmapKsw;
+    xv[r - 1] = rings[r]->opaque + kOpaqueTmapVsw;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (n_splits > 1) {
+    m.part_o = static_cast<float*>(workspace);
+    m.part_ml = m.part_o + (size_t)n_splits * n_q * H * D;
+  }
+  int rc = launch_attention_sm100_d128(m, rings[0]->opaque + kOpaqueTmapKsw,
+                                       rings[0]->opaque + kOpaqueTmapVsw, s, n_splits, xk, xv);
+  if (rc || n_splits == 1) return rc;
+  return launch_split_combine(m, D, n_splits, s);
 }
 
 int chunk_key_mass(const kv_ring_t* main_ring, const kv_ring_t* cand_ring, const void* q,
