@@ -297,9 +297,10 @@ KV_API int chunk_attention_split(const kv_ring_t* kv, const void* q, int n_q, in
  * n_rings * n_splits) bytes (device, 16-byte aligned, caller-owned, uninitialised is
  * fine); the launch uses its first n_splits slices.
  * rings: host array of n_rings (1..KV_MAX_RINGS) initialised rings with equal n_heads,
- * head_dim (128) and rope_base.  Each ring's RoPE table must cover q_pos0 .. q_pos0 + n_q - 1;
- * the queries are rotated once per ring from that ring's table, so the tables must hold the
- * same angles (kv_rope_table_build with that base).  n_rings * n_splits <= 64.
+ * head_dim (128) and rope_base.  Each ring's RoPE table must cover q_pos0 .. q_pos0 + n_q - 1
+ * (checked); the queries are rotated once, from rings[0]'s table, and every ring's keys
+ * were rotated with the same angles (kv_rope_table_build with that base).
+ * n_rings * n_splits <= 64.
  * Errors, all before anything is enqueued: KV_EINVAL (rings null or n_rings out of range,
  * a null entry, n_splits out of range, rings that differ in heads, head_dim or base, the
  * errors of chunk_attention_split), KV_EUNSUPPORTED (head_dim 64), KV_ERANGE (workspace too
