@@ -254,27 +254,89 @@ __device__ __forceinline__ bool before_in_score(const Cand& x, const Cand& y) {
   return x.idx < y.idx;
 }
 
-// In-place bitonic sort of n_pow2 entries (padding entries sort last), all threads.
+// Bitonic sort of n_pow2 <= 4 * kSelThreads entries of v (padding entries sort last), all
+// threads.  Thread t holds entries 4t .. 4t + 3 in registers: pairs closer than 4 entries
+// are exchanged in registers, pairs up to 128 apart through warp shuffles, and only the
+// wider strides go through shared memory (one barrier each).
+template <bool kByFrame>
+__device__ __forceinline__ bool before(const Cand& x, const Cand& y) {
+  return kByFrame ? before_in_frame(x, y) : before_in_score(x, y);
+}
+__device__ __forceinline__ Cand shfl_cand(const Cand& c, int lane_mask) {
+  Cand o;
+  o.q = __shfl_xor_sync(0xffffffffu, c.q, lane_mask);
+  o.idx = __shfl_xor_sync(0xffffffffu, c.idx, lane_mask);
+  o.pos = __shfl_xor_sync(0xffffffffu, c.pos, lane_mask);
+  o.frame = __shfl_xor_sync(0xffffffffu, c.frame, lane_mask);
+  return o;
+}
 template <bool kByFrame>
 __device__ void bitonic(Cand* v, int n_pow2) {
+  const int tid = threadIdx.x;
+  const bool live = 4 * tid < n_pow2;                  // threads past the entries idle
+  Cand x[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) x[k] = live ? v[4 * tid + k] : v[0];
   for (int size = 2; size <= n_pow2; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int t = threadIdx.x; t < (n_pow2 >> 1); t += blockDim.x) {
-        // t-th pair: i has bit `stride` clear, j = i + stride
-        const int i = ((t & ~(stride - 1)) << 1) | (t & (stride - 1));
-        const int j = i + stride;
-        const Cand x = v[i], y = v[j];
-        const bool up = (i & size) == 0;
-        const bool swap = kByFrame ? (up ? before_in_frame(y, x) : before_in_frame(x, y))
-                                   : (up ? before_in_score(y, x) : before_in_score(x, y));
-        if (swap) {
-          v[i] = y;
-          v[j] = x;
+    int stride = size >> 1;
+    if (stride >= 128) {                               // wide strides: shared memory
+      if (live) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) v[4 * tid + k] = x[k];
+      }
+      __syncthreads();
+      for (; stride >= 128; stride >>= 1) {
+        for (int t = tid; t < (n_pow2 >> 1); t += blockDim.x) {
+          const int i = ((t & ~(stride - 1)) << 1) | (t & (stride - 1));
+          const int j = i + stride;
+          const Cand a = v[i], b = v[j];
+          const bool up = (i & size) == 0;
+          if (up ? before<kByFrame>(b, a) : before<kByFrame>(a, b)) {
+            v[i] = b;
+            v[j] = a;
+          }
         }
+        __syncthreads();
+      }
+      if (live) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) x[k] = v[4 * tid + k];
       }
       __syncthreads();
     }
+    for (; stride >= 4; stride >>= 1) {                // within the warp: shuffles
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int e = 4 * tid + k;
+        const Cand o = shfl_cand(x[k], stride >> 2);
+        const bool lower = (e & stride) == 0, up = (e & size) == 0;
+        const bool mine_first = before<kByFrame>(x[k], o);
+        // the lower entry keeps the first of the pair (descending runs: the last)
+        const bool keep_mine = (lower == up) ? mine_first : !mine_first;
+        if (live && !keep_mine) x[k] = o;
+      }
+    }
+    // within the thread: strides 2 and 1
+    auto cx = [&](Cand& a, Cand& b, int e) {
+      const bool up = (e & size) == 0;
+      if (up ? before<kByFrame>(b, a) : before<kByFrame>(a, b)) {
+        const Cand t = a;
+        a = b;
+        b = t;
+      }
+    };
+    if (size >= 4) {
+      cx(x[0], x[2], 4 * tid);
+      cx(x[1], x[3], 4 * tid + 1);
+    }
+    cx(x[0], x[1], 4 * tid);
+    cx(x[2], x[3], 4 * tid + 2);
   }
+  if (live) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[4 * tid + k] = x[k];
+  }
+  __syncthreads();
 }
 
 // Block-wide inclusive max-scan of one int per thread (kSelThreads threads).
@@ -310,7 +372,7 @@ __global__ void __launch_bounds__(kSelThreads) memory_select_kernel(const Select
   __shared__ int wpre[KV_MEMORY_MAX_CANDIDATES / 32];
   const int tid = threadIdx.x;
   const int n = a.n_mem + a.n_fifo;
-  int n_pow2 = 1;
+  int n_pow2 = 4;                                    // at least one thread's four entries
   while (n_pow2 < n) n_pow2 <<= 1;
   for (int i = tid; i < n_pow2; i += blockDim.x) {
     Cand c;
@@ -453,7 +515,7 @@ int launch_key_mass(const KeyMassArgs& a, cudaStream_t s) {
 }
 
 size_t select_smem_bytes(int n) {
-  size_t p = 1;
+  size_t p = 4;
   while ((int)p < n) p <<= 1;
   return p * sizeof(Cand);
 }
