@@ -329,6 +329,7 @@ def config_timings(torch, kv, inputs, dev, stream, peaks, reps: int = 10) -> dic
     Wan-style chunk (bias sweep), joint audio+video paths, long-stream chunk."""
     out = {}
     bf16_sus = peaks["bf16_sus"]
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
     # Wan-style: 4 committed chunks + the pending one, 4 passes with bias -3..0
     w = inputs.WAN
     ring = _filled_ring(torch, kv, inputs, w, dev, 4)
@@ -345,7 +346,19 @@ def config_timings(torch, kv, inputs, dev, stream, peaks, reps: int = 10) -> dic
                              "tflops": flop / (ms * 1e-3) / 1e12,
                              "frac_bf16_sustained": flop / (ms * 1e-3) / 1e12 / bf16_sus,
                              "biases": list(w.biases)}
-    del ring, q, k, v, o
+    # the same passes with the keys split as the wave-filling helper suggests
+    z = kv.chunk_attention_suggest_splits(w.n, w.H, w.C, n_sms)
+    ws = torch.empty(kv.chunk_attention_workspace_size(w.n, w.H, w.D, z), dtype=torch.uint8,
+                     device=dev)
+    def wan_z():
+        for b in w.biases:
+            kv.chunk_attention_split(ring, q, ring.next_pos, w.n, z, ws, mask=w.mask,
+                                     cache_bias=b, out=o, want_lse=False)
+    wan_z()
+    ms_z = graph_timed(torch, wan_z, reps, stream, inner=2) / len(w.biases)
+    out["wan_4680x23400"].update({"key_splits": z, "us_per_call_split": ms_z * 1e3,
+                                  "tflops_split": flop / (ms_z * 1e-3) / 1e12})
+    del ring, q, k, v, o, ws
     # joint audio+video: 20 prior blocks in each ring plus the pending block
     wv, wa = inputs.AV_VIDEO, inputs.AV_AUDIO
     # both rings cover the video positions: cross-modal queries keep their own positions
@@ -374,17 +387,27 @@ def config_timings(torch, kv, inputs, dev, stream, peaks, reps: int = 10) -> dic
     t_av = graph_timed(torch, av_, reps, stream)
     t_va = graph_timed(torch, va_, reps, stream)
     t_aa = graph_timed(torch, aa_, reps, stream)
+    z_vv = kv.chunk_attention_suggest_splits(wv.n, wv.H, wv.C, n_sms)
+    ws_vv = torch.empty(kv.chunk_attention_workspace_size(wv.n, wv.H, wv.D, z_vv),
+                        dtype=torch.uint8, device=dev)
+    def vvz_():
+        kv.chunk_attention_split(rv, qv, rv.next_pos, wv.n, z_vv, ws_vv, cache_bias=0.0,
+                                 out=ov, want_lse=False)
+    vvz_()
+    t_vvz = graph_timed(torch, vvz_, reps, stream)
     f_vv = 4 * wv.D * wv.H * wv.n * wv.C
     av_bytes = wv.C * wv.H * (2 * wv.D + 8)          # K, V codes and scales of the video ring
     out["av_v2v_1152x24192"] = {"us_per_call": t_vv * 1e3, "gflop_per_call": f_vv / 1e9,
                                 "tflops": f_vv / (t_vv * 1e-3) / 1e12,
-                                "frac_bf16_sustained": f_vv / (t_vv * 1e-3) / 1e12 / bf16_sus}
+                                "frac_bf16_sustained": f_vv / (t_vv * 1e-3) / 1e12 / bf16_sus,
+                                "key_splits": z_vv, "us_per_call_split": t_vvz * 1e3,
+                                "tflops_split": f_vv / (t_vvz * 1e-3) / 1e12}
     out["av_a2v_25x24192_split16"] = {"us_per_call": t_av * 1e3, "bytes_per_call": av_bytes,
                                       "gbs": av_bytes / (t_av * 1e-3) / 1e9,
                                       "frac_hbm": av_bytes / (t_av * 1e-3) / 1e9 / peaks["hbm"]}
     out["av_v2a_1152x525"] = {"us_per_call": t_va * 1e3}
     out["av_a2a_25x525"] = {"us_per_call": t_aa * 1e3}
-    del rv, ra, ws
+    del rv, ra, ws, ws_vv
     # long stream: a full 32,768-slot ring of Student-t keys/values, a 1,024-token chunk
     w = inputs.STRESS
     ring = _filled_ring(torch, kv, inputs, w, dev, w.C // w.n)
@@ -417,7 +440,17 @@ def config_timings(torch, kv, inputs, dev, stream, peaks, reps: int = 10) -> dic
     t_a4 = graph_timed(torch, at4, reps, stream, inner=2)
     out["stress_1024x32768"]["attn_split4_us"] = t_a4 * 1e3
     out["stress_1024x32768"]["attn_split4_tflops"] = f_a / (t_a4 * 1e-3) / 1e12
-    del ring, ws
+    z = kv.chunk_attention_suggest_splits(w.n, w.H, w.C, n_sms)
+    wsz = torch.empty(kv.chunk_attention_workspace_size(w.n, w.H, w.D, z), dtype=torch.uint8,
+                      device=dev)
+    def atz():
+        kv.chunk_attention_split(ring, q, ring.next_pos, w.n, z, wsz, cache_bias=-4.0,
+                                 out=o, want_lse=False)
+    atz()
+    t_az = graph_timed(torch, atz, reps, stream, inner=2)
+    out["stress_1024x32768"].update({"key_splits": z, "attn_split_us": t_az * 1e3,
+                                     "attn_split_tflops": f_a / (t_az * 1e-3) / 1e12})
+    del ring, ws, wsz
     torch.cuda.synchronize()
     return out
 

@@ -262,6 +262,15 @@ KV_API int chunk_attention_rows(const kv_ring_t* kv, const void* q, int n_q, int
  * 0 for invalid arguments. */
 KV_API size_t chunk_attention_workspace_size(int n_q, int n_heads, int head_dim, int n_splits);
 
+/* Key splits (1..16) for chunk_attention_split on a GPU of n_sms SMs (148 on B200) that
+ * fill it in whole waves: head_dim-128 attention runs one CTA per 256 query rows and
+ * head per SM, so n_q queries x n_heads over n_keys valid slots make
+ * ceil(n_q / 256) * n_heads CTAs of ceil(n_keys / 64) key tiles each.  The choice
+ * minimises waves * (tiles / splits + 10), the 10 standing for a CTA's fixed cost (query
+ * prologue, epilogue, partials) in key tiles; ties go to fewer splits, and no split gets
+ * fewer than 4 key tiles.  Host arithmetic only; 1 for arguments out of range. */
+KV_API int chunk_attention_suggest_splits(int n_q, int n_heads, int64_t n_keys, int n_sms);
+
 /* chunk_attention with the keys split over n_splits (1..64) groups of consecutive valid
  * tiles, for few queries over a long ring (e.g. the 25 audio latents of a 1 s block in
  * "Stream LTX", section "Training", attending a 20-block video ring): every split keeps

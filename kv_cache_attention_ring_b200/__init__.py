@@ -31,7 +31,7 @@ KV_PV_FP8 = 2
 EXPORTS = ("kv_rope_table_build", "kv_rope3d_table_build", "kv_ring_init", "kv_ring_write", "kv_ring_commit",
            "kv_ring_delta_rotate", "chunk_attention", "chunk_attention_workspace_size",
            "chunk_attention_split", "chunk_attention_split_noalloc", "chunk_attention_multi",
-           "chunk_attention_rows", "chunk_key_mass", "kv_memory_select", "kv_status_string",
+           "chunk_attention_rows", "chunk_attention_suggest_splits", "chunk_key_mass", "kv_memory_select", "kv_status_string",
            "kv_wait_timeout_count")
 KV_NOALLOC_SCRATCH_BYTES = 16 << 20
 KV_MEMORY_MAX_CANDIDATES = 8192
@@ -91,6 +91,8 @@ def lib() -> ctypes.CDLL:
                                       ctypes.c_uint32, P]
         L.chunk_attention_rows.argtypes = [P, P, I, I64, I, P, I, P, P, ctypes.c_float, P, P,
                                            I, P, ctypes.c_size_t, ctypes.c_uint32, P]
+        L.chunk_attention_suggest_splits.argtypes = [I, I, I64, I]
+        L.chunk_attention_suggest_splits.restype = I
         L.chunk_key_mass.argtypes = [P, P, P, I, I64, P, P, ctypes.c_float, I64, I, P, P]
         L.kv_memory_select.argtypes = [P, P, P, P, I64, I, I, I64, ctypes.c_float, P, P, P]
         L.kv_status_string.argtypes = [I]
@@ -286,6 +288,11 @@ def chunk_attention_rows(ring: KvRing, q, q_pos0: int, n_current: int, rows, out
                                       KV_QK_FP8 if mode_b else 0, _stream(stream)),
            "chunk_attention_rows")
     return out, lse
+
+
+def chunk_attention_suggest_splits(n_q: int, n_heads: int, n_keys: int, n_sms: int = 148) -> int:
+    """Key splits for chunk_attention_split that fill the GPU in whole waves."""
+    return int(lib().chunk_attention_suggest_splits(int(n_q), int(n_heads), int(n_keys), int(n_sms)))
 
 
 def chunk_attention_workspace_size(n_q: int, n_heads: int, head_dim: int, n_splits: int) -> int:

@@ -470,6 +470,25 @@ size_t chunk_attention_workspace_size(int n_q, int n_heads, int head_dim, int n_
   return (size_t)n_splits * (size_t)n_q * (size_t)n_heads * ((size_t)head_dim * 4 + 8);
 }
 
+int chunk_attention_suggest_splits(int n_q, int n_heads, int64_t n_keys, int n_sms) {
+  if (n_q < 1 || n_heads < 1 || n_keys < 1 || n_sms < 1) return 1;
+  const int64_t units = ((int64_t)n_q + 255) / 256 * n_heads;
+  const int64_t n_tiles = (n_keys + 63) / 64;
+  const double tiles = (double)n_tiles;
+  const int z_max = (int)(n_tiles / 4 < 16 ? (n_tiles / 4 < 1 ? 1 : n_tiles / 4) : 16);
+  int best = 1;
+  double best_cost = 0.0;
+  for (int z = 1; z <= z_max; ++z) {
+    const int64_t waves = (units * z + n_sms - 1) / n_sms;
+    const double cost = (double)waves * (tiles / z + 10.0);
+    if (z == 1 || cost < best_cost) {
+      best = z;
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
 int chunk_attention_split(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
                           int n_current, const kv_block_mask_t* mask,
                           const kv_cache_bias_t* bias, float softmax_scale, void* out,

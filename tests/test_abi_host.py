@@ -276,6 +276,47 @@ def test_split_workspace_size_and_validation(L):
                                    4, 16, need, 0, None) in (kv.KV_EUNSUPPORTED, kv.KV_ECUDA)
 
 
+def _waves_cost(n_q, n_heads, n_keys, n_sms, z):
+    """One wave-filling cost, counted CTA by CTA: the SMs take the CTAs in waves of n_sms,
+    each CTA costs its key tiles plus a fixed 10."""
+    n_cta = -(-n_q // 256) * n_heads * z
+    tiles = -(-n_keys // 64)
+    waves = 0
+    left = n_cta
+    while left > 0:
+        waves += 1
+        left -= n_sms
+    return waves * (tiles / z + 10.0)
+
+
+@pytest.mark.parametrize("n_q,n_heads,n_keys,n_sms", [
+    (757, 40, 5788, 148), (4680, 40, 23400, 148), (1152, 32, 24192, 148),
+    (1024, 40, 32768, 148), (25, 32, 24192, 148), (189, 40, 5788, 148), (256, 1, 1024, 148),
+    (4096, 8, 200000, 132), (1, 1, 100000, 1)])
+def test_suggest_splits_minimises_the_wave_cost(n_q, n_heads, n_keys, n_sms):
+    z = kv.chunk_attention_suggest_splits(n_q, n_heads, n_keys, n_sms)
+    tiles = -(-n_keys // 64)
+    z_max = max(1, min(16, tiles // 4))
+    assert 1 <= z <= z_max
+    costs = {c: _waves_cost(n_q, n_heads, n_keys, n_sms, c) for c in range(1, z_max + 1)}
+    best = min(costs.values())
+    assert costs[z] <= best * (1 + 1e-12)
+    assert all(costs[c] > best * (1 + 1e-12) for c in range(1, z))       # ties: fewest splits
+
+
+def test_suggest_splits_special_cases():
+    # a chunk whose CTAs already fill less than one wave over a short ring is not split
+    assert kv.chunk_attention_suggest_splits(757, 40, 5788, 148) == 1
+    # fewer than 8 key tiles never split; out-of-range arguments give 1
+    assert kv.chunk_attention_suggest_splits(1, 1, 448, 148) == 1
+    assert kv.chunk_attention_suggest_splits(1, 1, 512, 148) == 2
+    for bad in [(0, 1, 100, 148), (1, 0, 100, 148), (1, 1, 0, 148), (1, 1, 100, 0),
+                (-5, 1, 100, 148)]:
+        assert kv.chunk_attention_suggest_splits(*bad) == 1
+    # one query tile, one head, a long ring and a large GPU: the cap of 16 holds
+    assert kv.chunk_attention_suggest_splits(1, 1, 10 ** 7, 148) == 16
+
+
 def test_noalloc_rejects_oversize_before_any_cuda_call(L):
     s = _fake_ring(C=4096, D=128)
     s.live = 2048
