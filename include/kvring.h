@@ -268,7 +268,9 @@ KV_API size_t chunk_attention_workspace_size(int n_q, int n_heads, int head_dim,
  * ceil(n_q / 256) * n_heads CTAs of ceil(n_keys / 64) key tiles each.  The choice
  * minimises waves * (tiles / splits + 10), the 10 standing for a CTA's fixed cost (query
  * prologue, epilogue, partials) in key tiles; ties go to fewer splits, and no split gets
- * fewer than 4 key tiles.  Host arithmetic only; 1 for arguments out of range. */
+ * fewer than 4 key tiles.  Unless that cost is at most 0.9 of the unsplit one, the answer
+ * is 1: the fp32 partials and their merge cost HBM traffic the count leaves out.  Host
+ * arithmetic only; 1 for arguments out of range. */
 KV_API int chunk_attention_suggest_splits(int n_q, int n_heads, int64_t n_keys, int n_sms);
 
 /* chunk_attention with the keys split over n_splits (1..64) groups of consecutive valid

@@ -486,7 +486,9 @@ int chunk_attention_suggest_splits(int n_q, int n_heads, int64_t n_keys, int n_s
       best_cost = cost;
     }
   }
-  return best;
+  // partials and their merge cost HBM traffic the waves leave out: split only for a clear gain
+  const double unsplit = (double)((units + n_sms - 1) / n_sms) * (tiles + 10.0);
+  return best_cost <= 0.9 * unsplit ? best : 1;
 }
 
 int chunk_attention_split(const kv_ring_t* kv, const void* q, int n_q, int64_t q_pos0,
