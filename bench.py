@@ -54,9 +54,11 @@ def parse_args():
                     help="rings per step (60 = the Runway step; fewer for profiler captures)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the rotate, end-to-end and CPU legs (profiler captures)")
-    ap.add_argument("--leg", choices=["all", "rotate"], default="all",
-                    help="rotate: time only the delta rotation of a full 32,768 x 40 ring "
-                         "(one JSON line; for profiler captures of that kernel)")
+    ap.add_argument("--leg", choices=["all", "rotate", "wan", "av", "stress", "next"],
+                    default="all",
+                    help="one leg alone, one JSON line (profiler captures): rotate = the "
+                         "delta rotation of a full 32,768 x 40 ring; wan, av, stress = one "
+                         "workload of the configs; next = gathered rows and content memory")
     return ap.parse_args()
 
 
@@ -328,9 +330,18 @@ def config_timings(torch, kv, inputs, dev, stream, peaks, reps: int = 10) -> dic
     """The other workloads, each timed on its own ring (every ring is larger than L2):
     Wan-style chunk (bias sweep), joint audio+video paths, long-stream chunk."""
     out = {}
+    out.update(wan_timing(torch, kv, inputs, dev, stream, peaks, reps))
+    out.update(av_timing(torch, kv, inputs, dev, stream, peaks, reps))
+    out.update(stress_timing(torch, kv, inputs, dev, stream, peaks, reps))
+    return out
+
+
+def wan_timing(torch, kv, inputs, dev, stream, peaks, reps: int = 10) -> dict:
+    """Wan-style chunk: 4 committed chunks + the pending one, 4 passes with bias -3..0.
+    The first attention launch is the bias -3 pass."""
+    out = {}
     bf16_sus = peaks["bf16_sus"]
     n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    # Wan-style: 4 committed chunks + the pending one, 4 passes with bias -3..0
     w = inputs.WAN
     ring = _filled_ring(torch, kv, inputs, w, dev, 4)
     q, k, v = inputs.chunk_qkv_torch(w, 4, device=dev)
@@ -363,7 +374,16 @@ def config_timings(torch, kv, inputs, dev, stream, peaks, reps: int = 10) -> dic
                                       "tflops_split": flop / (ms_z * 1e-3) / 1e12})
         del ws
     del ring, q, k, v, o
-    # joint audio+video: 20 prior blocks in each ring plus the pending block
+    torch.cuda.synchronize()
+    return out
+
+
+def av_timing(torch, kv, inputs, dev, stream, peaks, reps: int = 10) -> dict:
+    """Joint audio+video paths: 20 prior blocks in each ring plus the pending block.
+    Attention launches in order: v->v, a->v (16 key splits, then the merge), v->a, a->a."""
+    out = {}
+    bf16_sus = peaks["bf16_sus"]
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
     wv, wa = inputs.AV_VIDEO, inputs.AV_AUDIO
     # both rings cover the video positions: cross-modal queries keep their own positions
     rv = _filled_ring(torch, kv, inputs, wv, dev, 20, wv.extra["first_n"], span=2 * wv.C)
@@ -412,7 +432,15 @@ def config_timings(torch, kv, inputs, dev, stream, peaks, reps: int = 10) -> dic
     out["av_v2a_1152x525"] = {"us_per_call": t_va * 1e3}
     out["av_a2a_25x525"] = {"us_per_call": t_aa * 1e3}
     del rv, ra, ws, ws_vv
-    # long stream: a full 32,768-slot ring of Student-t keys/values, a 1,024-token chunk
+    torch.cuda.synchronize()
+    return out
+
+
+def stress_timing(torch, kv, inputs, dev, stream, peaks, reps: int = 10) -> dict:
+    """Long stream: a full 32,768-slot ring of Student-t keys/values, a 1,024-token chunk."""
+    out = {}
+    bf16_sus = peaks["bf16_sus"]
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
     w = inputs.STRESS
     ring = _filled_ring(torch, kv, inputs, w, dev, w.C // w.n)
     q, k, v = inputs.chunk_qkv_torch(w, w.C // w.n, device=dev)
@@ -506,9 +534,9 @@ def next_rows_timing(torch, kv, inputs, dev, stream, reps: int = 10) -> dict:
     mf = torch.empty((w.H, w.n), dtype=torch.float32, device=dev)
     mm = torch.empty((w.H, n_mem), dtype=torch.float32, device=dev)
     kept = torch.empty((M,), dtype=torch.int32, device=dev)
-    def mass():
-        kv.chunk_key_mass(fifo, fifo, q, fifo.next_pos, lse, first, w.n, mass=mf)
-        kv.chunk_key_mass(fifo, mem, q, fifo.next_pos, lse, mem_first, n_mem, mass=mm)
+    def mass():                                          # both sets in one launch
+        kv.chunk_key_mass_multi(fifo, [fifo, mem], q, fifo.next_pos, lse, [first, mem_first],
+                                [w.n, n_mem], masses=[mf, mm])
     def select():
         kv.kv_memory_select(mem, mm, fifo, mf, first, w.n, M, frame_len, dst, kept=kept)
     mass()
@@ -744,6 +772,16 @@ def main():
         if rank == 0:
             print(json.dumps({"leg": "rotate", "shape": "32768 slots x 40 heads x 128", **rot}),
                   flush=True)
+        return
+    if args.leg in ("wan", "av", "stress", "next"):
+        reps = max(1, args.steps)
+        if args.leg == "next":
+            res = next_rows_timing(torch, kv, inputs, dev, stream, reps)
+        else:
+            fn = {"wan": wan_timing, "av": av_timing, "stress": stress_timing}[args.leg]
+            res = fn(torch, kv, inputs, dev, stream, peaks, reps)
+        if rank == 0:
+            print(json.dumps({"leg": args.leg, **res}), flush=True)
         return
 
     step = RunwayStep(torch, kv, inputs, dev, seed=1000 + 2 + rank, rings=args.rings)

@@ -381,6 +381,25 @@ KV_API int chunk_key_mass(const kv_ring_t* main_ring, const kv_ring_t* cand_ring
                           const kv_cache_bias_t* bias, float softmax_scale,
                           int64_t slot_first, int n_cand, float* mass, void* stream);
 
+/* Most candidate sets of one chunk_key_mass_multi call. */
+#define KV_KEY_MASS_MAX_SETS 4
+
+/* chunk_key_mass for n_sets candidate sets of the same attention call in one launch, so
+ * that the CTAs of all sets fill the GPU together (an eviction scores the memory ring's
+ * slots and the FIFO block the next write overwrites).  Set t: the n_cand[t] slots
+ * (slot_first[t] + c) mod capacity of cand_rings[t], masses to mass[t] (device fp32
+ * [H][n_cand[t]]).  Each set's result is bit for bit the one chunk_key_mass gives for it
+ * alone.  cand_rings, slot_first, n_cand and mass are host arrays of n_sets entries,
+ * 1 <= n_sets <= KV_KEY_MASS_MAX_SETS; sets with n_cand 0 are skipped.  Other arguments
+ * and errors as chunk_key_mass, checked for every set before anything is launched;
+ * KV_EINVAL also for n_sets out of range or a null array. */
+KV_API int chunk_key_mass_multi(const kv_ring_t* main_ring, int n_sets,
+                                const kv_ring_t* const* cand_rings, const void* q, int n_q,
+                                int64_t q_pos0, const float* lse,
+                                const kv_cache_bias_t* bias, float softmax_scale,
+                                const int64_t* slot_first, const int* n_cand,
+                                float* const* mass, void* stream);
+
 /* Largest candidate count (memory slots + FIFO block) of one kv_memory_select call. */
 #define KV_MEMORY_MAX_CANDIDATES 8192
 

@@ -74,10 +74,16 @@ struct KeyMassArgs {
   const uint16_t* q;        // bf16 [n_q][H][D]
   const float* rope_q0;     // main ring's table row of q_pos0
   const float* lse;         // [H][n_q] natural log, from the attention call
-  const uint8_t* kc;        // candidate ring codes [H][C][D]
-  const float* ks;          // candidate ring scales [H][C]
-  float* mass;              // [H][n_cand]
-  int n_q, H, C, n_cand, slot_first;
+  int n_q, H;
+  int n_sets;               // candidate sets, 1 .. KV_KEY_MASS_MAX_SETS
+  // set t: candidate ring codes [H][C][D] and scales [H][C], masses [H][n_cand]; its CTAs
+  // are blockIdx.x in [blk_first[t], blk_first[t + 1])
+  const uint8_t* kc[KV_KEY_MASS_MAX_SETS];
+  const float* ks[KV_KEY_MASS_MAX_SETS];
+  float* mass[KV_KEY_MASS_MAX_SETS];
+  int C[KV_KEY_MASS_MAX_SETS], n_cand[KV_KEY_MASS_MAX_SETS];
+  int slot_first[KV_KEY_MASS_MAX_SETS];
+  int blk_first[KV_KEY_MASS_MAX_SETS + 1];
   float score_scale_log2;   // softmax_scale * log2(e)
   float bias_log2;          // history_bias * log2(e)
   unsigned int* timeouts;

@@ -5,8 +5,9 @@
 //
 // key_mass_kernel: mass_h[h][c] = sum over query rows i of exp(s_ihc - lse_ih), the
 // probability head h of row i gives candidate key c in the attention call whose
-// log-sum-exp `lse` the caller passes.  One CTA takes 4 groups of 128 candidate keys of
-// one head (512 threads) and computes S^T = K Q^T on the tensor core (M = 128 keys per
+// log-sum-exp `lse` the caller passes.  One launch may score several candidate sets of
+// that call (their CTAs side by side in the grid).  One CTA takes 4 groups of 128
+// candidate keys of one set and head (512 threads) and computes S^T = K Q^T on the tensor core (M = 128 keys per
 // group, N = 128 queries per tile, the query split exactly into e4m3 hi + lo as in the
 // attention kernel, once per tile for all 512 keys), so every thread owns one key as its
 // tensor-memory lane and sums its own row: no cross-thread reduction.
@@ -62,8 +63,11 @@ __global__ void __launch_bounds__(kThreads, 1) key_mass_kernel(const KeyMassArgs
   const int grp = warp >> 2, quad = warp & 3;
   const int krow = 32 * quad + lane;                   // TMEM lane = row in group grp
   const int h = blockIdx.y;
-  const int c = blockIdx.x * (KG * KM) + grp * KM + krow;   // this thread's candidate
-  const bool live_c = c < a.n_cand;
+  int set = 0;                                         // candidate set of this CTA
+  while (set + 1 < a.n_sets && (int)blockIdx.x >= a.blk_first[set + 1]) ++set;
+  const int n_cand = a.n_cand[set], C = a.C[set];
+  const int c = ((int)blockIdx.x - a.blk_first[set]) * (KG * KM) + grp * KM + krow;
+  const bool live_c = c < n_cand;                      // this thread's candidate
 
   if (warp == 0) {
     tmem_alloc(tmem_slot, KG * 128);
@@ -79,12 +83,12 @@ __global__ void __launch_bounds__(kThreads, 1) key_mass_kernel(const KeyMassArgs
   {
     uint4 w[8];
     if (live_c) {
-      int slot = a.slot_first + c;
-      slot = slot >= a.C ? slot - a.C : slot;
-      const uint4* src = reinterpret_cast<const uint4*>(a.kc + ((size_t)h * a.C + slot) * D);
+      int slot = a.slot_first[set] + c;
+      slot = slot >= C ? slot - C : slot;
+      const uint4* src = reinterpret_cast<const uint4*>(a.kc[set] + ((size_t)h * C + slot) * D);
 #pragma unroll
       for (int i = 0; i < 8; ++i) w[i] = __ldg(src + i);
-      kscl = __ldg(a.ks + (size_t)h * a.C + slot) * a.score_scale_log2;
+      kscl = __ldg(a.ks[set] + (size_t)h * C + slot) * a.score_scale_log2;
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) w[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -219,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1) key_mass_kernel(const KeyMassArgs
     mbar_wait(bar, phase ^ 1, a.timeouts);             // bounded: let an issued MMA land
     acc = __uint_as_float(0x7FC00000u);
   }
-  if (live_c) a.mass[(size_t)h * a.n_cand + c] = acc;
+  if (live_c) a.mass[set][(size_t)h * n_cand + c] = acc;
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -509,8 +513,14 @@ int launch_key_mass(const KeyMassArgs& a, cudaStream_t s) {
   if (!smem_attr_set(reinterpret_cast<const void*>(key_mass_kernel), (int)MassLayout::bytes,
                      configured))
     return KV_ECUDA;
-  const dim3 grid((unsigned)((a.n_cand + KG * KM - 1) / (KG * KM)), (unsigned)a.H);
-  key_mass_kernel<<<grid, kThreads, MassLayout::bytes, s>>>(a);
+  // every set's CTAs in one grid: blk_first is the running sum of their block counts
+  KeyMassArgs b = a;
+  b.blk_first[0] = 0;
+  for (int t = 0; t < b.n_sets; ++t)
+    b.blk_first[t + 1] = b.blk_first[t] + (b.n_cand[t] + KG * KM - 1) / (KG * KM);
+  if (b.blk_first[b.n_sets] == 0) return KV_OK;
+  const dim3 grid((unsigned)b.blk_first[b.n_sets], (unsigned)b.H);
+  key_mass_kernel<<<grid, kThreads, MassLayout::bytes, s>>>(b);
   return cudaPeekAtLastError() == cudaSuccess ? KV_OK : KV_ECUDA;
 }
 

@@ -591,44 +591,72 @@ int chunk_attention_multi(const kv_ring_t* const* rings, int n_rings, const void
   return launch_split_combine(m, D, n_splits, s);
 }
 
-int chunk_key_mass(const kv_ring_t* main_ring, const kv_ring_t* cand_ring, const void* q,
-                   int n_q, int64_t q_pos0, const float* lse, const kv_cache_bias_t* bias,
-                   float softmax_scale, int64_t slot_first, int n_cand, float* mass,
-                   void* stream) {
+int chunk_key_mass_multi(const kv_ring_t* main_ring, int n_sets,
+                         const kv_ring_t* const* cand_rings, const void* q, int n_q,
+                         int64_t q_pos0, const float* lse, const kv_cache_bias_t* bias,
+                         float softmax_scale, const int64_t* slot_first, const int* n_cand,
+                         float* const* mass, void* stream) {
   int rc = check_ring(main_ring);
   if (rc) return rc;
-  if ((rc = check_ring(cand_ring))) return rc;
-  if (main_ring->n_heads != cand_ring->n_heads || main_ring->head_dim != cand_ring->head_dim ||
-      main_ring->rope_base != cand_ring->rope_base)
+  if (n_sets < 1 || n_sets > KV_KEY_MASS_MAX_SETS || !cand_rings || !slot_first || !n_cand ||
+      !mass)
     return KV_EINVAL;
+  for (int t = 0; t < n_sets; ++t) {
+    const kv_ring_t* cr = cand_rings[t];
+    if (!cr) return KV_EINVAL;
+    if ((rc = check_ring(cr))) return rc;
+    if (main_ring->n_heads != cr->n_heads || main_ring->head_dim != cr->head_dim ||
+        main_ring->rope_base != cr->rope_base)
+      return KV_EINVAL;
+  }
   if (main_ring->head_dim != 128) return KV_EUNSUPPORTED;
-  if (n_q < 0 || n_cand < 0 || n_cand > cand_ring->capacity) return KV_EINVAL;
-  if (slot_first < 0 || slot_first >= cand_ring->capacity) return KV_EINVAL;
+  if (n_q < 0) return KV_EINVAL;
+  bool any = false;
+  for (int t = 0; t < n_sets; ++t) {
+    if (n_cand[t] < 0 || n_cand[t] > cand_rings[t]->capacity) return KV_EINVAL;
+    if (slot_first[t] < 0 || slot_first[t] >= cand_rings[t]->capacity) return KV_EINVAL;
+    any = any || n_cand[t] > 0;
+  }
   if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return KV_EINVAL;
   const float b = bias ? bias->history_bias : 0.f;
   if (isnan(b) || b == INFINITY) return KV_EINVAL;
-  if (n_q == 0 || n_cand == 0) return KV_OK;
-  if (!q || !lse || !mass || !aligned16(q) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
-      (reinterpret_cast<uintptr_t>(mass) & 3u))
-    return KV_EINVAL;
+  if (n_q == 0 || !any) return KV_OK;
+  if (!q || !lse || !aligned16(q) || (reinterpret_cast<uintptr_t>(lse) & 3u)) return KV_EINVAL;
+  for (int t = 0; t < n_sets; ++t)
+    if (n_cand[t] > 0 && (!mass[t] || (reinterpret_cast<uintptr_t>(mass[t]) & 3u)))
+      return KV_EINVAL;
   if (!in_table(main_ring, q_pos0, q_pos0 + n_q - 1)) return KV_ERANGE;
   KeyMassArgs a;
+  memset(&a, 0, sizeof(a));
   a.q = static_cast<const uint16_t*>(q);
   a.rope_q0 = main_ring->rope_table + (size_t)(q_pos0 - main_ring->rope_pos_min) * 128;
   a.lse = lse;
-  a.kc = cand_ring->k_codes;
-  a.ks = cand_ring->k_scale;
-  a.mass = mass;
   a.n_q = n_q;
   a.H = main_ring->n_heads;
-  a.C = cand_ring->capacity;
-  a.n_cand = n_cand;
-  a.slot_first = (int)slot_first;
+  for (int t = 0; t < n_sets; ++t) {
+    if (n_cand[t] == 0) continue;                     // nothing to score in this set
+    const int u = a.n_sets++;
+    a.kc[u] = cand_rings[t]->k_codes;
+    a.ks[u] = cand_rings[t]->k_scale;
+    a.mass[u] = mass[t];
+    a.C[u] = cand_rings[t]->capacity;
+    a.n_cand[u] = n_cand[t];
+    a.slot_first[u] = (int)slot_first[t];
+  }
   a.score_scale_log2 = softmax_scale * 1.4426950408889634f;
   a.bias_log2 = b * 1.4426950408889634f;
   a.timeouts = timeout_counter();
   if (!a.timeouts) return KV_ECUDA;
   return launch_key_mass(a, static_cast<cudaStream_t>(stream));
+}
+
+int chunk_key_mass(const kv_ring_t* main_ring, const kv_ring_t* cand_ring, const void* q,
+                   int n_q, int64_t q_pos0, const float* lse, const kv_cache_bias_t* bias,
+                   float softmax_scale, int64_t slot_first, int n_cand, float* mass,
+                   void* stream) {
+  if (!cand_ring) return KV_EINVAL;
+  return chunk_key_mass_multi(main_ring, 1, &cand_ring, q, n_q, q_pos0, lse, bias,
+                              softmax_scale, &slot_first, &n_cand, &mass, stream);
 }
 
 int kv_memory_select(const kv_ring_t* memory, const float* mass_memory, const kv_ring_t* fifo,

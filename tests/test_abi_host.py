@@ -257,6 +257,47 @@ def test_content_memory_validation(L):
     assert sel(memory=ctypes.byref(big)) == kv.KV_ERANGE               # > 8,192 candidates
 
 
+def test_key_mass_multi_validation(L):
+    main, c1, c2 = _fake_ring(D=128), _fake_ring(C=64, D=128), _fake_ring(C=32, D=128)
+    main.live, c1.live, c2.live = 64, 64, 32
+    rm = ctypes.byref(main)
+
+    def multi(rings=(c1, c2), firsts=(0, 0), counts=(16, 8), outs=(16, 32), n_sets=None,
+              n_q=8, lse=16, scale=0.125):
+        n = len(rings) if n_sets is None else n_sets
+        k = max(1, len(rings))
+        ra = (ctypes.c_void_p * k)(*[None if r is None else ctypes.addressof(r) for r in rings])
+        fa = (ctypes.c_int64 * k)(*firsts)
+        ca = (ctypes.c_int * k)(*counts)
+        oa = (ctypes.c_void_p * k)(*outs)
+        return L.chunk_key_mass_multi(rm, n, ra, 16, n_q, 0, lse, None, scale, fa, ca, oa, None)
+
+    assert multi(n_sets=0) == kv.KV_EINVAL
+    five = (c1,) * 5
+    assert multi(rings=five, firsts=(0,) * 5, counts=(1,) * 5, outs=(16,) * 5) == kv.KV_EINVAL
+    assert L.chunk_key_mass_multi(rm, 1, None, 16, 8, 0, 16, None, 0.125, None, None, None,
+                                  None) == kv.KV_EINVAL                  # null arrays
+    assert multi(rings=(c1, None)) == kv.KV_EINVAL
+    wide = _fake_ring(C=64, H=4, D=128)
+    assert multi(rings=(c1, wide)) == kv.KV_EINVAL                       # heads differ
+    assert multi(counts=(16, 33)) == kv.KV_EINVAL                        # > capacity of set 1
+    assert multi(firsts=(0, 32)) == kv.KV_EINVAL
+    assert multi(outs=(16, 34)) == kv.KV_EINVAL                          # misaligned mass
+    assert multi(outs=(16, None)) == kv.KV_EINVAL
+    assert multi(counts=(0, 0)) == kv.KV_OK                              # nothing to score
+    assert multi(counts=(0, 8), outs=(None, 32)) == kv.KV_ECUDA          # an empty set's
+    assert multi(n_q=0) == kv.KV_OK                                      # mass is not read
+    assert multi() == kv.KV_ECUDA                                        # reaches the device
+    m64 = _fake_ring(D=64)
+    m64.live = 64
+    c64 = _fake_ring(C=64, D=64)
+    c64.live = 64
+    ra = (ctypes.c_void_p * 1)(ctypes.addressof(c64))
+    assert L.chunk_key_mass_multi(ctypes.byref(m64), 1, ra, 16, 8, 0, 16, None, 0.125,
+                                  (ctypes.c_int64 * 1)(0), (ctypes.c_int * 1)(8),
+                                  (ctypes.c_void_p * 1)(16), None) == kv.KV_EUNSUPPORTED
+
+
 def test_split_workspace_size_and_validation(L):
     assert kv.chunk_attention_workspace_size(25, 32, 128, 8) == 8 * 25 * 32 * (4 * 128 + 8)
     assert kv.chunk_attention_workspace_size(25, 32, 128, 0) == 0

@@ -77,6 +77,11 @@ def test_fifo_anchor_memory_stream(orc):
             mem_first = (mem.s.write_slot + mem.s.pending - n_mem) % M
             mm = (kv.chunk_key_mass(fifo, mem, qd, fifo.next_pos, lse, mem_first, n_mem,
                                     cache_bias=-0.25) if n_mem else None)
+            # the same two sets in one launch: bit for bit the separate calls
+            if n_mem:
+                both = kv.chunk_key_mass_multi(fifo, [fifo, mem], qd, fifo.next_pos, lse,
+                                               [first, mem_first], [n, n_mem], cache_bias=-0.25)
+                assert torch.equal(both[0], mf) and torch.equal(both[1], mm)
             torch.cuda.synchronize()
             # masses against the oracle's definition (ages of the scored slots)
             newest = (o_fifo.write_slot + o_fifo.pending - 1) % C_fifo
@@ -125,3 +130,34 @@ def test_fifo_anchor_memory_stream(orc):
         o_fifo.commit()
     assert events >= 5
     assert kv.kv_wait_timeout_count() == 0
+
+
+def test_key_mass_multi_sets_match_single_calls():
+    """Four sets in one launch (several CTAs each, a range that wraps the ring's end, an
+    empty set, a second ring): every set's masses equal its own chunk_key_mass call."""
+    H, D, C, n = 4, 128, 1500, 300
+    ring = kv.KvRing(C, H, D, 0, 1 << 14)
+    other = kv.KvRing(700, H, D, 0, 1 << 14, rope_table=ring.rope_table)
+    for ch in range(6):
+        k, v = (inputs.draw(inputs.seed_of(57, ch, t), (n, H, D), "normal", 1.0, "bf16")
+                for t in (1, 2))
+        kv.kv_ring_write(ring, to_dev(k), to_dev(v), commit=True)
+        if ch < 2:
+            kv.kv_ring_write(other, to_dev(k), to_dev(v), commit=True)
+    q = to_dev(inputs.draw(inputs.seed_of(57, 9, 3), (n, H, D), "normal", 1.0, "bf16"))
+    k, v = (to_dev(inputs.draw(inputs.seed_of(57, 9, t), (n, H, D), "normal", 1.0, "bf16"))
+            for t in (1, 2))
+    kv.kv_ring_write(ring, k, v)
+    _, lse = kv.chunk_attention(ring, q, ring.next_pos, n, None, -0.5)
+    # history: the pending chunk is slots 300 .. 599; 1,300 .. 299 wraps the end
+    sets = [(ring, 600, 700), (ring, 1300, 500), (ring, 0, 0), (other, 50, 550)]
+    multi = kv.chunk_key_mass_multi(ring, [r for r, _, _ in sets], q, ring.next_pos, lse,
+                                    [f for _, f, _ in sets], [c for _, _, c in sets],
+                                    cache_bias=-0.5)
+    for (r, f, c), m in zip(sets, multi):
+        if c == 0:
+            continue
+        one = kv.chunk_key_mass(ring, r, q, ring.next_pos, lse, f, c, cache_bias=-0.5)
+        torch.cuda.synchronize()
+        assert torch.isfinite(one).all()
+        assert torch.equal(one, m), (f, c)
