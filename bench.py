@@ -534,9 +534,10 @@ def next_rows_timing(torch, kv, inputs, dev, stream, reps: int = 10) -> dict:
     mf = torch.empty((w.H, w.n), dtype=torch.float32, device=dev)
     mm = torch.empty((w.H, n_mem), dtype=torch.float32, device=dev)
     kept = torch.empty((M,), dtype=torch.int32, device=dev)
-    def mass():                                          # both sets in one launch
+    wsm = torch.empty(kv.chunk_key_mass_workspace_size(w.n, w.H), dtype=torch.uint8, device=dev)
+    def mass():               # both sets in one launch, the queries split once into wsm
         kv.chunk_key_mass_multi(fifo, [fifo, mem], q, fifo.next_pos, lse, [first, mem_first],
-                                [w.n, n_mem], masses=[mf, mm])
+                                [w.n, n_mem], masses=[mf, mm], workspace=wsm)
     def select():
         kv.kv_memory_select(mem, mm, fifo, mf, first, w.n, M, frame_len, dst, kept=kept)
     mass()

@@ -388,17 +388,27 @@ KV_API int chunk_key_mass(const kv_ring_t* main_ring, const kv_ring_t* cand_ring
  * that the CTAs of all sets fill the GPU together (an eviction scores the memory ring's
  * slots and the FIFO block the next write overwrites).  Set t: the n_cand[t] slots
  * (slot_first[t] + c) mod capacity of cand_rings[t], masses to mass[t] (device fp32
- * [H][n_cand[t]]).  Each set's result is bit for bit the one chunk_key_mass gives for it
- * alone.  cand_rings, slot_first, n_cand and mass are host arrays of n_sets entries,
- * 1 <= n_sets <= KV_KEY_MASS_MAX_SETS; sets with n_cand 0 are skipped.  Other arguments
- * and errors as chunk_key_mass, checked for every set before anything is launched;
- * KV_EINVAL also for n_sets out of range or a null array. */
+ * [H][n_cand[t]]).  cand_rings, slot_first, n_cand and mass are host arrays of n_sets
+ * entries, 1 <= n_sets <= KV_KEY_MASS_MAX_SETS; sets with n_cand 0 are skipped.
+ * workspace: null, or device memory of at least chunk_key_mass_workspace_size(n_q, H)
+ * bytes, 16-byte aligned, owned by the caller and free for the call's duration.  With
+ * it the query rows are rotated and split once per call (a second kernel before the
+ * scoring one) and the scoring CTAs stream them in; without it every CTA splits the
+ * rows itself (slower, nothing to allocate).  Each candidate's sum adds its queries in
+ * the same order either way.  Other arguments and errors as chunk_key_mass, checked for
+ * every set before anything is launched; KV_EINVAL also for n_sets out of range, a null
+ * array or a misaligned workspace, KV_ERANGE for a workspace that is too small. */
 KV_API int chunk_key_mass_multi(const kv_ring_t* main_ring, int n_sets,
                                 const kv_ring_t* const* cand_rings, const void* q, int n_q,
                                 int64_t q_pos0, const float* lse,
                                 const kv_cache_bias_t* bias, float softmax_scale,
                                 const int64_t* slot_first, const int* n_cand,
-                                float* const* mass, void* stream);
+                                float* const* mass, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/* Bytes of workspace chunk_key_mass_multi takes for n_q query rows of n_heads heads:
+ * n_heads * ceil(n_q / 64) * 16,896.  0 for n_q < 0 or n_heads < 1. */
+KV_API size_t chunk_key_mass_workspace_size(int n_q, int n_heads);
 
 /* Largest candidate count (memory slots + FIFO block) of one kv_memory_select call. */
 #define KV_MEMORY_MAX_CANDIDATES 8192

@@ -31,7 +31,8 @@ KV_PV_FP8 = 2
 EXPORTS = ("kv_rope_table_build", "kv_rope3d_table_build", "kv_ring_init", "kv_ring_write", "kv_ring_commit",
            "kv_ring_delta_rotate", "chunk_attention", "chunk_attention_workspace_size",
            "chunk_attention_split", "chunk_attention_split_noalloc", "chunk_attention_multi",
-           "chunk_attention_rows", "chunk_attention_suggest_splits", "chunk_key_mass", "chunk_key_mass_multi", "kv_memory_select", "kv_status_string",
+           "chunk_attention_rows", "chunk_attention_suggest_splits", "chunk_key_mass", "chunk_key_mass_multi", "chunk_key_mass_workspace_size",
+           "kv_memory_select", "kv_status_string",
            "kv_wait_timeout_count")
 KV_NOALLOC_SCRATCH_BYTES = 16 << 20
 KV_MEMORY_MAX_CANDIDATES = 8192
@@ -94,7 +95,10 @@ def lib() -> ctypes.CDLL:
         L.chunk_attention_suggest_splits.argtypes = [I, I, I64, I]
         L.chunk_attention_suggest_splits.restype = I
         L.chunk_key_mass.argtypes = [P, P, P, I, I64, P, P, ctypes.c_float, I64, I, P, P]
-        L.chunk_key_mass_multi.argtypes = [P, I, P, P, I, I64, P, P, ctypes.c_float, P, P, P, P]
+        L.chunk_key_mass_multi.argtypes = [P, I, P, P, I, I64, P, P, ctypes.c_float, P, P, P,
+                                           P, ctypes.c_size_t, P]
+        L.chunk_key_mass_workspace_size.argtypes = [I, I]
+        L.chunk_key_mass_workspace_size.restype = ctypes.c_size_t
         L.kv_memory_select.argtypes = [P, P, P, P, I64, I, I, I64, ctypes.c_float, P, P, P]
         L.kv_status_string.argtypes = [I]
         L.kv_status_string.restype = ctypes.c_char_p
@@ -421,12 +425,17 @@ def chunk_key_mass(main: KvRing, cand: KvRing, q, q_pos0: int, lse, slot_first: 
     return mass
 
 
+def chunk_key_mass_workspace_size(n_q: int, n_heads: int) -> int:
+    return int(lib().chunk_key_mass_workspace_size(int(n_q), int(n_heads)))
+
+
 def chunk_key_mass_multi(main: KvRing, cands, q, q_pos0: int, lse, slot_firsts, n_cands,
                          cache_bias: float = 0.0, softmax_scale: float | None = None,
-                         masses=None, stream=None):
+                         masses=None, workspace=None, stream=None):
     """chunk_key_mass for several candidate sets (rings `cands`, first slots, counts) of
-    one attention call in one launch.  Returns the list of masses [H][n_cand] (fp32,
-    device), one per set."""
+    one attention call in one launch.  `workspace` (device, at least
+    chunk_key_mass_workspace_size bytes) lets the queries be split once per call.
+    Returns the list of masses [H][n_cand] (fp32, device), one per set."""
     import torch
     assert q.is_cuda and q.dtype == torch.bfloat16 and q.is_contiguous()
     assert lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous()
@@ -442,9 +451,11 @@ def chunk_key_mass_multi(main: KvRing, cands, q, q_pos0: int, lse, slot_firsts, 
     firsts = (ctypes.c_int64 * n)(*[int(f) for f in slot_firsts])
     counts = (ctypes.c_int * n)(*[int(c) for c in n_cands])
     outs = (ctypes.c_void_p * n)(*[_ptr(m) for m in masses])
+    ws = None if workspace is None else _ptr(workspace)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().chunk_key_mass_multi(main.ref, n, rings, _ptr(q), int(q.shape[0]), int(q_pos0),
                                       _ptr(lse), ctypes.byref(b), float(softmax_scale), firsts,
-                                      counts, outs, _stream(stream)),
+                                      counts, outs, ws, ws_bytes, _stream(stream)),
            "chunk_key_mass_multi")
     return masses
 

@@ -91,8 +91,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tmv, const AttnArgs a) {
   using S = Smem<D>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned by pointer arithmetic on the shared array (an integer round trip
+  // would hide from the compiler that sm addresses shared memory)
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   float* kscl = reinterpret_cast<float*>(sm + S::kscl);
   float* kbias = reinterpret_cast<float*>(sm + S::kbias);
   int* ktok = reinterpret_cast<int*>(sm + S::ktok);

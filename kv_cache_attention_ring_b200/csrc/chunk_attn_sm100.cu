@@ -341,8 +341,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const __grid_constant__ ExtraMaps xm, const AttnArgs a) {
   constexpr float kThr = kPv8 ? 0.f : kRescaleLog2;   // lazy-maximum threshold (log2)
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned by pointer arithmetic on the shared array (an integer round trip
+  // would hide from the compiler that sm addresses shared memory)
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   Bars bars{reinterpret_cast<uint64_t*>(sm + Layout::bars)};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Layout::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Layout::misc + 4);

@@ -87,7 +87,12 @@ struct KeyMassArgs {
   float score_scale_log2;   // softmax_scale * log2(e)
   float bias_log2;          // history_bias * log2(e)
   unsigned int* timeouts;
+  uint8_t* qws;             // split query images (workspace), or null: split in every CTA
+  int n_qt;                 // their 64-row tiles per head
 };
+
+// Bytes of the split query images of n_q rows x n_heads (the pipelined key mass).
+size_t key_mass_workspace_bytes(int n_q, int n_heads);
 
 // Top-M selection over a memory ring's slots and a FIFO block, and the gather of the kept
 // entries into a fresh ring (see key_mass.cu).

@@ -51,10 +51,70 @@ __device__ __forceinline__ float ex2f(float x) {
   return y;
 }
 
+// One lane of a query row's group of 8 lanes (16 elements each): row i of head h rotated
+// with the main ring's table, rounded to bf16 and split exactly into e4m3 hi + lo with the
+// row's power of two r = 2^k (zeros for i >= n_q).  All 8 lanes of the group call it
+// together: the row maximum is shuffled among them.
+__device__ __forceinline__ void q_split_lane(const KeyMassArgs& a, int i, int h, int lc,
+                                             uint32_t (&hw)[4], uint32_t (&lw)[4], int& k) {
+  float y[16];
+  if (i < a.n_q) {
+    const uint4* qp = reinterpret_cast<const uint4*>(a.q + ((size_t)i * a.H + h) * D + 16 * lc);
+    const uint4 q0v = __ldg(qp), q1v = __ldg(qp + 1);
+    const float4* tb = reinterpret_cast<const float4*>(a.rope_q0 + (size_t)i * D + 16 * lc);
+    const uint32_t w[8] = {q0v.x, q0v.y, q0v.z, q0v.w, q1v.x, q1v.y, q1v.z, q1v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float4 cs = __ldg(tb + j);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const uint32_t pr = w[2 * j + u];
+        const float c = u ? cs.z : cs.x, s = u ? cs.w : cs.y;
+        const float x0 = bf16_bits_to_float(pr & 0xFFFFu), x1 = bf16_bits_to_float(pr >> 16);
+        const uint32_t b = pack_bf16x2(sub_rn(mul_rn(x0, c), mul_rn(x1, s)),
+                                       add_rn(mul_rn(x0, s), mul_rn(x1, c)));
+        y[4 * j + 2 * u] = bf16_bits_to_float(b & 0xFFFFu);
+        y[4 * j + 2 * u + 1] = bf16_bits_to_float(b >> 16);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) y[e] = 0.f;
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) amax = max_nan(amax, fabsf(y[e]));
+#pragma unroll
+  for (int off = 4; off > 0; off >>= 1) amax = max_nan(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  k = 0;
+  if (amax > 0.f && amax <= 3.402823466e38f) {
+    int e;
+    const float m = frexpf(amax, &e);
+    k = max(-126, min(127, (e - 1) - 8 + (m > 0.875f ? 1 : 0)));
+  }
+  const float inv_r = ldexpf(1.f, -k);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float x[4], lv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[e] = y[4 * j + e] * inv_r;
+    const uint32_t h01 = e4m3x2(x[0], x[1]), h23 = e4m3x2(x[2], x[3]);
+    const float2 d01 = f16x2_to_float2(e4m3x2_to_f16x2((uint16_t)h01));
+    const float2 d23 = f16x2_to_float2(e4m3x2_to_f16x2((uint16_t)h23));
+    lv[0] = x[0] - d01.x;
+    lv[1] = x[1] - d01.y;
+    lv[2] = x[2] - d23.x;
+    lv[3] = x[3] - d23.y;
+    hw[j] = h01 | (h23 << 16);
+    lw[j] = e4m3x2(lv[0], lv[1]) | (e4m3x2(lv[2], lv[3]) << 16);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1) key_mass_kernel(const KeyMassArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned by pointer arithmetic on the shared array (an integer round trip
+  // would hide from the compiler that sm addresses shared memory)
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + MassLayout::bar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + MassLayout::misc);
   float* rq = reinterpret_cast<float*>(sm + MassLayout::rq);
@@ -118,58 +178,9 @@ __global__ void __launch_bounds__(kThreads, 1) key_mass_kernel(const KeyMassArgs
     // of two r), 16 rows per pass of the 128 threads
     for (int rr = tid >> 3; rr < QN; rr += kThreads / 8) {
       const int i = q0 + rr;
-      float y[16];
-      if (i < a.n_q) {
-        const uint4* qp = reinterpret_cast<const uint4*>(a.q + ((size_t)i * a.H + h) * D + 16 * lc);
-        const uint4 q0v = __ldg(qp), q1v = __ldg(qp + 1);
-        const float4* tb = reinterpret_cast<const float4*>(a.rope_q0 + (size_t)i * D + 16 * lc);
-        const uint32_t w[8] = {q0v.x, q0v.y, q0v.z, q0v.w, q1v.x, q1v.y, q1v.z, q1v.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float4 cs = __ldg(tb + j);
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const uint32_t pr = w[2 * j + u];
-            const float c = u ? cs.z : cs.x, s = u ? cs.w : cs.y;
-            const float x0 = bf16_bits_to_float(pr & 0xFFFFu), x1 = bf16_bits_to_float(pr >> 16);
-            const uint32_t b = pack_bf16x2(sub_rn(mul_rn(x0, c), mul_rn(x1, s)),
-                                           add_rn(mul_rn(x0, s), mul_rn(x1, c)));
-            y[4 * j + 2 * u] = bf16_bits_to_float(b & 0xFFFFu);
-            y[4 * j + 2 * u + 1] = bf16_bits_to_float(b >> 16);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) y[e] = 0.f;
-      }
-      float amax = 0.f;
-#pragma unroll
-      for (int e = 0; e < 16; ++e) amax = max_nan(amax, fabsf(y[e]));
-#pragma unroll
-      for (int off = 4; off > 0; off >>= 1) amax = max_nan(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-      int k = 0;
-      if (amax > 0.f && amax <= 3.402823466e38f) {
-        int e;
-        const float m = frexpf(amax, &e);
-        k = max(-126, min(127, (e - 1) - 8 + (m > 0.875f ? 1 : 0)));
-      }
-      const float inv_r = ldexpf(1.f, -k);
       uint32_t hw[4], lw[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float x[4], lv[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = y[4 * j + e] * inv_r;
-        const uint32_t h01 = e4m3x2(x[0], x[1]), h23 = e4m3x2(x[2], x[3]);
-        const float2 d01 = f16x2_to_float2(e4m3x2_to_f16x2((uint16_t)h01));
-        const float2 d23 = f16x2_to_float2(e4m3x2_to_f16x2((uint16_t)h23));
-        lv[0] = x[0] - d01.x;
-        lv[1] = x[1] - d01.y;
-        lv[2] = x[2] - d23.x;
-        lv[3] = x[3] - d23.y;
-        hw[j] = h01 | (h23 << 16);
-        lw[j] = e4m3x2(lv[0], lv[1]) | (e4m3x2(lv[2], lv[3]) << 16);
-      }
+      int k;
+      q_split_lane(a, i, h, lc, hw, lw, k);
       const uint32_t off = (uint32_t)rr * 128u + ((uint32_t)(lc ^ (rr & 7)) << 4);
       *reinterpret_cast<uint4*>(sm + MassLayout::qhi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
       *reinterpret_cast<uint4*>(sm + MassLayout::qlo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
@@ -229,6 +240,206 @@ __global__ void __launch_bounds__(kThreads, 1) key_mass_kernel(const KeyMassArgs
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, KG * 128);
+  }
+}
+
+// ------------------------------------------------------------------ pipelined key mass
+// With a caller workspace the query split runs once per call instead of once per CTA:
+// key_mass_qsplit_kernel writes, per head and tile of 64 query rows, the image the MMA
+// reads (hi and lo codes, K-major with the 128-byte swizzle, then r and lse * log2(e) per
+// row); key_mass_pipe_kernel streams those images into shared memory with bulk copies,
+// NQS tiles ahead, and double-buffers S in tensor memory, so that the MMAs of tile t + 1
+// run while the threads sum tile t.  One warp per key group issues that group's eight
+// MMAs (a single issuer for all 32 held every other warp at the tile barrier).  Each
+// candidate's sum runs over the queries in the same order as in key_mass_kernel.
+constexpr int QT = 64;                       // query rows per pipelined tile (MMA N)
+constexpr int NQS = 3;                       // tile images in flight
+struct QTile {                               // one (head, tile) image, workspace and smem
+  static constexpr uint32_t hi = 0;                   // e4m3 [64 queries][128], sw128
+  static constexpr uint32_t lo = QT * D;
+  static constexpr uint32_t rq = 2 * QT * D;          // per query: r, or 0
+  static constexpr uint32_t lq = rq + QT * 4;         // per query: lse * log2(e), or +inf
+  static constexpr uint32_t bytes = lq + QT * 4;      // 16,896 (a multiple of 16)
+};
+struct PipeLayout {
+  static constexpr uint32_t k = 0;                    // KG x e4m3 [128 keys][128], sw128
+  static constexpr uint32_t qstride = (QTile::bytes + 1023u) & ~1023u;
+  static constexpr uint32_t q = k + KG * KM * D;      // NQS tile images, 1024-aligned
+  static constexpr uint32_t bar = q + NQS * qstride;  // qfull[NQS], sfull[2]
+  static constexpr uint32_t misc = bar + 8 * (NQS + 2);   // tmem address, abort flag
+  static constexpr uint32_t bytes = misc + 8 + 1024;      // + alignment slack
+};
+
+__global__ void __launch_bounds__(512) key_mass_qsplit_kernel(const KeyMassArgs a) {
+  const int t = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+  const int rr = tid >> 3, lc = tid & 7, i = t * QT + rr;
+  uint8_t* img = a.qws + ((size_t)h * a.n_qt + t) * QTile::bytes;
+  uint32_t hw[4], lw[4];
+  int k;
+  q_split_lane(a, i, h, lc, hw, lw, k);
+  const uint32_t off = (uint32_t)rr * 128u + ((uint32_t)(lc ^ (rr & 7)) << 4);
+  *reinterpret_cast<uint4*>(img + QTile::hi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+  *reinterpret_cast<uint4*>(img + QTile::lo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  if (lc == 0) {
+    // rows past n_q, rows that attended nothing (lse not finite): no contribution
+    const float l = i < a.n_q ? __ldg(a.lse + (size_t)h * a.n_q + i) : INFINITY;
+    const bool use = isfinite(l);
+    reinterpret_cast<float*>(img + QTile::rq)[rr] = use ? ldexpf(1.f, k) : 0.f;
+    reinterpret_cast<float*>(img + QTile::lq)[rr] = use ? l * 1.4426950408889634f : INFINITY;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) key_mass_pipe_kernel(const KeyMassArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte aligned by pointer arithmetic on the shared array (an integer round trip
+  // would hide from the compiler that sm addresses shared memory)
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* qfull = reinterpret_cast<uint64_t*>(sm + PipeLayout::bar);
+  uint64_t* sfull = qfull + NQS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + PipeLayout::misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + PipeLayout::misc + 4);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int grp = warp >> 2, quad = warp & 3;
+  const int krow = 32 * quad + lane;                   // TMEM lane = row in group grp
+  const int h = blockIdx.y;
+  int set = 0;                                         // candidate set of this CTA
+  while (set + 1 < a.n_sets && (int)blockIdx.x >= a.blk_first[set + 1]) ++set;
+  const int n_cand = a.n_cand[set], C = a.C[set];
+  const int c = ((int)blockIdx.x - a.blk_first[set]) * (KG * KM) + grp * KM + krow;
+  const bool live_c = c < n_cand;                      // this thread's candidate
+  const int n_t = a.n_qt;
+
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 2 * KG * QT);                // S double-buffered: 512 columns
+    tmem_relinquish();
+  }
+  if (tid == 32) {
+    for (int st = 0; st < NQS; ++st) mbar_init(&qfull[st], 1);
+    mbar_init(&sfull[0], KG);                          // one commit per group's issuer
+    mbar_init(&sfull[1], KG);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // candidate key row, as in key_mass_kernel
+  float kscl = 0.f;
+  {
+    uint4 w[8];
+    if (live_c) {
+      int slot = a.slot_first[set] + c;
+      slot = slot >= C ? slot - C : slot;
+      const uint4* src = reinterpret_cast<const uint4*>(a.kc[set] + ((size_t)h * C + slot) * D);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[i] = __ldg(src + i);
+      kscl = __ldg(a.ks[set] + (size_t)h * C + slot) * a.score_scale_log2;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    uint8_t* krow_sm = sm + PipeLayout::k + grp * KM * D + krow * 128;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      *reinterpret_cast<uint4*>(krow_sm + ((i ^ (krow & 7)) << 4)) = w[i];
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
+  const uint8_t* img0 = a.qws + (size_t)h * n_t * QTile::bytes;
+  int n_loads = 0;                                     // thread 0: tile images requested
+  auto load = [&](int t) {
+    uint8_t* dst = sm + PipeLayout::q + (t % NQS) * PipeLayout::qstride;
+    mbar_arrive_expect_tx(&qfull[t % NQS], QTile::bytes);
+    bulk_load(dst, img0 + (size_t)t * QTile::bytes, QTile::bytes, &qfull[t % NQS]);
+    n_loads = t + 1;
+  };
+  if (tid == 0)
+    for (int t = 0; t < NQS && t < n_t; ++t) load(t);
+
+  constexpr uint32_t idS = idesc_e4m3_f32(KM, QT);
+  const uint64_t dK = smem_desc_sw128(smem_u32(sm + PipeLayout::k), 16, 1024);
+  // warp 5 g of group g (one per SM sub-partition), converged: S_g(t) = K_g Q(t)^T into
+  // buffer t & 1 once tile t's image has landed
+  const bool issuer = warp == 5 * grp;
+  int n_mma = 0;                                       // issuers: tiles whose MMAs went out
+  auto issue = [&](int t) -> bool {
+    if (!mbar_wait_warp(&qfull[t % NQS], (t / NQS) & 1, abort_flag, a.timeouts)) return false;
+    tc_fence_after();
+    const uint32_t qs = smem_u32(sm + PipeLayout::q + (t % NQS) * PipeLayout::qstride);
+    const uint64_t dQhi = smem_desc_sw128(qs + QTile::hi, 16, 1024);
+    const uint64_t dQlo = smem_desc_sw128(qs + QTile::lo, 16, 1024);
+    const uint64_t kd = dK + ((grp * KM * D) >> 4);
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const uint64_t qd = hf == 0 ? dQhi : dQlo;
+#pragma unroll
+      for (int kk = 0; kk < D / 32; ++kk)
+        el_mma_f8_ss(tmem + KG * QT * (t & 1) + QT * grp, kd + 2 * kk, qd + 2 * kk, idS,
+                     (hf | kk) != 0);
+    }
+    el_commit(&sfull[t & 1]);
+    n_mma = t + 1;
+    return true;
+  };
+
+  float acc = 0.f;
+  bool ok = true;
+  if (issuer && n_t > 0) ok = issue(0);
+  for (int t = 0; t < n_t; ++t) {
+    // S(t + 1) goes into the buffer every thread finished reading before the last barrier
+    if (issuer && ok && t + 1 < n_t) ok = issue(t + 1);
+    // S(t), and tile t's image itself (its r and lse are read below; complete already)
+    auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      if (mbar_try_wait(bar, parity)) return true;
+      if (*abort_flag) return false;
+      if (mbar_wait(bar, parity, a.timeouts)) return true;
+      *abort_flag = 1;
+      return false;
+    };
+    bool got = wait(&sfull[t & 1], (t >> 1) & 1) && wait(&qfull[t % NQS], (t / NQS) & 1);
+    tc_fence_after();
+    if (__all_sync(0xffffffffu, got)) {
+      const uint8_t* img = sm + PipeLayout::q + (t % NQS) * PipeLayout::qstride;
+      const float* rq = reinterpret_cast<const float*>(img + QTile::rq);
+      const float* lq = reinterpret_cast<const float*>(img + QTile::lq);
+#pragma unroll 1
+      for (int cb = 0; cb < QT; cb += 32) {
+        uint32_t sr[32];
+        tmem_ld32(tmem + lane_base + KG * QT * (t & 1) + QT * grp + cb, sr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          // s' = S kscl r + bias - lse (log2 units); 2^-inf = 0 for unused rows
+          const float x = fmaf(__uint_as_float(sr[u]) * kscl, rq[cb + u], a.bias_log2) - lq[cb + u];
+          acc += ex2f(x);
+        }
+      }
+    }
+    tc_fence_before();
+    ok = __syncthreads_and(ok && got);
+    if (!ok) break;
+    // tile t's image is free (its MMAs completed before sfull(t) did): refill it
+    if (tid == 0 && t + NQS < n_t) load(t + NQS);
+  }
+  if (!ok) {
+    // abandoned: wait (bounded) for the copies and MMAs this CTA issued, the last of
+    // each barrier standing for every earlier one on it (an S phase that another issuer
+    // never committed to ends the wait by its time limit)
+    if (tid == 0)
+      for (int u = max(0, n_loads - NQS); u < n_loads; ++u)
+        mbar_wait(&qfull[u % NQS], (u / NQS) & 1, a.timeouts);
+    if (issuer && lane == 0)
+      for (int u = max(0, n_mma - 2); u < n_mma; ++u)
+        mbar_wait(&sfull[u & 1], (u >> 1) & 1, a.timeouts);
+    acc = __uint_as_float(0x7FC00000u);
+  }
+  if (live_c) a.mass[set][(size_t)h * n_cand + c] = acc;
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 2 * KG * QT);
   }
 }
 
@@ -508,19 +719,35 @@ __global__ void __launch_bounds__(256) memory_gather_kernel(const SelectArgs a) 
 
 }  // namespace
 
+size_t key_mass_workspace_bytes(int n_q, int n_heads) {
+  if (n_q < 0 || n_heads < 1) return 0;
+  return (size_t)n_heads * (size_t)((n_q + QT - 1) / QT) * QTile::bytes;
+}
+
 int launch_key_mass(const KeyMassArgs& a, cudaStream_t s) {
-  static unsigned char configured[kMaxDevices] = {};
-  if (!smem_attr_set(reinterpret_cast<const void*>(key_mass_kernel), (int)MassLayout::bytes,
-                     configured))
-    return KV_ECUDA;
   // every set's CTAs in one grid: blk_first is the running sum of their block counts
   KeyMassArgs b = a;
   b.blk_first[0] = 0;
   for (int t = 0; t < b.n_sets; ++t)
     b.blk_first[t + 1] = b.blk_first[t] + (b.n_cand[t] + KG * KM - 1) / (KG * KM);
-  if (b.blk_first[b.n_sets] == 0) return KV_OK;
+  if (b.blk_first[b.n_sets] == 0 || b.n_q == 0) return KV_OK;
   const dim3 grid((unsigned)b.blk_first[b.n_sets], (unsigned)b.H);
-  key_mass_kernel<<<grid, kThreads, MassLayout::bytes, s>>>(b);
+  if (b.qws) {
+    static unsigned char configured[kMaxDevices] = {};
+    if (!smem_attr_set(reinterpret_cast<const void*>(key_mass_pipe_kernel),
+                       (int)PipeLayout::bytes, configured))
+      return KV_ECUDA;
+    b.n_qt = (b.n_q + QT - 1) / QT;
+    key_mass_qsplit_kernel<<<dim3((unsigned)b.n_qt, (unsigned)b.H), 512, 0, s>>>(b);
+    if (cudaPeekAtLastError() != cudaSuccess) return KV_ECUDA;
+    key_mass_pipe_kernel<<<grid, kThreads, PipeLayout::bytes, s>>>(b);
+  } else {
+    static unsigned char configured[kMaxDevices] = {};
+    if (!smem_attr_set(reinterpret_cast<const void*>(key_mass_kernel), (int)MassLayout::bytes,
+                       configured))
+      return KV_ECUDA;
+    key_mass_kernel<<<grid, kThreads, MassLayout::bytes, s>>>(b);
+  }
   return cudaPeekAtLastError() == cudaSuccess ? KV_OK : KV_ECUDA;
 }
 

@@ -595,7 +595,8 @@ int chunk_key_mass_multi(const kv_ring_t* main_ring, int n_sets,
                          const kv_ring_t* const* cand_rings, const void* q, int n_q,
                          int64_t q_pos0, const float* lse, const kv_cache_bias_t* bias,
                          float softmax_scale, const int64_t* slot_first, const int* n_cand,
-                         float* const* mass, void* stream) {
+                         float* const* mass, void* workspace, size_t workspace_bytes,
+                         void* stream) {
   int rc = check_ring(main_ring);
   if (rc) return rc;
   if (n_sets < 1 || n_sets > KV_KEY_MASS_MAX_SETS || !cand_rings || !slot_first || !n_cand ||
@@ -625,6 +626,9 @@ int chunk_key_mass_multi(const kv_ring_t* main_ring, int n_sets,
   for (int t = 0; t < n_sets; ++t)
     if (n_cand[t] > 0 && (!mass[t] || (reinterpret_cast<uintptr_t>(mass[t]) & 3u)))
       return KV_EINVAL;
+  if (workspace && !aligned16(workspace)) return KV_EINVAL;
+  if (workspace && workspace_bytes < key_mass_workspace_bytes(n_q, main_ring->n_heads))
+    return KV_ERANGE;
   if (!in_table(main_ring, q_pos0, q_pos0 + n_q - 1)) return KV_ERANGE;
   KeyMassArgs a;
   memset(&a, 0, sizeof(a));
@@ -645,9 +649,14 @@ int chunk_key_mass_multi(const kv_ring_t* main_ring, int n_sets,
   }
   a.score_scale_log2 = softmax_scale * 1.4426950408889634f;
   a.bias_log2 = b * 1.4426950408889634f;
+  a.qws = static_cast<uint8_t*>(workspace);
   a.timeouts = timeout_counter();
   if (!a.timeouts) return KV_ECUDA;
   return launch_key_mass(a, static_cast<cudaStream_t>(stream));
+}
+
+size_t chunk_key_mass_workspace_size(int n_q, int n_heads) {
+  return key_mass_workspace_bytes(n_q, n_heads);
 }
 
 int chunk_key_mass(const kv_ring_t* main_ring, const kv_ring_t* cand_ring, const void* q,
@@ -656,7 +665,7 @@ int chunk_key_mass(const kv_ring_t* main_ring, const kv_ring_t* cand_ring, const
                    void* stream) {
   if (!cand_ring) return KV_EINVAL;
   return chunk_key_mass_multi(main_ring, 1, &cand_ring, q, n_q, q_pos0, lse, bias,
-                              softmax_scale, &slot_first, &n_cand, &mass, stream);
+                              softmax_scale, &slot_first, &n_cand, &mass, nullptr, 0, stream);
 }
 
 int kv_memory_select(const kv_ring_t* memory, const float* mass_memory, const kv_ring_t* fifo,

@@ -263,20 +263,21 @@ def test_key_mass_multi_validation(L):
     rm = ctypes.byref(main)
 
     def multi(rings=(c1, c2), firsts=(0, 0), counts=(16, 8), outs=(16, 32), n_sets=None,
-              n_q=8, lse=16, scale=0.125):
+              n_q=8, lse=16, scale=0.125, ws=None, ws_bytes=0):
         n = len(rings) if n_sets is None else n_sets
         k = max(1, len(rings))
         ra = (ctypes.c_void_p * k)(*[None if r is None else ctypes.addressof(r) for r in rings])
         fa = (ctypes.c_int64 * k)(*firsts)
         ca = (ctypes.c_int * k)(*counts)
         oa = (ctypes.c_void_p * k)(*outs)
-        return L.chunk_key_mass_multi(rm, n, ra, 16, n_q, 0, lse, None, scale, fa, ca, oa, None)
+        return L.chunk_key_mass_multi(rm, n, ra, 16, n_q, 0, lse, None, scale, fa, ca, oa, ws,
+                                      ws_bytes, None)
 
     assert multi(n_sets=0) == kv.KV_EINVAL
     five = (c1,) * 5
     assert multi(rings=five, firsts=(0,) * 5, counts=(1,) * 5, outs=(16,) * 5) == kv.KV_EINVAL
     assert L.chunk_key_mass_multi(rm, 1, None, 16, 8, 0, 16, None, 0.125, None, None, None,
-                                  None) == kv.KV_EINVAL                  # null arrays
+                                  None, 0, None) == kv.KV_EINVAL         # null arrays
     assert multi(rings=(c1, None)) == kv.KV_EINVAL
     wide = _fake_ring(C=64, H=4, D=128)
     assert multi(rings=(c1, wide)) == kv.KV_EINVAL                       # heads differ
@@ -288,6 +289,12 @@ def test_key_mass_multi_validation(L):
     assert multi(counts=(0, 8), outs=(None, 32)) == kv.KV_ECUDA          # an empty set's
     assert multi(n_q=0) == kv.KV_OK                                      # mass is not read
     assert multi() == kv.KV_ECUDA                                        # reaches the device
+    need = kv.chunk_key_mass_workspace_size(8, 2)
+    assert need == 2 * 1 * 16896 and kv.chunk_key_mass_workspace_size(65, 40) == 40 * 2 * 16896
+    assert kv.chunk_key_mass_workspace_size(-1, 2) == 0
+    assert multi(ws=24, ws_bytes=need) == kv.KV_EINVAL                   # misaligned
+    assert multi(ws=256, ws_bytes=need - 16) == kv.KV_ERANGE             # too small
+    assert multi(ws=256, ws_bytes=need) == kv.KV_ECUDA
     m64 = _fake_ring(D=64)
     m64.live = 64
     c64 = _fake_ring(C=64, D=64)
@@ -295,7 +302,7 @@ def test_key_mass_multi_validation(L):
     ra = (ctypes.c_void_p * 1)(ctypes.addressof(c64))
     assert L.chunk_key_mass_multi(ctypes.byref(m64), 1, ra, 16, 8, 0, 16, None, 0.125,
                                   (ctypes.c_int64 * 1)(0), (ctypes.c_int * 1)(8),
-                                  (ctypes.c_void_p * 1)(16), None) == kv.KV_EUNSUPPORTED
+                                  (ctypes.c_void_p * 1)(16), None, 0, None) == kv.KV_EUNSUPPORTED
 
 
 def test_split_workspace_size_and_validation(L):

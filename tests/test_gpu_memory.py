@@ -78,10 +78,17 @@ def test_fifo_anchor_memory_stream(orc):
             mm = (kv.chunk_key_mass(fifo, mem, qd, fifo.next_pos, lse, mem_first, n_mem,
                                     cache_bias=-0.25) if n_mem else None)
             # the same two sets in one launch: bit for bit the separate calls
+            # (and with the workspace: queries split once, streamed into the scoring CTAs)
             if n_mem:
                 both = kv.chunk_key_mass_multi(fifo, [fifo, mem], qd, fifo.next_pos, lse,
                                                [first, mem_first], [n, n_mem], cache_bias=-0.25)
                 assert torch.equal(both[0], mf) and torch.equal(both[1], mm)
+                wsm = torch.empty(kv.chunk_key_mass_workspace_size(n, H), dtype=torch.uint8,
+                                  device="cuda")
+                piped = kv.chunk_key_mass_multi(fifo, [fifo, mem], qd, fifo.next_pos, lse,
+                                                [first, mem_first], [n, n_mem],
+                                                cache_bias=-0.25, workspace=wsm)
+                assert torch.equal(piped[0], mf) and torch.equal(piped[1], mm)
             torch.cuda.synchronize()
             # masses against the oracle's definition (ages of the scored slots)
             newest = (o_fifo.write_slot + o_fifo.pending - 1) % C_fifo
@@ -134,7 +141,8 @@ def test_fifo_anchor_memory_stream(orc):
 
 def test_key_mass_multi_sets_match_single_calls():
     """Four sets in one launch (several CTAs each, a range that wraps the ring's end, an
-    empty set, a second ring): every set's masses equal its own chunk_key_mass call."""
+    empty set, a second ring): every set's masses equal its own chunk_key_mass call, with
+    and without the workspace (300 queries: four whole 64-row tiles and a ragged one)."""
     H, D, C, n = 4, 128, 1500, 300
     ring = kv.KvRing(C, H, D, 0, 1 << 14)
     other = kv.KvRing(700, H, D, 0, 1 << 14, rope_table=ring.rope_table)
@@ -154,10 +162,15 @@ def test_key_mass_multi_sets_match_single_calls():
     multi = kv.chunk_key_mass_multi(ring, [r for r, _, _ in sets], q, ring.next_pos, lse,
                                     [f for _, f, _ in sets], [c for _, _, c in sets],
                                     cache_bias=-0.5)
-    for (r, f, c), m in zip(sets, multi):
+    ws = torch.empty(kv.chunk_key_mass_workspace_size(n, H), dtype=torch.uint8, device="cuda")
+    piped = kv.chunk_key_mass_multi(ring, [r for r, _, _ in sets], q, ring.next_pos, lse,
+                                    [f for _, f, _ in sets], [c for _, _, c in sets],
+                                    cache_bias=-0.5, workspace=ws)
+    for (r, f, c), m, p in zip(sets, multi, piped):
         if c == 0:
             continue
         one = kv.chunk_key_mass(ring, r, q, ring.next_pos, lse, f, c, cache_bias=-0.5)
         torch.cuda.synchronize()
         assert torch.isfinite(one).all()
         assert torch.equal(one, m), (f, c)
+        assert torch.equal(one, p), (f, c, (one - p).abs().max().item())
