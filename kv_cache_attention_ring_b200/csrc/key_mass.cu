@@ -401,18 +401,23 @@ __global__ void __launch_bounds__(kThreads, 1) key_mass_pipe_kernel(const KeyMas
     tc_fence_after();
     if (__all_sync(0xffffffffu, got)) {
       const uint8_t* img = sm + PipeLayout::q + (t % NQS) * PipeLayout::qstride;
-      const float* rq = reinterpret_cast<const float*>(img + QTile::rq);
-      const float* lq = reinterpret_cast<const float*>(img + QTile::lq);
+      const float4* rq4 = reinterpret_cast<const float4*>(img + QTile::rq);
+      const float4* lq4 = reinterpret_cast<const float4*>(img + QTile::lq);
 #pragma unroll 1
       for (int cb = 0; cb < QT; cb += 32) {
         uint32_t sr[32];
         tmem_ld32(tmem + lane_base + KG * QT * (t & 1) + QT * grp + cb, sr);
         tmem_wait_ld();
 #pragma unroll
-        for (int u = 0; u < 32; ++u) {
-          // s' = S kscl r + bias - lse (log2 units); 2^-inf = 0 for unused rows
-          const float x = fmaf(__uint_as_float(sr[u]) * kscl, rq[cb + u], a.bias_log2) - lq[cb + u];
-          acc += ex2f(x);
+        for (int u4 = 0; u4 < 8; ++u4) {
+          const float4 r = rq4[cb / 4 + u4], l = lq4[cb / 4 + u4];
+          const float rr[4] = {r.x, r.y, r.z, r.w}, ll[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            // s' = S kscl r + bias - lse (log2 units); 2^-inf = 0 for unused rows
+            const float x = fmaf(__uint_as_float(sr[4 * u4 + e]) * kscl, rr[e], a.bias_log2) - ll[e];
+            acc += ex2f(x);
+          }
         }
       }
     }
@@ -469,10 +474,10 @@ __device__ __forceinline__ bool before_in_score(const Cand& x, const Cand& y) {
   return x.idx < y.idx;
 }
 
-// Bitonic sort of n_pow2 <= 4 * kSelThreads entries of v (padding entries sort last), all
-// threads.  Thread t holds entries 4t .. 4t + 3 in registers: pairs closer than 4 entries
-// are exchanged in registers, pairs up to 128 apart through warp shuffles, and only the
-// wider strides go through shared memory (one barrier each).
+// Bitonic sort of n_pow2 <= EPT * kSelThreads entries of v (padding entries sort last), all
+// threads.  Thread t holds entries EPT t .. EPT t + EPT - 1 in registers: pairs closer than
+// EPT entries are exchanged in registers, pairs up to 16 EPT apart through warp shuffles,
+// and only the wider strides go through shared memory (one barrier each).
 template <bool kByFrame>
 __device__ __forceinline__ bool before(const Cand& x, const Cand& y) {
   return kByFrame ? before_in_frame(x, y) : before_in_score(x, y);
@@ -485,22 +490,22 @@ __device__ __forceinline__ Cand shfl_cand(const Cand& c, int lane_mask) {
   o.frame = __shfl_xor_sync(0xffffffffu, c.frame, lane_mask);
   return o;
 }
-template <bool kByFrame>
+template <bool kByFrame, int EPT>
 __device__ void bitonic(Cand* v, int n_pow2) {
   const int tid = threadIdx.x;
-  const bool live = 4 * tid < n_pow2;                  // threads past the entries idle
-  Cand x[4];
+  const bool live = EPT * tid < n_pow2;                // threads past the entries idle
+  Cand x[EPT];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) x[k] = live ? v[4 * tid + k] : v[0];
+  for (int k = 0; k < EPT; ++k) x[k] = live ? v[EPT * tid + k] : v[0];
   for (int size = 2; size <= n_pow2; size <<= 1) {
     int stride = size >> 1;
-    if (stride >= 128) {                               // wide strides: shared memory
+    if (stride >= 32 * EPT) {                          // wide strides: shared memory
       if (live) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) v[4 * tid + k] = x[k];
+        for (int k = 0; k < EPT; ++k) v[EPT * tid + k] = x[k];
       }
       __syncthreads();
-      for (; stride >= 128; stride >>= 1) {
+      for (; stride >= 32 * EPT; stride >>= 1) {
         for (int t = tid; t < (n_pow2 >> 1); t += blockDim.x) {
           const int i = ((t & ~(stride - 1)) << 1) | (t & (stride - 1));
           const int j = i + stride;
@@ -515,15 +520,15 @@ __device__ void bitonic(Cand* v, int n_pow2) {
       }
       if (live) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) x[k] = v[4 * tid + k];
+        for (int k = 0; k < EPT; ++k) x[k] = v[EPT * tid + k];
       }
       __syncthreads();
     }
-    for (; stride >= 4; stride >>= 1) {                // within the warp: shuffles
+    for (; stride >= EPT; stride >>= 1) {              // within the warp: shuffles
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int e = 4 * tid + k;
-        const Cand o = shfl_cand(x[k], stride >> 2);
+      for (int k = 0; k < EPT; ++k) {
+        const int e = EPT * tid + k;
+        const Cand o = shfl_cand(x[k], stride / EPT);
         const bool lower = (e & stride) == 0, up = (e & size) == 0;
         const bool mine_first = before<kByFrame>(x[k], o);
         // the lower entry keeps the first of the pair (descending runs: the last)
@@ -531,7 +536,7 @@ __device__ void bitonic(Cand* v, int n_pow2) {
         if (live && !keep_mine) x[k] = o;
       }
     }
-    // within the thread: strides 2 and 1
+    // within the thread: the strides below EPT
     auto cx = [&](Cand& a, Cand& b, int e) {
       const bool up = (e & size) == 0;
       if (up ? before<kByFrame>(b, a) : before<kByFrame>(a, b)) {
@@ -540,16 +545,18 @@ __device__ void bitonic(Cand* v, int n_pow2) {
         b = t;
       }
     };
-    if (size >= 4) {
-      cx(x[0], x[2], 4 * tid);
-      cx(x[1], x[3], 4 * tid + 1);
+#pragma unroll
+    for (int s = EPT / 2; s >= 1; s >>= 1) {
+      if (s < size) {
+#pragma unroll
+        for (int k = 0; k < EPT; ++k)
+          if ((k & s) == 0) cx(x[k], x[k + s], EPT * tid + k);
+      }
     }
-    cx(x[0], x[1], 4 * tid);
-    cx(x[2], x[3], 4 * tid + 2);
   }
   if (live) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) v[4 * tid + k] = x[k];
+    for (int k = 0; k < EPT; ++k) v[EPT * tid + k] = x[k];
   }
   __syncthreads();
 }
@@ -585,6 +592,8 @@ __global__ void __launch_bounds__(kSelThreads) memory_select_kernel(const Select
   __shared__ int red[32];
   __shared__ uint32_t kbits[KV_MEMORY_MAX_CANDIDATES / 32];
   __shared__ int wpre[KV_MEMORY_MAX_CANDIDATES / 32];
+  __shared__ int hist[256];
+  __shared__ int sel[3];
   const int tid = threadIdx.x;
   const int n = a.n_mem + a.n_fifo;
   int n_pow2 = 4;                                    // at least one thread's four entries
@@ -623,7 +632,10 @@ __global__ void __launch_bounds__(kSelThreads) memory_select_kernel(const Select
     v[i] = c;
   }
   __syncthreads();
-  bitonic<true>(v, n_pow2);
+  if (n_pow2 > 4 * kSelThreads)                      // up to 8,192 entries: eight per thread
+    bitonic<true, 8>(v, n_pow2);
+  else
+    bitonic<true, 4>(v, n_pow2);
   // rank within the frame: the k-th entry of a frame run scores quality * gamma^k, gamma^k
   // formed by repeated multiplication.  Each thread takes a contiguous chunk; the run in
   // effect at its first entry comes from a max-scan of the chunks' last run starts.
@@ -652,14 +664,93 @@ __global__ void __launch_bounds__(kSelThreads) memory_select_kernel(const Select
     for (int i = lo; i < hi; ++i) v[i].q = qs[i - lo];
   }
   __syncthreads();
-  bitonic<false>(v, n_pow2);
-  // the best min(n, M), listed in ascending candidate index: a bitmap of the kept indices
-  // and a prefix count over it
+  // the best min(n, M) by (score desc, position asc, index asc): a radix select over that
+  // composite key (unique, since indices are), most significant byte first, marks them in
+  // a bitmap of candidate indices without sorting by score
   const int m = n < a.M ? n : a.M;
   const int n_words = (n + 31) >> 5;
   for (int w = tid; w < n_words; w += blockDim.x) kbits[w] = 0u;
-  __syncthreads();
-  for (int i = tid; i < m; i += blockDim.x) atomicOr(&kbits[v[i].idx >> 5], 1u << (v[i].idx & 31));
+  {
+    constexpr int kPer = KV_MEMORY_MAX_CANDIDATES / kSelThreads;   // entries i = tid + k * 1024
+    uint32_t key[kPer][3];
+    int state[kPer];                                 // 0 undecided, 1 kept, 2 dropped
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int i = tid + k * kSelThreads;
+      state[k] = i < n ? 0 : 2;
+      if (i < n) {
+        uint32_t b = __float_as_uint(v[i].q);
+        if (b == 0x80000000u) b = 0u;                // -0 ranks as +0
+        const uint32_t asc = (b & 0x80000000u) ? ~b : (b | 0x80000000u);   // float order
+        key[k][0] = ~asc;                            // higher score first
+        key[k][1] = (uint32_t)v[i].pos ^ 0x80000000u;   // lower position first
+        key[k][2] = (uint32_t)v[i].idx;              // lower index first (< 2^13)
+      } else {
+        key[k][0] = key[k][1] = key[k][2] = 0u;
+      }
+    }
+    int r = m;                                       // still to keep among the undecided
+    for (int pass = 0; pass < 10; ++pass) {
+      const int word = pass < 4 ? 0 : (pass < 8 ? 1 : 2);
+      const int shift = pass < 8 ? 24 - 8 * (pass & 3) : 8 - 8 * (pass - 8);
+      for (int d = tid; d < 256; d += kSelThreads) hist[d] = 0;
+      __syncthreads();
+      // the word by constant indices (a runtime index would put key[] in local memory)
+      auto digit = [&](int k) -> int {
+        const uint32_t w = word == 0 ? key[k][0] : (word == 1 ? key[k][1] : key[k][2]);
+        return (int)((w >> shift) & 0xFFu);
+      };
+#pragma unroll
+      for (int k = 0; k < kPer; ++k)
+        if (state[k] == 0) atomicAdd(&hist[digit(k)], 1);
+      __syncthreads();
+      if (tid < 32) {                                // the digit where the r-th key falls
+        int c8[8], run = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          c8[e] = hist[8 * tid + e];
+          run += c8[e];
+        }
+        int incl = run;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (tid >= o) incl += y;
+        }
+        int below = incl - run;                      // keys in the digits under 8 tid
+        if (below < r && r <= incl) {                // exactly one lane
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (below < r && r <= below + c8[e]) {
+              sel[0] = 8 * tid + e;
+              sel[1] = below;
+              sel[2] = c8[e];
+            }
+            below += c8[e];
+          }
+        }
+      }
+      __syncthreads();
+      const int dsel = sel[0], below = sel[1], cnt = sel[2];
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        if (state[k] != 0) continue;
+        const int d = digit(k);
+        state[k] = d < dsel ? 1 : (d > dsel ? 2 : 0);
+      }
+      r -= below;
+      __syncthreads();                               // sel and hist are reused
+      if (cnt == r) break;                           // every key left in that digit is kept
+    }
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int i = tid + k * kSelThreads;
+      if (i < n && state[k] != 2) {                  // kept, or left undecided in a full digit
+        state[k] = 1;
+        atomicOr(&kbits[v[i].idx >> 5], 1u << (v[i].idx & 31));
+      }
+    }
+  }
   __syncthreads();
   if (tid < 32) {                                    // exclusive prefix of the words' counts
     const int per_w = (n_words + 31) >> 5;
@@ -684,8 +775,9 @@ __global__ void __launch_bounds__(kSelThreads) memory_select_kernel(const Select
     }
   }
   __syncthreads();
-  for (int i = tid; i < m; i += blockDim.x) {
+  for (int i = tid; i < n; i += blockDim.x) {
     const int idx = v[i].idx;
+    if (!(kbits[idx >> 5] & (1u << (idx & 31)))) continue;
     const int r = wpre[idx >> 5] + __popc(kbits[idx >> 5] & ((1u << (idx & 31)) - 1u));
     a.kept[r] = idx;
   }

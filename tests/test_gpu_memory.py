@@ -174,3 +174,70 @@ def test_key_mass_multi_sets_match_single_calls():
         assert torch.isfinite(one).all()
         assert torch.equal(one, m), (f, c)
         assert torch.equal(one, p), (f, c, (one - p).abs().max().item())
+
+
+def _select_case(orc, H, C_mem, n_mem_fill, C_fifo, n_fifo, M, frame_len, masses, positions,
+                 seed):
+    """One kv_memory_select call on engineered masses and slot positions; the kept list
+    must equal the oracle's rule applied to the GPU's binary32 qualities."""
+    D = 128
+    fifo = kv.KvRing(C_fifo, H, D, -(1 << 20), 1 << 20)
+    mem = kv.KvRing(C_mem, H, D, -(1 << 20), 1 << 20, rope_table=fifo.rope_table) if C_mem else None
+    for ring, fill in ((mem, n_mem_fill), (fifo, C_fifo)):
+        if ring is None:
+            continue
+        done = 0
+        while done < fill:
+            n = min(256, fill - done)
+            k, v = (inputs.draw(inputs.seed_of(seed, done, t), (n, H, D), "normal", 1.0, "bf16")
+                    for t in (1, 2))
+            kv.kv_ring_write(ring, to_dev(k), to_dev(v), commit=True)
+            done += n
+    n_mem = mem.n_valid if mem is not None else 0
+    mem_first = (mem.s.write_slot + mem.s.pending - n_mem) % C_mem if mem is not None else 0
+    first = (fifo.s.write_slot + 7) % C_fifo
+    n = n_mem + n_fifo
+    pos_mem, pos_fifo = positions[:n_mem], positions[n_mem:n]
+    if mem is not None:
+        mem.slot_pos[(mem_first + torch.arange(n_mem)) % C_mem] = torch.as_tensor(
+            pos_mem, dtype=torch.int32, device="cuda")
+    fifo.slot_pos[(first + torch.arange(n_fifo)) % C_fifo] = torch.as_tensor(
+        pos_fifo, dtype=torch.int32, device="cuda")
+    mm = torch.as_tensor(masses[:, :n_mem], dtype=torch.float32, device="cuda").contiguous()
+    mf = torch.as_tensor(masses[:, n_mem:n], dtype=torch.float32, device="cuda").contiguous()
+    dst = kv.KvRing(max(M, 1), H, D, -(1 << 20), 1 << 20, rope_table=fifo.rope_table)
+    kept = kv.kv_memory_select(mem, mm if n_mem else None, fifo, mf, first, n_fifo, M,
+                               frame_len, dst)
+    torch.cuda.synchronize()
+    qual = np.zeros(n, np.float32)
+    for h in range(H):                                   # heads in order, binary32
+        qual = qual + masses[h, :n].astype(np.float32)
+    pos = np.asarray(positions[:n], np.int64)
+    want = orc.memory_select(qual.astype(np.float64), np.floor_divide(pos, frame_len), pos, M,
+                             0.5)
+    assert kept.cpu().numpy().tolist() == want.tolist()
+    assert dst.n_valid == len(want)
+
+
+@pytest.mark.parametrize("case", ["ties_max", "all_kept", "one_kept", "zeros", "fifo_only"])
+def test_memory_select_ties_and_edges(orc, case):
+    """Selection on engineered candidates: qualities from a few small integers (most
+    scores tie, so position and then index decide), repeated and negative positions, the
+    largest candidate count (8,192), budgets of all and of one, all-zero masses, and no
+    memory ring."""
+    rng = np.random.default_rng(71)
+    H = 2
+    if case == "fifo_only":
+        C_mem, n_mem_fill, C_fifo, n_fifo, M = 0, 0, 300, 5, 3
+    else:
+        C_mem, n_mem_fill, C_fifo, n_fifo = 3000, 3000, 5200, 5192
+        M = {"ties_max": 4000, "all_kept": 8192, "one_kept": 1, "zeros": 100}[case]
+    n = n_mem_fill + n_fifo
+    masses = rng.integers(0, 4, size=(H, n)).astype(np.float32) * 0.25
+    if case == "zeros":
+        masses[:] = 0.0
+    # spread positions, plus about 50 candidates at one position (one deep frame: ranks up
+    # to ~55, so quality * 2^-rank stays a normal binary32, as exact as the oracle's fp64)
+    positions = rng.integers(-200000, 200000, size=n)
+    positions[::160] = positions[0]
+    _select_case(orc, H, C_mem, n_mem_fill, C_fifo, n_fifo, M, 64, masses, positions, 72)
