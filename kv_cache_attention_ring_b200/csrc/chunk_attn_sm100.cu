@@ -356,6 +356,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.y;
   const int q0 = blockIdx.x * BM;
+  // a CTA with at most 128 rows (few queries, a short last block) leaves query tile 1
+  // out: none of its MMAs, its softmax warps idle until the epilogue
+  const bool one_tile = a.n_rows - q0 <= BM / 2;
   const int C = a.C;
   const int newest = (int)a.newest_slot, n_valid = (int)a.n_valid;
 
@@ -401,7 +404,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bars.vempty(s), kPv8 ? 1 : kConvThreads);  // released by the MMAs (kPv8)
     }
     for (int s = 0; s < NB; ++s) { mbar_init(bars.vhfull(s), kConvThreads); mbar_init(bars.vhempty(s), 1); }
-    for (int s = 0; s < NI; ++s) { mbar_init(bars.ifull(s), 32); mbar_init(bars.iempty(s), 256); }
+    for (int s = 0; s < NI; ++s) {
+      mbar_init(bars.ifull(s), 32);
+      mbar_init(bars.iempty(s), one_tile ? 128 : 256);   // the softmax threads that run
+    }
     for (int g = 0; g < 2; ++g) {
       mbar_init(bars.sfull(g, 0), 1);
       mbar_init(bars.sfull(g, 1), 1);
@@ -656,14 +662,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = wait_w(bars.kfull(jj % NK), (jj / NK) & 1))) break;
         tc_fence_after();
         issue_s(0, jj);
-        issue_s(1, jj);
-        el_commit(bars.kempty(jj % NK));           // both tiles have read K(jj)
+        if (!one_tile) issue_s(1, jj);
+        el_commit(bars.kempty(jj % NK));           // every query tile has read K(jj)
       }
       // lockstep: per key tile j, query tile 0 then query tile 1, blocking waits
+      const int last_g = one_tile ? 0 : 1;
       for (int j = 0; ok && j < n_mine; ++j) {
         const bool more = j + 2 < n_mine;
 #pragma unroll
         for (int gg = 0; gg < 2; ++gg) {
+          if (gg > last_g) break;
           ok = wait_w(bars.pfull(gg, j & 1), (j >> 1) & 1) &&
                (kPv8 ? wait_w(bars.vready(j % NV), (j / NV) & 1)
                      : wait_w(bars.vhfull(j % NB), (j / NB) & 1)) &&
@@ -671,10 +679,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           tc_fence_after();
           issue_pv(gg, j);
-          if (gg == 1) el_commit(kPv8 ? bars.vempty(j % NV) : bars.vhempty(j % NB));
+          if (gg == last_g) el_commit(kPv8 ? bars.vempty(j % NV) : bars.vhempty(j % NB));
           if (more) {
             issue_s(gg, j + 2);
-            if (gg == 1) el_commit(bars.kempty((j + 2) % NK));
+            if (gg == last_g) el_commit(bars.kempty((j + 2) % NK));
           }
         }
       }
@@ -745,7 +753,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t r2 = f2_pack(rowmul, rowmul);
     float m_run = -INFINITY, l_run = 0.f;
     int j = 0;
-    for (; j < n_mine; ++j) {
+    const int n_soft = (g == 1 && one_tile) ? 0 : n_mine;    // tile 1 left out: no rows
+    for (; j < n_soft; ++j) {
       const int si = j % NI, buf = j & 1;
       const uint32_t t_s = tmem + lane_base + 128 * g + 64 * buf;   // S_g(j) / P_g(j)
       bool ok = wait(bars.sfull(g, buf), (j >> 1) & 1) && wait(bars.ifull(si), (j / NI) & 1);
