@@ -467,21 +467,11 @@ __device__ __forceinline__ bool before_in_frame(const Cand& x, const Cand& y) {
   if (x.pos != y.pos) return x.pos < y.pos;
   return x.idx < y.idx;
 }
-// (score desc, position asc, index asc)
-__device__ __forceinline__ bool before_in_score(const Cand& x, const Cand& y) {
-  if (x.q != y.q) return x.q > y.q;
-  if (x.pos != y.pos) return x.pos < y.pos;
-  return x.idx < y.idx;
-}
 
 // Bitonic sort of n_pow2 <= EPT * kSelThreads entries of v (padding entries sort last), all
 // threads.  Thread t holds entries EPT t .. EPT t + EPT - 1 in registers: pairs closer than
 // EPT entries are exchanged in registers, pairs up to 16 EPT apart through warp shuffles,
 // and only the wider strides go through shared memory (one barrier each).
-template <bool kByFrame>
-__device__ __forceinline__ bool before(const Cand& x, const Cand& y) {
-  return kByFrame ? before_in_frame(x, y) : before_in_score(x, y);
-}
 __device__ __forceinline__ Cand shfl_cand(const Cand& c, int lane_mask) {
   Cand o;
   o.q = __shfl_xor_sync(0xffffffffu, c.q, lane_mask);
@@ -490,7 +480,7 @@ __device__ __forceinline__ Cand shfl_cand(const Cand& c, int lane_mask) {
   o.frame = __shfl_xor_sync(0xffffffffu, c.frame, lane_mask);
   return o;
 }
-template <bool kByFrame, int EPT>
+template <int EPT>
 __device__ void bitonic(Cand* v, int n_pow2) {
   const int tid = threadIdx.x;
   const bool live = EPT * tid < n_pow2;                // threads past the entries idle
@@ -511,7 +501,7 @@ __device__ void bitonic(Cand* v, int n_pow2) {
           const int j = i + stride;
           const Cand a = v[i], b = v[j];
           const bool up = (i & size) == 0;
-          if (up ? before<kByFrame>(b, a) : before<kByFrame>(a, b)) {
+          if (up ? before_in_frame(b, a) : before_in_frame(a, b)) {
             v[i] = b;
             v[j] = a;
           }
@@ -530,7 +520,7 @@ __device__ void bitonic(Cand* v, int n_pow2) {
         const int e = EPT * tid + k;
         const Cand o = shfl_cand(x[k], stride / EPT);
         const bool lower = (e & stride) == 0, up = (e & size) == 0;
-        const bool mine_first = before<kByFrame>(x[k], o);
+        const bool mine_first = before_in_frame(x[k], o);
         // the lower entry keeps the first of the pair (descending runs: the last)
         const bool keep_mine = (lower == up) ? mine_first : !mine_first;
         if (live && !keep_mine) x[k] = o;
@@ -539,7 +529,7 @@ __device__ void bitonic(Cand* v, int n_pow2) {
     // within the thread: the strides below EPT
     auto cx = [&](Cand& a, Cand& b, int e) {
       const bool up = (e & size) == 0;
-      if (up ? before<kByFrame>(b, a) : before<kByFrame>(a, b)) {
+      if (up ? before_in_frame(b, a) : before_in_frame(a, b)) {
         const Cand t = a;
         a = b;
         b = t;
@@ -633,9 +623,9 @@ __global__ void __launch_bounds__(kSelThreads) memory_select_kernel(const Select
   }
   __syncthreads();
   if (n_pow2 > 4 * kSelThreads)                      // up to 8,192 entries: eight per thread
-    bitonic<true, 8>(v, n_pow2);
+    bitonic<8>(v, n_pow2);
   else
-    bitonic<true, 4>(v, n_pow2);
+    bitonic<4>(v, n_pow2);
   // rank within the frame: the k-th entry of a frame run scores quality * gamma^k, gamma^k
   // formed by repeated multiplication.  Each thread takes a contiguous chunk; the run in
   // effect at its first entry comes from a max-scan of the chunks' last run starts.
