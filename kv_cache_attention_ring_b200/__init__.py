@@ -444,6 +444,12 @@ def chunk_key_mass_multi(main: KvRing, cands, q, q_pos0: int, lse, slot_firsts, 
     if masses is None:
         masses = [torch.empty((main.H, int(c)), dtype=torch.float32, device=q.device)
                   for c in n_cands]
+    assert len(masses) == n
+    for m, c in zip(masses, n_cands):
+        assert m.is_cuda and m.dtype == torch.float32 and m.is_contiguous()
+        assert m.numel() >= main.H * int(c)
+    if workspace is not None:
+        assert workspace.is_cuda and workspace.is_contiguous()
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(main.D)
     b = kv_cache_bias_t(float(cache_bias))
