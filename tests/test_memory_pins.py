@@ -88,6 +88,22 @@ def test_selection_equals_independent_greedy(orc, seed):
         assert got.tolist() == _greedy(quality, frame, pos, M, gamma), (seed, gamma)
 
 
+@pytest.mark.parametrize("seed", range(4))
+def test_selection_ties_on_quality_and_position(orc, seed):
+    """Quality from four values and positions from a narrow range around zero: most
+    candidates tie on quality, many share a position (the candidate index decides), and
+    negative positions fall in negative frames (floor division)."""
+    rng = np.random.default_rng(100 + seed)
+    n = int(rng.integers(2, 250))
+    quality = rng.choice([0.0, 0.25, 0.5, 1.0], size=n)
+    pos = rng.integers(-60, 60, size=n)
+    frame = np.floor_divide(pos, 24)
+    M = int(rng.integers(1, n + 3))
+    for gamma in (0.5, 0.25, 1.0):
+        got = orc.memory_select(quality, frame, pos, M, gamma)
+        assert got.tolist() == _greedy(quality, frame, pos, M, gamma), (seed, gamma)
+
+
 def test_selection_limits(orc):
     rng = np.random.default_rng(11)
     quality = rng.random(200)
